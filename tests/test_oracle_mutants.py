@@ -1,0 +1,65 @@
+"""Planted mistakes in a copy of the oracle must each fail a pin (CPU only).
+
+Each mutant is oracle.c with one plausible slip applied as a text substitution,
+compiled to a temporary library and bound in place of the real one while a
+battery of the pin tests runs.  A mutant that passes every pin would mean the
+pins leave that part of the oracle unchecked.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+MUTANTS = {
+    "tie_break_flipped": ("return (a->e > b->e) - (a->e < b->e);", "return (a->e < b->e) - (a->e > b->e);"),
+    "renorm_dropped": ("double inv = sum_sel > 1e-20 ? 1.0 / sum_sel : 1.0 / (double)K;", "double inv = 1.0;"),
+    "gelu_cubic_coefficient": ("0.044715 * g * g * g", "0.44715 * g * g * g"),
+    "silu_sign": ("return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));"),
+    "down_row_base": ("load_row(Wd, dtype, drow0 + j, F, row);", "load_row(Wd, dtype, row0 + j, F, row);"),
+    "shared_gate_ignored": ("for (int64_t j = 0; j < H; ++j) o[j] += s * y[j];",
+                            "for (int64_t j = 0; j < H; ++j) o[j] += y[j];"),
+    "router_bias_dropped": ("s += (double)w->bias[e];", "s += 0.0;"),
+    "permutation_unstable": ("int32_t pos = offsets[e] + fill[e]++;", "int32_t pos = offsets[e + 1] - 1 - fill[e]++;"),
+    "q8_unsigned": ("d * (double)(int8_t)p[b * 34 + 2 + j]", "d * (double)(uint8_t)p[b * 34 + 2 + j]"),
+    "slot_weight_index": ("o[j] += wk[k] * y[j];", "o[j] += wk[0] * y[j];"),
+    "up_reads_gate": ("load_row(Wu, dtype, row0 + i, Hin, row);", "load_row(Wg, dtype, row0 + i, Hin, row);"),
+    "fp16_exponent_bias": ("ldexp(1024.0 + man, ex - 25)", "ldexp(1024.0 + man, ex - 24)"),
+}
+
+BATTERY = [
+    pins.test_silu_known_values, pins.test_gelu_asymptotics, pins.test_topk_worked_example,
+    lambda g: pins.test_selection_matches_brute_force_sort(16, 5), lambda g: pins.test_renormalised_weights_sum_to_one(),
+    lambda g: pins.test_weights_closed_form_renorm_and_not(), lambda g: pins.test_router_logits_and_bias(),
+    lambda g: pins.test_permutation_properties(50, 8, 16), lambda g: pins.test_q8_0_and_bf16_loads(),
+    lambda g: pins.test_fp16_decode_all_finite_patterns(),
+    lambda g: pins.test_dense_special_case("silu", "f32"),
+    lambda g: pins.test_layer_matches_numpy_restatement(48, True, True),
+    pins.test_shared_gate_linearity,
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path, golden_dir):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.c")).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation anchor not found once: {old}"
+    path = tmp_path / "mut.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", str(so), str(path), "-lm"])
+    saved = oracle._lib_handle
+    oracle._lib_handle = oracle.bind(ctypes.CDLL(str(so)))
+    caught = []
+    try:
+        for check in BATTERY:
+            try:
+                check(golden_dir)
+            except AssertionError:
+                caught.append(getattr(check, "__name__", "lambda"))
+    finally:
+        oracle._lib_handle = saved
+    assert caught, f"mutant {name} passed every pin"

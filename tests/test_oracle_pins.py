@@ -1,0 +1,305 @@
+"""Pins of the f64 oracle to facts outside itself (CPU only).
+
+Each pin comes from the pages (worked values, printed tolerances), a closed form,
+brute force on tiny inputs, an invariant, or a special case that reduces to a
+textbook formula.  Together they are chosen so that a plausible slip in the
+oracle (dropped term, flipped tie-break, transposed weight, wrong constant,
+missing renormalisation, wrong shared-gate scale, wrong dequantisation) fails
+at least one of them; ``test_oracle_mutants.py`` checks exactly that by
+planting such slips in a copy of the oracle.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests._helpers import ACTS, numpy_layer, widen
+
+
+def _tiny(T=5, H=64, E=6, I=96, K=2, act="silu", act_dtype="f32", w_dtype="f32", router_dtype="f32",
+          shared_I=0, gated=False, bias=None, seed=7, renorm=True, router_std=0.5):
+    spec = workloads.Spec(T=T, H=H, E=E, I=I, K=K, act=act, act_dtype=act_dtype, w_dtype=w_dtype,
+                          router_dtype=router_dtype, shared_I=shared_I, shared_gated=gated, renormalize=renorm,
+                          router_std=router_std)
+    wl = workloads.make(spec, seed=seed)
+    if bias is not None:
+        wl.router_bias = np.asarray(bias, np.float32)
+    return oracle.from_workload(wl)
+
+
+# ---------------------------------------------------------------- activations
+
+def test_silu_known_values(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "silu_known_values.json")))
+    gate = np.array(g["gate"])
+    up = np.array(g["up"])
+    got = oracle.act("silu", gate) * up
+    printed = g["silu_of_gate_printed"]
+    for i, (gv, uv) in enumerate(zip(gate, up)):
+        key = repr(float(gv))
+        if key in printed:
+            assert abs(got[i] - printed[key] * uv) < g["tolerance"] * max(1.0, abs(uv))
+    # the fourth element is the page's own formula 2/(1+e^-2) * 0.5
+    assert abs(got[3] - (2.0 / (1.0 + math.exp(-2.0))) * 0.5) < 1e-15
+
+
+def test_silu_closed_form_and_symmetry():
+    g = np.linspace(-20, 20, 4001)
+    s = oracle.act("silu", g)
+    assert np.allclose(s, g / (1.0 + np.exp(-g)), rtol=0, atol=1e-15)
+    # silu(g) - silu(-g) = g  (sigma(g) + sigma(-g) = 1)
+    assert np.allclose(s - oracle.act("silu", -g), g, atol=1e-12)
+
+
+def test_gelu_asymptotics(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "gelu_asymptotics.json")))
+    for pt in g["points"]:
+        assert abs(oracle.act("gelu_tanh", pt["g"])[0] - pt["gelu"]) <= pt["tol"]
+    h = 1e-5
+    fd = (oracle.act("gelu_tanh", h)[0] - oracle.act("gelu_tanh", -h)[0]) / (2 * h)
+    assert abs(fd - g["derivative_at_zero"]) < g["derivative_tol"]
+    # the page's literal constant differs from sqrt(2/pi) by ~3e-11: same function to 1e-9
+    c = g["page_constant_sqrt_2_over_pi"]
+    xs = np.linspace(-8, 8, 1601)
+    page = 0.5 * xs * (1.0 + np.tanh(c * (xs + 0.044715 * xs ** 3)))
+    assert np.max(np.abs(oracle.act("gelu_tanh", xs) - page)) < 1e-9
+
+
+def test_gelu_cubic_term_matters():
+    # gelu(g) - g*Phi_tanh(g) with the cubic term: at g=2 the tanh argument is sqrt(2/pi)*(2+0.35772)
+    v = oracle.act("gelu_tanh", 2.0)[0]
+    assert abs(v - 0.5 * 2.0 * (1 + math.tanh(math.sqrt(2 / math.pi) * (2.0 + 0.044715 * 8.0)))) < 1e-15
+
+
+# ---------------------------------------------------------------- routing
+
+def test_topk_worked_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "topk_worked_example.json")))
+    ids, w = oracle.select(np.array([g["logits"]]), g["top_k"], True)
+    assert ids[0, 0] == g["first_id"]
+    assert ids[0, 1] == 1  # lower index wins the three-way tie
+    assert abs(w.sum() - g["weight_sum"]) < g["weight_sum_tolerance"]
+    # closed form: renormalised over {0,1}: w0 = e^9/(e^9+1)
+    assert abs(w[0, 0] - math.exp(9) / (math.exp(9) + 1)) < 1e-15
+    assert w[0, 0] > 100 * w[0, 1]
+
+
+@pytest.mark.parametrize("E,K", [(1, 1), (2, 1), (4, 2), (7, 3), (12, 12), (16, 5), (64, 8), (256, 8)])
+def test_selection_matches_brute_force_sort(E, K):
+    rng = np.random.default_rng(E * 100 + K)
+    # coarse grid -> many exact ties, which is where a tie-break slip shows
+    l = np.round(rng.normal(size=(40, E)) * 2) / 2
+    ids, _ = oracle.select(l, K, True)
+    for t in range(l.shape[0]):
+        ref = sorted(range(E), key=lambda e: (-l[t, e], e))[:K]
+        assert list(ids[t]) == ref
+
+
+def test_weights_closed_form_renorm_and_not():
+    rng = np.random.default_rng(3)
+    l = rng.normal(size=(30, 9)) * 3
+    for renorm in (True, False):
+        ids, w = oracle.select(l, 4, renorm)
+        for t in range(30):
+            den = sum(math.exp(v - l[t].max()) for v in l[t])
+            p = [math.exp(l[t, e] - l[t].max()) / den for e in ids[t]]
+            if renorm:
+                s = sum(p)
+                p = [v / s for v in p]
+            assert np.allclose(w[t], p, rtol=1e-14, atol=0)
+
+
+def test_renormalised_weights_sum_to_one():
+    rng = np.random.default_rng(11)
+    l = rng.normal(size=(200, 128)) * 4
+    _, w = oracle.select(l, 8, True)
+    assert np.max(np.abs(w.sum(1) - 1.0)) < 1e-12
+    # without renormalisation, K = E gives the full softmax, which also sums to 1
+    _, w2 = oracle.select(l[:, :16], 16, False)
+    assert np.max(np.abs(w2.sum(1) - 1.0)) < 1e-12
+
+
+def test_softmax_shift_invariance_and_extremes():
+    l = np.array([[1000.0, 999.0, -1000.0, 0.0]])
+    ids, w = oracle.select(l, 2, True)
+    assert list(ids[0]) == [0, 1]
+    assert abs(w[0, 0] - 1 / (1 + math.exp(-1))) < 1e-15
+    ids2, w2 = oracle.select(l - 12345.0, 2, True)
+    assert (ids2 == ids).all() and np.allclose(w2, w, rtol=1e-13)
+
+
+def test_single_expert_weight_is_exactly_one():
+    # ferrox-models decoder.rs, is_dense_layer: top-1 of one expert has weight exactly 1.0
+    l = np.random.default_rng(1).normal(size=(10, 1))
+    ids, w = oracle.select(l, 1, True)
+    assert (ids == 0).all() and (w == 1.0).all()
+    ids, w = oracle.select(l, 1, False)
+    assert (w == 1.0).all()
+
+
+def test_router_logits_and_bias():
+    L = _tiny(T=6, E=5, bias=[0.0, 0.0, 0.0, 0.0, 50.0])
+    lg, am = oracle.logits(L)
+    x = widen(L.x, "f32")
+    Wr = widen(L.router, "f32")
+    assert np.allclose(lg, x @ Wr.T + np.array(L.bias, np.float64), rtol=1e-12, atol=1e-12)
+    assert np.allclose(am, (np.abs(x[:, None, :] * Wr[None]).sum(-1) + np.abs(L.bias)).max(1), rtol=1e-12)
+    r = oracle.layer(L)
+    assert (r["ids"][:, 0] == 4).all()   # the +50 bias wins every token's first slot
+
+
+# ---------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("T,K,E", [(1, 1, 1), (3, 2, 4), (50, 8, 16), (200, 8, 256), (97, 3, 5)])
+def test_permutation_properties(T, K, E):
+    rng = np.random.default_rng(T * K + E)
+    # K distinct experts per token, skewed towards low ids
+    ids = np.stack([rng.choice(E, size=K, replace=False, p=None) for _ in range(T)]).astype(np.int32)
+    counts, offsets, sp, pp = oracle.permute(ids, E)
+    P = T * K
+    assert counts.sum() == P
+    assert offsets[0] == 0 and offsets[-1] == P and (np.diff(offsets) == counts).all()
+    assert sorted(sp.tolist()) == list(range(P))
+    assert (sp[pp] == np.arange(P)).all()
+    flat = ids.reshape(-1)
+    assert sp.tolist() == sorted(range(P), key=lambda p: (flat[p], p))   # stable counting sort
+    for e in range(E):
+        assert (flat[sp[offsets[e]:offsets[e + 1]]] == e).all()
+
+
+def test_permutation_rejects_out_of_range():
+    with pytest.raises(ValueError):
+        oracle.permute(np.array([[0, 5]], np.int32), 4)
+
+
+# ---------------------------------------------------------------- formats
+
+def test_fp16_decode_all_finite_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    fin = np.isfinite(ref)
+    got = np.array([oracle.fp16_to_double(int(b)) for b in bits[fin][::7]])
+    assert np.array_equal(got, ref[fin][::7])
+    for b in (0x0001, 0x03FF, 0x0400, 0x3C00, 0x7BFF, 0x8001, 0xFBFF):
+        assert oracle.fp16_to_double(b) == float(np.array([b], np.uint16).view(np.float16)[0])
+
+
+def test_q8_0_and_bf16_loads():
+    blk = workloads.q8_0_blocks(5, 1, (3, 64))
+    got = oracle.load_rows(blk, "q8_0", 64)
+    assert np.array_equal(got, widen(blk, "q8_0"))
+    # fp16 scale times int8 fits exactly in f32 (11 + 8 significant bits)
+    assert np.array_equal(got.astype(np.float32).astype(np.float64), got)
+    b = workloads.normal(5, 2, (4, 32), 1.0, "bf16")
+    assert np.array_equal(oracle.load_rows(b, "bf16", 32), widen(b, "bf16"))
+
+
+# ---------------------------------------------------------------- the layer
+
+@pytest.mark.parametrize("act", ["silu", "gelu_tanh"])
+@pytest.mark.parametrize("dt", ["f32", "bf16", "q8_0"])
+def test_dense_special_case(act, dt):
+    """E=1, K=1, no shared expert: the weight is exactly 1 and the layer is a dense gated FFN."""
+    L = _tiny(T=4, H=64, E=1, I=96, K=1, act=act, w_dtype=dt, act_dtype="bf16" if dt == "bf16" else "f32",
+              router_dtype="bf16" if dt == "bf16" else "f32")
+    r = oracle.layer(L)
+    assert (r["w"] == 1.0).all() and (r["ids"] == 0).all()
+    x = widen(L.x, L.act_dtype)
+    g = widen(L.gate, dt).reshape(96, 64)
+    u = widen(L.up, dt).reshape(96, 64)
+    d = widen(L.down, dt).reshape(64, 96)
+    dense = (ACTS[act](x @ g.T) * (x @ u.T)) @ d.T
+    assert np.max(np.abs(r["out"] - dense)) <= 1e-12 * np.max(np.abs(dense))
+
+
+@pytest.mark.parametrize("shared,gated", [(0, False), (48, True), (48, False)])
+@pytest.mark.parametrize("renorm", [True, False])
+def test_layer_matches_numpy_restatement(shared, gated, renorm):
+    L = _tiny(T=7, H=64, E=6, I=32, K=3, shared_I=shared, gated=gated, renorm=renorm, act="gelu_tanh")
+    r = oracle.layer(L)
+    ref = numpy_layer(L)
+    assert (r["ids"] == ref["ids"]).all()
+    assert np.allclose(r["w"], ref["w"], rtol=1e-13, atol=0)
+    assert np.allclose(r["logits"], ref["logits"], rtol=1e-12, atol=1e-12)
+    assert np.max(np.abs(r["out"] - ref["out"])) <= 1e-12 * np.max(np.abs(ref["out"]))
+
+
+def test_layer_bf16_and_q8_0_match_numpy_restatement():
+    for w_dtype, a_dtype in (("bf16", "bf16"), ("q8_0", "f32")):
+        L = _tiny(T=5, H=64, E=5, I=64, K=2, act_dtype=a_dtype, w_dtype=w_dtype, router_dtype=a_dtype,
+                  shared_I=32, gated=True)
+        r = oracle.layer(L)
+        ref = numpy_layer(L)
+        assert (r["ids"] == ref["ids"]).all()
+        assert np.max(np.abs(r["out"] - ref["out"])) <= 1e-12 * np.max(np.abs(ref["out"]))
+
+
+def test_token_order_invariance():
+    L = _tiny(T=9, E=8, K=3, shared_I=32, gated=True)
+    base = oracle.layer(L)["out"]
+    perm = np.random.default_rng(0).permutation(9)
+    L.x = np.ascontiguousarray(L.x[perm])
+    got = oracle.layer(L)["out"]
+    assert np.array_equal(got, base[perm])      # bit-exact: tokens are independent
+
+
+def test_token_subset_equals_full():
+    L = _tiny(T=9, E=8, K=3)
+    full = oracle.layer(L)
+    sub = oracle.layer(L, tokens=[8, 0, 3])
+    assert np.array_equal(sub["out"], full["out"][[8, 0, 3]])
+    assert np.array_equal(sub["ids"], full["ids"][[8, 0, 3]])
+
+
+def test_forced_selection_reproduces_own_selection():
+    L = _tiny(T=6, E=8, K=3)
+    full = oracle.layer(L)
+    forced = oracle.layer(L, force_ids=full["ids"])
+    assert np.array_equal(forced["out"], full["out"])
+
+
+def test_routed_sum_is_weighted_expert_sum():
+    """out[t] = sum_k w_k * expert(t, id_k), summed in k order (the combine)."""
+    L = _tiny(T=3, E=5, K=3)
+    r = oracle.layer(L)
+    for t in range(3):
+        acc = np.zeros(L.H)
+        for k in range(3):
+            acc += r["w"][t, k] * oracle.expert(L, t, int(r["ids"][t, k]))
+        assert np.array_equal(acc, r["out"][t])
+
+
+def test_shared_gate_linearity(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "shared_gate_linearity.json")))
+    L = _tiny(T=1, H=g["hidden"], E=g["experts"], K=g["top_k"], I=g["intermediate"],
+              shared_I=g["shared_intermediate"], gated=True)
+    L.H = g["hidden"]
+    outs = []
+    for v in g["gate_weight_values"]:
+        L.sh_gate_w = np.full(L.H, v, np.float32)
+        outs.append(oracle.layer(L)["out"][0])
+    mid, a, b = outs
+    assert np.max(np.abs(mid - 0.5 * (a + b))) < 1e-12 * np.max(np.abs(mid))
+    # with a saturating gate weight, off and on differ by exactly the ungated shared term
+    sat = []
+    for v in (-1e9, 1e9):
+        L.sh_gate_w = np.full(L.H, v, np.float32)
+        sat.append(oracle.layer(L)["out"][0])
+    a, b = sat
+    L.sh_gate_w = None
+    y_s, s = oracle.shared(L)
+    assert (s == 1.0).all()
+    assert np.max(np.abs(np.abs(a - b) - np.abs(y_s[0]))) < 1e-12 * np.max(np.abs(y_s))
+
+
+def test_ungated_shared_is_added_with_scale_one():
+    L = _tiny(T=4, E=4, K=2, shared_I=32, gated=False)
+    full = oracle.layer(L)["out"]
+    y_s, s = oracle.shared(L)
+    Ls = _tiny(T=4, E=4, K=2, shared_I=0)
+    routed = oracle.layer(Ls)["out"]
+    assert np.max(np.abs(full - (routed + y_s))) < 1e-13 * np.max(np.abs(full))
