@@ -1,0 +1,369 @@
+"""Benchmark of the MoE FFN layer on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one moe_layer call (router, top-K, permutation, expert GEMMs, shared
+expert, combine) over one batch of the workload, inputs resident in HBM.  The
+default workload is the batched prefill layer (T=512, H=2048, E=64, K=8,
+I=1024, SiLU, bf16).  Under torchrun (N > 1) every rank runs an independent
+replica of the layer on its own GPU (the layer does not shard); the time is
+the max over ranks and `value` counts the tokens of all ranks.
+
+--impl reference times the f64 CPU oracle on the host cores instead (rank 0
+only), on bounded token samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "MoE layer tokens/s at 1 B200; % of BF16 tensor peak (prefill) / HBM BW (decode)"
+UNIT = "tokens/s"
+DEFAULT_CONFIG = "prefill_bf16_t512"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ algorithmic work per kernel launch
+def algorithmic(spec, counts):
+    """Bytes (and flops) each kernel of one step must move at minimum, from the actual routing.
+
+    Weights are counted once per touched expert; activations read once and outputs written once."""
+    T, H, E, I, K, Is = spec.T, spec.H, spec.E, spec.I, spec.K, spec.shared_I
+    P = T * K
+    touched = int(np.count_nonzero(counts))
+    wb = {"f32": 4, "bf16": 2, "q8_0": 1 + 2.0 / 32}[spec.w_dtype]
+    ab = 4 if spec.act_dtype == "f32" else 2
+    rb = 4 if spec.router_dtype == "f32" else 2
+    tc = spec.act_dtype == "bf16" and spec.w_dtype == "bf16" and T > 64
+    hb = 2 if tc else 4
+    k = {}
+    k["expert_gate_up_gemm"] = k["stream_gate_up"] = dict(
+        bytes=touched * 2 * I * H * wb + P * H * ab + P * I * hb, flops=2.0 * P * 2 * I * H)
+    k["expert_down_gemm"] = k["stream_down"] = dict(
+        bytes=touched * H * I * wb + P * I * hb + P * H * 4 + P * 4, flops=2.0 * P * H * I)
+    k["router_gemm"] = k["router_logits"] = dict(bytes=E * H * rb + T * H * ab + T * E * 4, flops=2.0 * T * E * H)
+    k["router_topk"] = dict(bytes=T * E * 4 * (2 if spec.router_bias else 1) + P * 8, flops=0)
+    k["permute"] = dict(bytes=P * 4 * 3 + (2 * E + 1) * 4, flops=0)
+    k["gather_rows"] = dict(bytes=P * H * ab * 2 + P * 4, flops=0)
+    k["combine"] = dict(bytes=P * H * 4 + (T * H * 4 if Is else 0) + T * H * ab, flops=0)
+    if Is:
+        k["shared_gate_up_gemm"] = dict(bytes=2 * Is * H * wb + T * H * ab + T * Is * hb, flops=2.0 * T * 2 * Is * H)
+        k["shared_down_gemm"] = dict(bytes=Is * H * wb + T * Is * hb + T * H * 4, flops=2.0 * T * H * Is)
+    layer = dict(bytes=touched * 3 * I * H * wb + E * H * rb + (3 * Is * H * wb if Is else 0) + 2 * T * H * ab,
+                 flops=2.0 * (T * E * H + P * 3 * H * I + T * 3 * H * Is))
+    return k, layer, touched
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            self._stop.wait(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok and self._t:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ traffic from a committed ncu capture
+def _traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from profiles/traffic.json, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(f"{kernel}@{workload}")
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "mixture_experts_ffn_07_b200", "csrc", rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha"]:
+        return None
+    return rec["bytes_per_launch"]
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(spec, wl, budget_s: float, max_tokens=None):
+    """Oracle on host cores over a bounded token sample sized to ~budget_s seconds. Returns (tokens/s, info)."""
+    import oracle
+    L = oracle.from_workload(wl)
+    cores = oracle.threads()
+    n0 = max(1, min(spec.T, cores))
+    t0 = time.perf_counter()
+    oracle.layer(L, tokens=np.arange(n0))
+    dt = time.perf_counter() - t0
+    n = int(min(spec.T if max_tokens is None else max_tokens, max(n0, n0 * budget_s / max(dt, 1e-6))))
+    if n > n0:
+        tok = np.linspace(0, spec.T - 1, n).round().astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.layer(L, tokens=tok)
+        dt = time.perf_counter() - t0
+    else:
+        n = n0
+    return n / dt, dict(cores=cores, sample=f"{n} of {spec.T} tokens, full layer in f64 ({dt:.2f} s)", tokens=n,
+                        seconds=dt)
+
+
+def run_reference(args, spec):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    wl = workloads.make(spec)
+    import oracle
+    L = oracle.from_workload(wl)
+    cores = oracle.threads()
+    per_step = max(1, min(spec.T, cores))
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        oracle.layer(L, tokens=rng.integers(0, spec.T, per_step))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.layer(L, tokens=rng.integers(0, spec.T, per_step))
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
+                       "shared_I": spec.shared_I, "step_sample_tokens": per_step},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} random tokens of {spec.T} per step, full layer in f64"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, spec):
+    import torch
+    ws_n, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws_n > 1:
+        import datetime
+
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import mixture_experts_ffn_07_b200 as moe
+    from mixture_experts_ffn_07_b200 import host
+
+    wl = workloads.make(spec)
+    desc, w, x = host.upload(wl)
+    T, H = spec.T, spec.H
+    out = torch.empty((T, H), dtype=x.dtype, device="cuda")
+    wsb = torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    # routing once (outside timing) for the touched-expert count of the algorithmic bytes
+    _, ids, _, _ = host.run_route(desc, w, x)
+    counts = np.bincount(ids.cpu().numpy().reshape(-1), minlength=spec.E)
+    kern_alg, layer_alg, touched = algorithmic(spec, counts)
+
+    for _ in range(max(args.warmup, 3)):
+        moe.layer(desc, x, w, out, wsb)
+    torch.cuda.synchronize()
+    assert moe.last_device_status() == moe.MOE_OK
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    moe.trace_enable(True)
+    n_launch0 = moe.launch_count()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        moe.layer(desc, x, w, out, wsb)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    n_launch = moe.launch_count() - n_launch0
+    moe.trace_enable(False)
+    clocks.stop()
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    status = moe.last_device_status()
+    trace = moe.trace_read()
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = ws_n * T * args.steps / (ms / 1e3)
+
+    # per-kernel durations (CUDA events around each launch on the launching stream)
+    per = {}
+    for name, t in trace:
+        per.setdefault(name, []).append(t)
+    kernels = {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "total_ms": sum(v)} for n, v in per.items()}
+    tot = sum(k["total_ms"] for k in kernels.values()) or 1.0
+    for k in kernels.values():
+        k["share"] = k["total_ms"] / tot
+    dom = max(kernels, key=lambda n: kernels[n]["total_ms"]) if kernels else None
+
+    peaks, peak_src = _peaks()
+    roofline = None
+    if dom:
+        alg = kern_alg.get(dom, {"bytes": 0, "flops": 0})
+        avg_s = kernels[dom]["avg_ms"] / 1e3
+        tensor_bound = alg["flops"] / max(alg["bytes"], 1) > 1e3 * peaks["bf16_tflops"] / peaks["hbm_gbs"]
+        if tensor_bound:
+            achieved, peak, unit = alg["flops"] / avg_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        else:
+            achieved, peak, unit = alg["bytes"] / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        roofline = {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
+                    "frac": achieved / peak, "traffic": _traffic(dom, spec.name), "kernel": dom,
+                    "algorithmic_bytes_per_launch": alg["bytes"], "algorithmic_flops_per_launch": alg["flops"],
+                    "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if tensor_bound else 'hbm_gbs'})"}
+    layer_s = ms_step / 1e3
+    layer_roof = {"bytes": layer_alg["bytes"], "flops": layer_alg["flops"],
+                  "GB/s": layer_alg["bytes"] / layer_s / 1e9, "TFLOP/s": layer_alg["flops"] / layer_s / 1e12,
+                  "hbm_frac": layer_alg["bytes"] / layer_s / 1e9 / peaks["hbm_gbs"],
+                  "tensor_frac": layer_alg["flops"] / layer_s / 1e12 / peaks["bf16_tflops_sustained"],
+                  "touched_experts": touched}
+
+    # end to end through the public host-buffer call: H2D x, layer, D2H out every step
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    xd, od = torch.empty_like(x), torch.empty_like(x)
+    for _ in range(max(args.warmup, 3)):
+        moe.layer_host(desc, xh, w, oh, xd, od, wsb)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        moe.layer_host(desc, xh, w, oh, xd, od, wsb)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    io_bytes = T * H * x.element_size()
+
+    cpu = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        v, info = time_oracle(spec, wl, budget_s=args.cpu_budget)
+        cpu = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle", "sample": info["sample"]}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": spec.act_dtype if spec.w_dtype != "q8_0" else "q8_0xf32",
+            "data": "synthetic",
+            "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
+                       "act": spec.act, "shared_I": spec.shared_I, "parallelism": f"replicas{ws_n}",
+                       "l2": "no flush: inputs larger than L2 (expert weights streamed every step)"},
+            "e2e": {"value": ws_n * T * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
+                    "d2h_bytes_per_step": io_bytes},
+            "roofline": roofline, "layer_roofline": layer_roof, "cpu_baseline": cpu, "gpu_launches": n_launch,
+            "clocks": clocks.summary(), "device_status": moe.status_string(status),
+            "kernels": {n: {"launches": k["launches"], "avg_us": 1e3 * k["avg_ms"], "share": round(k["share"], 4)}
+                        for n, k in sorted(kernels.items(), key=lambda kv: -kv[1]["total_ms"])}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=workloads.CONFIG_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    spec = workloads.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, spec)
+    return run_ours(args, spec)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,227 @@
+/*
+ * libmoe -- a Mixture-of-Experts FFN layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer: router logits, softmax + top-K (+ renormalisation), dispatch of
+ * each token to its K experts, per expert act(x W_gate^T) * (x W_up^T) then
+ * W_down, a routing-weighted combine, and an optional sigmoid-gated shared
+ * expert.  Notation: T tokens, H hidden, E experts, K = top_k, I expert
+ * intermediate, Is shared intermediate, P = T*K (token, slot) pairs with pair
+ * id p = t*K + k.
+ *
+ * Conventions for every entry point
+ *  - Pointers to tensors are DEVICE pointers owned by the caller (moe_layer_host
+ *    is the one exception, see there).  The library never allocates, frees or
+ *    retains device memory; scratch comes from the caller's workspace.
+ *  - Tensors are dense and row-major.  Weights are stored out x in (the
+ *    nn.Linear convention): rows are contiguous along the input dimension.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream): they
+ *    return after enqueueing.  Arguments are checked on the host first; any
+ *    error return means nothing was launched and nothing was written.
+ *  - Device-side problems (an expert id out of range, a pipeline wait that ran
+ *    past its time limit) do not trap: kernels record a status word that
+ *    moe_last_device_status() reads.
+ *  - Limits: 1 <= E <= 256, 1 <= K <= min(E, 32), H, I and Is multiples of 32,
+ *    T <= 2^20.  T == 0 is valid and does nothing.  Every tensor pointer must
+ *    be 16-byte aligned.  Outputs may not alias inputs.
+ *  - The library keeps no per-call state; it is safe to call from several host
+ *    threads on different streams.
+ *
+ * Citations name the page (crate and file) and the function the operation
+ * follows.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* a size, flag or pointer is out of contract */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. H not a multiple of 32) */
+  MOE_ERR_WORKSPACE = 3,   /* workspace smaller than moe_workspace_bytes() */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute, copy) */
+  MOE_ERR_TIMEOUT = 5,     /* device: a pipeline wait ran past its limit (kernel gave up cleanly) */
+  MOE_ERR_DEVICE_INDEX = 6 /* device: an expert id outside [0, E) reached the permutation */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_Q8_0 = 2 } moe_dtype;
+
+/* SiLU(g) = g / (1 + e^-g)  (hf2q qwen35/gpu_ffn.rs, silu_mul_cpu);
+ * GELU_TANH(g) = 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3)))
+ * (mlx-native moe_dispatch.rs, fused_gelu_mul and its test oracle cpu_gelu). */
+typedef enum { MOE_ACT_SILU = 0, MOE_ACT_GELU_TANH = 1 } moe_act;
+
+typedef struct moe_desc {
+  int32_t T, H, E, I, top_k;
+  int32_t act;             /* moe_act, used by routed and shared experts */
+  int32_t renormalize;     /* 1: selected weights divided by their sum; 0: plain softmax probabilities */
+  int32_t act_dtype;       /* MOE_F32 | MOE_BF16: x and out */
+  int32_t w_dtype;         /* MOE_F32 | MOE_BF16 | MOE_Q8_0: expert and shared projections */
+  int32_t router_dtype;    /* MOE_F32 | MOE_BF16: router W and the shared-gate vector w_s */
+  int32_t has_router_bias; /* 1: logits += b_e before selection (ferrox-models decoder.rs, gpt_oss_ffn) */
+  int32_t shared_I;        /* 0: no shared expert */
+  int32_t has_shared_gate; /* 1: shared output scaled by sigmoid(w_s . x); 0: scale 1 */
+} moe_desc;
+
+/*
+ * Weights.  Shapes (out x in):
+ *   router [E,H], router_bias [E] f32, gate [E,I,H], up [E,I,H], down [E,H,I],
+ *   sh_gate [Is,H], sh_up [Is,H], sh_down [H,Is], sh_gate_w [H].
+ * For w_dtype == MOE_Q8_0 the projection pointers hold int8 quants with the
+ * same shapes and the *_scale pointers hold one fp16 scale per 32 consecutive
+ * inputs ([E,I,H/32], [E,H,I/32], [Is,H/32], [H,Is/32]); value = scale * q.
+ * moe_q8_0_split() converts GGML Q8_0 blocks into this split form.
+ * Unused pointers may be NULL.
+ */
+typedef struct moe_weights {
+  const void* router;
+  const float* router_bias;
+  const void* gate;
+  const void* up;
+  const void* down;
+  const void* sh_gate;
+  const void* sh_up;
+  const void* sh_down;
+  const void* sh_gate_w;
+  const void* gate_scale;
+  const void* up_scale;
+  const void* down_scale;
+  const void* sh_gate_scale;
+  const void* sh_up_scale;
+  const void* sh_down_scale;
+} moe_weights;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status s);
+
+/* Library version string (static). */
+const char* moe_version(void);
+
+/*
+ * Bytes of caller-provided device workspace moe_layer needs for `d` (affine in
+ * T for fixed sizes; 256-byte aligned regions).  Returns 0 for an invalid
+ * descriptor.  moe_expert_ffn and moe_combine need no more than this.
+ */
+size_t moe_workspace_bytes(const moe_desc* d);
+
+/*
+ * Router: logits, softmax, top-K with renormalisation.
+ * (hf2q qwen35/gpu_ffn.rs, softmax_topk_renorm_cpu and dispatch_moe_softmax_topk;
+ *  ferrum-kernels vnext_ops/moe.rs, route kernel, one 32-thread group per token)
+ *  x        [T,H] act_dtype
+ *  logits   [T,E] f32 out: x W_r^T (+ b), the values selection compared
+ *  topk_ids [T,K] int32 out: experts in order (logit desc, index asc)
+ *  topk_w   [T,K] f32 out: exp(l - m) over the selected (renormalised) or over all E
+ *  shared_gate [T] f32 out: sigmoid(w_s . x); required iff shared_I > 0 and has_shared_gate
+ */
+moe_status moe_route(const moe_desc* d, const void* x, const moe_weights* w, float* logits, int32_t* topk_ids,
+                     float* topk_w, float* shared_gate, moe_stream_t stream);
+
+/*
+ * Histogram, exclusive scan and stable permutation of the P pairs by expert
+ * (DS4Server qwen_mtplx.rs, gather_sort: argsort of the flat expert ids and
+ *  its inverse; ferrox-models decoder.rs, moe_ffn_batch buckets in token order).
+ *  topk_ids     [P] int32 in
+ *  counts       [E] int32 out: pairs routed to each expert
+ *  offsets      [E+1] int32 out: exclusive prefix sum, offsets[E] = P
+ *  sorted_pairs [P] int32 out: pair ids grouped by expert, ascending within an expert
+ *  pair_pos     [P] int32 out: inverse, sorted_pairs[pair_pos[p]] = p
+ * Ids outside [0,E) are skipped and reported as MOE_ERR_DEVICE_INDEX.
+ */
+moe_status moe_permute(const moe_desc* d, const int32_t* topk_ids, int32_t* counts, int32_t* offsets,
+                       int32_t* sorted_pairs, int32_t* pair_pos, moe_stream_t stream);
+
+/*
+ * Routed experts: for every expert e and each of its rows r in
+ * [offsets[e], offsets[e+1]) with pair p = sorted_pairs[r], token t = p / K:
+ *   y_slots[p,:] = topk_w[p] * W_down[e] (act(W_gate[e] x_t) * (W_up[e] x_t))
+ * (mlx-native moe_dispatch.rs, moe_dispatch per-expert loop; hf2q
+ *  qwen35/gpu_ffn.rs, quantized_matmul_id gate/up, silu_mul, down;
+ *  ferrum-kernels vnext_ops/moe.rs, routed_down_slots)
+ *  y_slots [P,H] f32 out.  Uses ws (>= moe_workspace_bytes(d) bytes).
+ */
+moe_status moe_expert_ffn(const moe_desc* d, const void* x, const moe_weights* w, const int32_t* offsets,
+                          const int32_t* sorted_pairs, const float* topk_w, float* y_slots, void* ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Combine: out[t,:] = sum_{k=0..K-1} y_slots[t*K+k,:] + s_t * shared(x_t), in
+ * that order, in f32, then converted to act_dtype; s_t = shared_gate[t] or 1.
+ * (mlx-native moe_dispatch.rs, moe_weighted_sum; hf2q qwen35/gpu_ffn.rs,
+ *  moe_weighted_reduce and the sigmoid-gated shared expert)
+ *  shared_gate [T] f32 from moe_route (ignored unless shared_I > 0 and has_shared_gate)
+ *  out [T,H] act_dtype out.  Runs the shared expert first when shared_I > 0 (uses ws).
+ */
+moe_status moe_combine(const moe_desc* d, const float* y_slots, const void* x, const moe_weights* w,
+                       const float* shared_gate, void* out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The whole layer in one call: route, permute, experts, shared expert, combine.
+ * Picks the tensor-core path (tcgen05 grouped GEMMs) when x and the expert
+ * weights are bf16 and T > 64, else the weight-streaming path.
+ *  x [T,H] act_dtype in, out [T,H] act_dtype out, ws >= moe_workspace_bytes(d).
+ */
+moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, void* out, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/*
+ * moe_layer with HOST activations: copies x_host (T*H elements of act_dtype)
+ * into x_dev, runs moe_layer, copies out_dev back into out_host, all on
+ * `stream` (one cudaMemcpyAsync per copy; pinned host memory makes them
+ * asynchronous).  x_dev and out_dev are caller-owned device buffers of the
+ * same size.  Returns after enqueueing; synchronise `stream` before reading
+ * out_host.
+ */
+moe_status moe_layer_host(const moe_desc* d, const void* x_host, const moe_weights* w, void* out_host, void* x_dev,
+                          void* out_dev, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Split GGML Q8_0 blocks ({fp16 d; int8 q[32]}, 34 bytes, along the input
+ * dimension) of a [rows, cols] matrix into int8 quants [rows, cols] and fp16
+ * scales [rows, cols/32], the form moe_weights expects for MOE_Q8_0.  A
+ * one-time load step (the pages repack weights at load: hf2q qwen35/gpu_ffn.rs,
+ * pre-cast to bf16; ferrox-models decoder.rs, MoePackedQ4Planes).
+ */
+moe_status moe_q8_0_split(const void* blocks, int64_t rows, int64_t cols, int8_t* q, void* scales,
+                          moe_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device (MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_INDEX), or
+ * MOE_ERR_CUDA if the synchronisation failed.
+ */
+moe_status moe_last_device_status(moe_stream_t stream);
+
+/* ---- instrumentation (host side only; no device memory) ---- */
+
+/* Total kernels this library has launched in this process. */
+uint64_t moe_launch_count(void);
+
+/* Per-kernel CUDA-event timing of later calls: on != 0 starts recording (and
+ * clears earlier records), 0 stops.  Records are kept for up to 4096 launches. */
+void moe_trace_enable(int on);
+
+/* Synchronises the recorded events and copies up to `max` records: kernel name
+ * (static string) and duration in milliseconds.  Returns the number of
+ * records available. */
+int moe_trace_read(const char** names, float* ms, int max);
+
+/* Debug: per-wait time limit in SM clock cycles for the pipeline waits of the
+ * tensor-core kernels (default 2^31, about a second); and a fault switch that
+ * makes the TMA producer of the next grouped-GEMM launches skip one stage's
+ * loads, so the consumer's wait runs out and MOE_ERR_TIMEOUT is reported.
+ * Used by the failure-detection test; never set in normal use. */
+void moe_debug_set_wait_limit(int64_t cycles);
+void moe_debug_set_skip_stage(int enable);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

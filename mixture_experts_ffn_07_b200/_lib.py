@@ -1,0 +1,91 @@
+"""ctypes declarations of libmoe.so (include/moe.h).  Argument marshalling only.
+
+Importing this module loads the library; it raises if ``libmoe.so`` has not
+been built -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+# enums (include/moe.h)
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
+    MOE_ERR_DEVICE_INDEX = range(7)
+MOE_F32, MOE_BF16, MOE_Q8_0 = 0, 1, 2
+MOE_ACT_SILU, MOE_ACT_GELU_TANH = 0, 1
+
+# every symbol include/moe.h declares
+EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
+           "moe_combine", "moe_layer", "moe_layer_host", "moe_q8_0_split", "moe_last_device_status",
+           "moe_launch_count", "moe_trace_enable", "moe_trace_read", "moe_debug_set_wait_limit",
+           "moe_debug_set_skip_stage")
+
+
+class MoeDesc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("T", "H", "E", "I", "top_k", "act", "renormalize", "act_dtype", "w_dtype", "router_dtype",
+                 "has_router_bias", "shared_I", "has_shared_gate")]
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("router", "router_bias", "gate", "up", "down", "sh_gate", "sh_up", "sh_down", "sh_gate_w",
+                 "gate_scale", "up_scale", "down_scale", "sh_gate_scale", "sh_up_scale", "sh_down_scale")]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run mixture_experts_ffn_07_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, DP, WP, I32, I64 = (ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(MoeDesc),
+                                  ctypes.POINTER(MoeWeights), ctypes.c_int, ctypes.c_int64)
+        L.moe_status_string.argtypes = [I32]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_version.restype = ctypes.c_char_p
+        L.moe_workspace_bytes.argtypes = [DP]
+        L.moe_workspace_bytes.restype = S
+        L.moe_route.argtypes = [DP, P, WP, P, P, P, P, P]
+        L.moe_permute.argtypes = [DP, P, P, P, P, P, P]
+        L.moe_expert_ffn.argtypes = [DP, P, WP, P, P, P, P, P, S, P]
+        L.moe_combine.argtypes = [DP, P, P, WP, P, P, P, S, P]
+        L.moe_layer.argtypes = [DP, P, WP, P, P, S, P]
+        L.moe_layer_host.argtypes = [DP, P, WP, P, P, P, P, S, P]
+        L.moe_q8_0_split.argtypes = [P, I64, I64, P, P, P]
+        L.moe_last_device_status.argtypes = [P]
+        for f in (L.moe_route, L.moe_permute, L.moe_expert_ffn, L.moe_combine, L.moe_layer, L.moe_layer_host,
+                  L.moe_q8_0_split, L.moe_last_device_status):
+            f.restype = I32
+        L.moe_launch_count.restype = ctypes.c_uint64
+        L.moe_trace_enable.argtypes = [I32]
+        L.moe_trace_enable.restype = None
+        L.moe_trace_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float), I32]
+        L.moe_trace_read.restype = I32
+        L.moe_debug_set_wait_limit.argtypes = [I64]
+        L.moe_debug_set_wait_limit.restype = None
+        L.moe_debug_set_skip_stage.argtypes = [I32]
+        L.moe_debug_set_skip_stage.restype = None
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().moe_status_string(code).decode()
+
+
+def check(code: int, where: str) -> None:
+    if code != MOE_OK:
+        raise MoeError(code, where)

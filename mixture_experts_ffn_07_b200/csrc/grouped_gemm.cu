@@ -1,0 +1,424 @@
+// Grouped GEMM on Blackwell tensor cores for the expert projections.
+//
+// Role of the pages' id-indexed matmuls (hf2q qwen35/gpu_ffn.rs,
+// quantized_matmul_id for gate/up and down; DS4Server qwen_mtplx.rs,
+// GatherQMM over expert-sorted rows) with the activation product fused into
+// the gate/up epilogue (hf2q, fused_gate_up_silu; ferrum-kernels
+// vnext_ops/moe.rs, gate_up_silu) and the routing weight fused into the down
+// epilogue (ferrum-kernels, routed_down_slots; mlx-native moe_dispatch.rs,
+// moe_weighted_sum).
+//
+// Design (sm_100a):
+//  * persistent grid, one CTA per SM; work items (group, n-tile, m-tile) with
+//    the m-tile fastest so CTAs running at the same time share weight tiles
+//    in L2;
+//  * warp 0: TMA producer (one lane) into a 4-stage shared-memory ring of
+//    128x64 A tiles and 256x64 B tiles, 128-byte swizzle;
+//  * warp 1: allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=256,
+//    K=16, bf16 in, f32 accumulate) from one lane; two accumulators so the
+//    epilogue of one tile overlaps the main loop of the next;
+//  * warps 2-5: epilogue, one TMEM lane (= output row) per thread;
+//  * dual mode (gate/up): the 256-row B tile is 128 rows of W_gate followed
+//    by the same 128 rows of W_up, so TMEM columns [0,128) hold x W_gate^T and
+//    [128,256) hold x W_up^T for the same outputs; the epilogue writes
+//    act(g) * u as bf16;
+//  * single mode (down, router): the epilogue scales row r by row_scale and
+//    stores it at row row_map[r] in f32 (the slot row of the pair).
+//  * every mbarrier wait is bounded; on expiry the CTA records
+//    MOE_ERR_TIMEOUT, lets in-flight copies and MMAs land, frees TMEM and exits.
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int BN_MMA = 256;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN_MMA * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN_MMA;
+constexpr int MAX_G = 256;
+constexpr int THREADS = 192;
+
+struct Aux {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+  int item_off[MAX_G + 1];
+  int row_off[MAX_G];
+  int cnt[MAX_G];
+};
+
+constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(Aux);
+
+struct KParams {
+  const int32_t* offsets;
+  int G;
+  int rows_single;
+  int N;
+  int Kdim;
+  int n_tiles;
+  int col_step;
+  int act;
+  __nv_bfloat16* out_bf16;
+  float* out_f32;
+  const int32_t* row_map;
+  const float* row_scale;
+  int* status;
+  long long wait_limit;
+  int skip_stage;
+};
+
+// Wait ignoring the abort flag (used to drain in-flight work before exit).
+__device__ __forceinline__ bool wait_cycles(uint64_t* bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit) return false;
+  return true;
+}
+
+__device__ __forceinline__ void decode_item(const Aux& aux, int G, int w, int& g, int& mt, int& nt) {
+  int lo = 0, hi = G - 1;  // largest g with item_off[g] <= w
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (aux.item_off[mid] <= w)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  g = lo;
+  const int tiles = (aux.cnt[g] + BM - 1) / BM;
+  const int local = w - aux.item_off[g];
+  nt = local / tiles;
+  mt = local - nt * tiles;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <bool DUAL>
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
+                        const __grid_constant__ CUtensorMap mapB1, const KParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Aux& aux = *reinterpret_cast<Aux*>(smem + STAGES * STAGE_BYTES);
+  volatile int* abort_flag = &aux.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int g = threadIdx.x; g < p.G; g += THREADS) {
+    const int r0 = p.offsets ? p.offsets[g] : 0;
+    const int r1 = p.offsets ? p.offsets[g + 1] : p.rows_single;
+    aux.row_off[g] = r0;
+    aux.cnt[g] = max(0, r1 - r0);
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&aux.full[s], 1);
+      mbar_init(&aux.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&aux.tfull[b], 1);
+      mbar_init(&aux.tempty[b], 4);
+    }
+    mbar_init(&aux.done, 1);
+    aux.abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of work items per group; lane owns groups [8*lane, 8*lane+8)
+    int v[8], local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int g = lane * 8 + i;
+      v[i] = g < p.G ? ((aux.cnt[g] + BM - 1) / BM) * p.n_tiles : 0;
+      local += v[i];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    int run = incl - local;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int g = lane * 8 + i;
+      if (g < p.G) aux.item_off[g] = run;
+      run += v[i];
+    }
+    if (lane == 31) aux.item_off[p.G] = incl;
+  } else if (warp == 1) {
+    tmem_alloc(&aux.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = aux.tmem_base;
+  const int total = aux.item_off[p.G];
+  const int nkb = (p.Kdim + BK - 1) / BK;
+  const long long limit = p.wait_limit;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      prefetch_tensormap(&mapA);
+      prefetch_tensormap(&mapB0);
+      if (DUAL) prefetch_tensormap(&mapB1);
+      uint32_t kbg = 0, outstanding = 0, out_phase = 0;
+      bool skipped = false;
+      for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
+        int g, mt, nt;
+        decode_item(aux, p.G, w, g, mt, nt);
+        const int a_row = aux.row_off[g] + mt * BM;
+        const int b_row = g * p.N + nt * p.col_step;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = kbg % STAGES;
+          const uint32_t ph = (kbg / STAGES) & 1u;
+          if (!mbar_wait_bounded(&aux.empty[s], ph ^ 1u, limit, abort_flag)) break;
+          outstanding &= ~(1u << s);
+          if (p.skip_stage && !skipped && blockIdx.x == 0) {  // debug: leave this stage unfilled
+            skipped = true;
+            continue;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(&aux.full[s], STAGE_BYTES);
+          tma_load_2d(sa, &mapA, &aux.full[s], kb * BK, a_row);
+          if (DUAL) {
+            tma_load_2d(sb, &mapB0, &aux.full[s], kb * BK, b_row);
+            tma_load_2d(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row);
+          } else {
+            tma_load_2d(sb, &mapB0, &aux.full[s], kb * BK, b_row);
+          }
+          outstanding |= 1u << s;
+          out_phase = (out_phase & ~(1u << s)) | (ph << s);
+        }
+      }
+      if (*abort_flag) {  // let issued copies land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (outstanding & (1u << s)) wait_cycles(&aux.full[s], (out_phase >> s) & 1u, limit);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(BM, BN_MMA);
+      uint32_t kbg = 0;
+      int it = 0;
+      for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_ph = (it >> 1) & 1u;
+        if (!mbar_wait_bounded(&aux.tempty[acc], acc_ph ^ 1u, limit, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN_MMA;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = kbg % STAGES;
+          const uint32_t ph = (kbg / STAGES) & 1u;
+          if (!mbar_wait_bounded(&aux.full[s], ph, limit, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(smem + s * STAGE_BYTES);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                      (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(&aux.empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&aux.tfull[acc]);
+      }
+      umma_commit(&aux.done);  // every MMA issued above completes before TMEM is released
+      wait_cycles(&aux.done, 0, limit);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are reachable from this warp
+    const int r = q * 32 + lane;
+    int it = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+      int g, mt, nt;
+      decode_item(aux, p.G, w, g, mt, nt);
+      const int acc = it & 1;
+      const uint32_t acc_ph = (it >> 1) & 1u;
+      // every lane waits; the outcome is made warp-uniform because the TMEM loads below are .sync.aligned
+      const bool ok = mbar_wait_bounded(&aux.tfull[acc], acc_ph, limit, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int rows_valid = min(BM, aux.cnt[g] - mt * BM);
+      const int a_row = aux.row_off[g] + mt * BM;
+      const int col0 = nt * p.col_step;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN_MMA;
+      if (DUAL) {
+        for (int c = 0; c < BN_MMA / 2; c += 32) {
+          uint32_t gr[32], ur[32];
+          tmem_ld_32x32b_x32(tbase + c, gr);
+          tmem_ld_32x32b_x32(tbase + BN_MMA / 2 + c, ur);
+          tmem_ld_wait();
+          if (r < rows_valid && col0 + c < p.N) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float h0 = act_fn(p.act, __uint_as_float(gr[2 * j])) * __uint_as_float(ur[2 * j]);
+              const float h1 = act_fn(p.act, __uint_as_float(gr[2 * j + 1])) * __uint_as_float(ur[2 * j + 1]);
+              packed[j] = pack_bf16x2(h0, h1);
+            }
+            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(a_row + r) * p.N + col0 + c;
+            if (col0 + c + 32 <= p.N) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            } else {
+              const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(packed);
+              for (int j = 0; j < 32 && col0 + c + j < p.N; ++j) dst[j] = hv[j];
+            }
+          }
+        }
+      } else {
+        int dest = -1;
+        float scale = 1.f;
+        if (r < rows_valid) {
+          const int src = a_row + r;
+          dest = p.row_map ? p.row_map[src] : src;
+          scale = p.row_scale ? p.row_scale[dest] : 1.f;
+        }
+        for (int c = 0; c < BN_MMA; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c, v);
+          tmem_ld_wait();
+          if (dest >= 0 && col0 + c < p.N) {
+            float* dst = p.out_f32 + static_cast<size_t>(dest) * p.N + col0 + c;
+            if (col0 + c + 32 <= p.N) {
+              float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                d4[j] = make_float4(scale * __uint_as_float(v[4 * j]), scale * __uint_as_float(v[4 * j + 1]),
+                                    scale * __uint_as_float(v[4 * j + 2]), scale * __uint_as_float(v[4 * j + 3]));
+            } else {
+              for (int j = 0; j < 32 && col0 + c + j < p.N; ++j) dst[j] = scale * __uint_as_float(v[j]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aux.tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && aux.abort) record_status(p.status, MOE_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read in boxes of box_rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool DUAL>
+cudaError_t set_smem_attr() {
+  static int done_mask = 0;  // bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 31 && (done_mask & (1 << dev))) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(SMEM_BYTES));
+  if (e == cudaSuccess && dev < 31) done_mask |= 1 << dev;
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
+  if (a.G <= 0 || a.max_rows <= 0 || a.N <= 0 || a.rows_A <= 0) return cudaSuccess;
+  if (a.G > MAX_G) return cudaErrorInvalidValue;
+  CUtensorMap mA, mB0, mB1;
+  const uint32_t brows = a.dual ? BN_MMA / 2 : BN_MMA;
+  if (!make_map(&mA, a.A, static_cast<uint64_t>(a.rows_A), static_cast<uint64_t>(a.Kdim), BM) ||
+      !make_map(&mB0, a.B0, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), brows))
+    return cudaErrorInvalidValue;
+  if (a.dual) {
+    if (!make_map(&mB1, a.B1, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), brows))
+      return cudaErrorInvalidValue;
+  } else {
+    mB1 = mB0;
+  }
+  KParams p;
+  p.offsets = a.offsets;
+  p.G = a.G;
+  p.rows_single = static_cast<int>(a.rows_A);
+  p.N = a.N;
+  p.Kdim = a.Kdim;
+  p.col_step = a.dual ? BN_MMA / 2 : BN_MMA;
+  p.n_tiles = (a.N + p.col_step - 1) / p.col_step;
+  p.act = a.act;
+  p.out_bf16 = a.out_bf16;
+  p.out_f32 = a.out_f32;
+  p.row_map = a.row_map;
+  p.row_scale = a.row_scale;
+  p.status = c.status;
+  p.wait_limit = c.wait_limit;
+  p.skip_stage = c.skip_stage;
+  const long long tiles_bound = static_cast<long long>(a.max_rows) / BM + std::min(a.G, a.max_rows);
+  const long long items_bound = tiles_bound * p.n_tiles;
+  const int grid = static_cast<int>(std::max(1LL, std::min<long long>(c.num_sms, items_bound)));
+  cudaError_t e = a.dual ? set_smem_attr<true>() : set_smem_attr<false>();
+  if (e != cudaSuccess) return e;
+  KernelScope ks(c, a.name ? a.name : (a.dual ? "grouped_gemm_dual" : "grouped_gemm"));
+  if (a.dual)
+    grouped_gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, c.stream>>>(mA, mB0, mB1, p);
+  else
+    grouped_gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, c.stream>>>(mA, mB0, mB1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,483 @@
+// The C ABI of libmoe (declared in include/moe.h): argument checks, the
+// workspace layout, the order of kernel launches for each entry point, the
+// device status word, and the host-side launch counter and event trace.
+//
+// Path choice: bf16 activations with bf16 expert weights and T > 64 take the
+// tensor-core path (row gather + tcgen05 grouped GEMMs); everything else takes
+// the weight-streaming path (expert-major GEMV kernels), which reads each
+// touched expert's weights once and is the bandwidth-optimal form for small T.
+#include <atomic>
+#include <mutex>
+
+#include "kernels.h"
+
+namespace {
+
+__device__ int g_device_status;  // one per device; first error wins, cleared by moe_last_device_status
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxT = 1 << 20;
+constexpr int kTraceCap = 4096;
+
+struct DeviceInfo {
+  bool ready = false;
+  int* status = nullptr;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<long long> g_wait_limit{1LL << 31};
+std::atomic<int> g_skip_stage{0};
+
+struct TraceRec {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+int g_trace_n = 0;
+TraceRec g_trace[kTraceCap];
+
+bool make_ctx(cudaStream_t s, moe::Ctx* c) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return false;
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return false;
+      d.status = static_cast<int*>(p);
+      d.num_sms = sms;
+      d.ready = true;
+    }
+    c->status = d.status;
+    c->num_sms = d.num_sms;
+  }
+  c->stream = s;
+  c->wait_limit = g_wait_limit.load();
+  c->skip_stage = g_skip_stage.load();
+  return true;
+}
+
+inline size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool tensor_path(const moe_desc& d) { return d.act_dtype == MOE_BF16 && d.w_dtype == MOE_BF16 && d.T > 64; }
+
+bool tensor_router(const moe_desc& d) {
+  return d.act_dtype == MOE_BF16 && d.router_dtype == MOE_BF16 && d.T > 64 && d.E % 32 == 0;
+}
+
+bool shared_gated(const moe_desc& d) { return d.shared_I > 0 && d.has_shared_gate; }
+
+moe_status check_desc(const moe_desc* d) {
+  if (!d) return MOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->T > kMaxT || d->H <= 0 || d->I <= 0 || d->E < 1 || d->E > 256 || d->top_k < 1 ||
+      d->top_k > d->E || d->top_k > 32 || d->shared_I < 0)
+    return MOE_ERR_INVALID_ARG;
+  if ((d->act != MOE_ACT_SILU && d->act != MOE_ACT_GELU_TANH) || (d->renormalize != 0 && d->renormalize != 1) ||
+      (d->has_router_bias != 0 && d->has_router_bias != 1) || (d->has_shared_gate != 0 && d->has_shared_gate != 1))
+    return MOE_ERR_INVALID_ARG;
+  if ((d->act_dtype != MOE_F32 && d->act_dtype != MOE_BF16) ||
+      (d->w_dtype != MOE_F32 && d->w_dtype != MOE_BF16 && d->w_dtype != MOE_Q8_0) ||
+      (d->router_dtype != MOE_F32 && d->router_dtype != MOE_BF16))
+    return MOE_ERR_INVALID_ARG;
+  if (d->H % 32 || d->I % 32 || d->shared_I % 32) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct Layout {
+  size_t logits, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos, y_slots, x_perm, h, h_s, y_s, total;
+};
+
+Layout layout_of(const moe_desc& d) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t T = d.T, H = d.H, E = d.E, I = d.I, P = T * d.top_k, Is = d.shared_I;
+  const bool tc = tensor_path(d);
+  L.logits = take(T * E * 4);
+  L.ids = take(P * 4);
+  L.w = take(P * 4);
+  L.shared_gate = take(T * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.sorted_pairs = take(P * 4);
+  L.pair_pos = take(P * 4);
+  L.y_slots = take(P * H * 4);
+  L.x_perm = tc ? take(P * H * 2) : 0;
+  L.h = take(P * I * (tc ? 2 : 4));
+  L.h_s = Is ? take(T * Is * (tc ? 2 : 4)) : 0;
+  L.y_s = Is ? take(T * H * 4) : 0;
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                          \
+  do {                                         \
+    const cudaError_t e_ = (expr);             \
+    if (e_ != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+// ---------------------------------------------------------------- stages
+moe_status route_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const moe_weights& w, float* logits,
+                      int32_t* ids, float* tw, float* shared_gate) {
+  const void* w_s = shared_gated(d) ? w.sh_gate_w : nullptr;
+  if (tensor_router(d)) {
+    moe::GemmArgs a{};
+    a.A = static_cast<const __nv_bfloat16*>(x);
+    a.rows_A = d.T;
+    a.Kdim = d.H;
+    a.B0 = static_cast<const __nv_bfloat16*>(w.router);
+    a.N = d.E;
+    a.G = 1;
+    a.max_rows = d.T;
+    a.dual = false;
+    a.out_f32 = logits;
+    a.name = "router_gemm";
+    MOE_TRY(moe::launch_grouped_gemm(c, a));
+    if (w_s)
+      MOE_TRY(moe::launch_router_logits(c, x, d.act_dtype, w.router, w_s, d.router_dtype, d.T, d.H, d.E, false,
+                                        logits, shared_gate));
+  } else {
+    MOE_TRY(moe::launch_router_logits(c, x, d.act_dtype, w.router, w_s, d.router_dtype, d.T, d.H, d.E, true, logits,
+                                      shared_gate));
+  }
+  MOE_TRY(moe::launch_router_topk(c, logits, d.has_router_bias ? w.router_bias : nullptr, d.T, d.E, d.top_k,
+                                  d.renormalize, ids, tw));
+  return MOE_OK;
+}
+
+moe_status expert_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const moe_weights& w,
+                       const int32_t* offsets, const int32_t* sorted_pairs, const float* tw, float* y_slots, void* ws,
+                       const Layout& L) {
+  const int P = d.T * d.top_k;
+  if (tensor_path(d)) {
+    __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.x_perm);
+    __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
+    MOE_TRY(moe::launch_gather_rows(c, static_cast<const __nv_bfloat16*>(x), sorted_pairs, offsets, d.E, d.top_k, P,
+                                    d.H, xp));
+    moe::GemmArgs a{};
+    a.A = xp;
+    a.rows_A = P;
+    a.Kdim = d.H;
+    a.B0 = static_cast<const __nv_bfloat16*>(w.gate);
+    a.B1 = static_cast<const __nv_bfloat16*>(w.up);
+    a.N = d.I;
+    a.G = d.E;
+    a.offsets = offsets;
+    a.max_rows = P;
+    a.dual = true;
+    a.act = d.act;
+    a.out_bf16 = h;
+    a.name = "expert_gate_up_gemm";
+    MOE_TRY(moe::launch_grouped_gemm(c, a));
+    moe::GemmArgs b{};
+    b.A = h;
+    b.rows_A = P;
+    b.Kdim = d.I;
+    b.B0 = static_cast<const __nv_bfloat16*>(w.down);
+    b.N = d.H;
+    b.G = d.E;
+    b.offsets = offsets;
+    b.max_rows = P;
+    b.dual = false;
+    b.out_f32 = y_slots;
+    b.row_map = sorted_pairs;
+    b.row_scale = tw;
+    b.name = "expert_down_gemm";
+    MOE_TRY(moe::launch_grouped_gemm(c, b));
+  } else {
+    float* h = at<float>(ws, L.h);
+    MOE_TRY(moe::launch_stream_gate_up(c, x, d.act_dtype, d.T, d.H, d.I, d.top_k, w.gate, w.up, w.gate_scale,
+                                       w.up_scale, d.w_dtype, offsets, d.E, sorted_pairs, P, d.act, h));
+    MOE_TRY(moe::launch_stream_down(c, h, d.I, d.H, w.down, w.down_scale, d.w_dtype, offsets, d.E, sorted_pairs, P,
+                                    tw, y_slots));
+  }
+  return MOE_OK;
+}
+
+moe_status combine_impl(const moe::Ctx& c, const moe_desc& d, const float* y_slots, const void* x,
+                        const moe_weights& w, const float* shared_gate, void* out, void* ws, const Layout& L) {
+  float* y_s = nullptr;
+  if (d.shared_I > 0) {
+    y_s = at<float>(ws, L.y_s);
+    const float* gate = shared_gated(d) ? shared_gate : nullptr;
+    if (tensor_path(d)) {
+      __nv_bfloat16* hs = at<__nv_bfloat16>(ws, L.h_s);
+      moe::GemmArgs a{};
+      a.A = static_cast<const __nv_bfloat16*>(x);
+      a.rows_A = d.T;
+      a.Kdim = d.H;
+      a.B0 = static_cast<const __nv_bfloat16*>(w.sh_gate);
+      a.B1 = static_cast<const __nv_bfloat16*>(w.sh_up);
+      a.N = d.shared_I;
+      a.G = 1;
+      a.max_rows = d.T;
+      a.dual = true;
+      a.act = d.act;
+      a.out_bf16 = hs;
+      a.name = "shared_gate_up_gemm";
+      MOE_TRY(moe::launch_grouped_gemm(c, a));
+      moe::GemmArgs b{};
+      b.A = hs;
+      b.rows_A = d.T;
+      b.Kdim = d.shared_I;
+      b.B0 = static_cast<const __nv_bfloat16*>(w.sh_down);
+      b.N = d.H;
+      b.G = 1;
+      b.max_rows = d.T;
+      b.dual = false;
+      b.out_f32 = y_s;
+      b.row_scale = gate;
+      b.name = "shared_down_gemm";
+      MOE_TRY(moe::launch_grouped_gemm(c, b));
+    } else {
+      float* hs = at<float>(ws, L.h_s);
+      MOE_TRY(moe::launch_stream_gate_up(c, x, d.act_dtype, d.T, d.H, d.shared_I, 1, w.sh_gate, w.sh_up,
+                                         w.sh_gate_scale, w.sh_up_scale, d.w_dtype, nullptr, 1, nullptr, d.T, d.act,
+                                         hs));
+      MOE_TRY(moe::launch_stream_down(c, hs, d.shared_I, d.H, w.sh_down, w.sh_down_scale, d.w_dtype, nullptr, 1,
+                                      nullptr, d.T, gate, y_s));
+    }
+  }
+  MOE_TRY(moe::launch_combine(c, y_slots, y_s, d.T, d.top_k, d.H, out, d.act_dtype));
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- argument checks
+moe_status check_router_args(const moe_desc& d, const void* x, const moe_weights* w) {
+  if (!x || !w || !w->router || !aligned16(x) || !aligned16(w->router)) return MOE_ERR_INVALID_ARG;
+  if (d.has_router_bias && !w->router_bias) return MOE_ERR_INVALID_ARG;
+  if (shared_gated(d) && (!w->sh_gate_w || !aligned16(w->sh_gate_w))) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status check_expert_weights(const moe_desc& d, const moe_weights* w) {
+  if (!w || !w->gate || !w->up || !w->down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->gate) || !aligned16(w->up) || !aligned16(w->down)) return MOE_ERR_INVALID_ARG;
+  if (d.w_dtype == MOE_Q8_0 && (!w->gate_scale || !w->up_scale || !w->down_scale)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status check_shared_weights(const moe_desc& d, const moe_weights* w) {
+  if (d.shared_I == 0) return MOE_OK;
+  if (!w || !w->sh_gate || !w->sh_up || !w->sh_down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->sh_gate) || !aligned16(w->sh_up) || !aligned16(w->sh_down)) return MOE_ERR_INVALID_ARG;
+  if (d.w_dtype == MOE_Q8_0 && (!w->sh_gate_scale || !w->sh_up_scale || !w->sh_down_scale))
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- instrumentation
+namespace moe {
+
+KernelScope::KernelScope(const Ctx& c, const char* name) : ctx(c), slot(-1) {
+  g_launches.fetch_add(1);
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  if (g_trace_on && g_trace_n < kTraceCap) {
+    TraceRec& r = g_trace[g_trace_n];
+    if (!r.start) {
+      cudaEventCreate(&r.start);
+      cudaEventCreate(&r.stop);
+    }
+    r.name = name;
+    slot = g_trace_n++;
+    cudaEventRecord(r.start, c.stream);
+  }
+}
+
+KernelScope::~KernelScope() {
+  if (slot >= 0) cudaEventRecord(g_trace[slot].stop, ctx.stream);
+}
+
+}  // namespace moe
+
+// ---------------------------------------------------------------- C ABI
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported size or format";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_INDEX: return "expert id out of range";
+  }
+  return "unknown status";
+}
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+size_t moe_workspace_bytes(const moe_desc* d) {
+  if (check_desc(d) != MOE_OK) return 0;
+  return layout_of(*d).total;
+}
+
+moe_status moe_route(const moe_desc* d, const void* x, const moe_weights* w, float* logits, int32_t* topk_ids,
+                     float* topk_w, float* shared_gate, moe_stream_t stream) {
+  moe_status st = check_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = check_router_args(*d, x, w)) != MOE_OK) return st;
+  if (!logits || !topk_ids || !topk_w || !aligned16(logits)) return MOE_ERR_INVALID_ARG;
+  if (shared_gated(*d) && !shared_gate) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return route_impl(c, *d, x, *w, logits, topk_ids, topk_w, shared_gate);
+}
+
+moe_status moe_permute(const moe_desc* d, const int32_t* topk_ids, int32_t* counts, int32_t* offsets,
+                       int32_t* sorted_pairs, int32_t* pair_pos, moe_stream_t stream) {
+  moe_status st = check_desc(d);
+  if (st != MOE_OK) return st;
+  if (!topk_ids || !counts || !offsets || !sorted_pairs || !pair_pos) return MOE_ERR_INVALID_ARG;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return from_cuda(moe::launch_permute(c, topk_ids, d->T * d->top_k, d->E, counts, offsets, sorted_pairs, pair_pos));
+}
+
+moe_status moe_expert_ffn(const moe_desc* d, const void* x, const moe_weights* w, const int32_t* offsets,
+                          const int32_t* sorted_pairs, const float* topk_w, float* y_slots, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = check_expert_weights(*d, w)) != MOE_OK) return st;
+  if (!x || !aligned16(x) || !offsets || !sorted_pairs || !topk_w || !y_slots || !aligned16(y_slots))
+    return MOE_ERR_INVALID_ARG;
+  const Layout L = layout_of(*d);
+  if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return expert_impl(c, *d, x, *w, offsets, sorted_pairs, topk_w, y_slots, ws, L);
+}
+
+moe_status moe_combine(const moe_desc* d, const float* y_slots, const void* x, const moe_weights* w,
+                       const float* shared_gate, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_desc(d);
+  if (st != MOE_OK) return st;
+  if (!y_slots || !out || !aligned16(y_slots) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (d->shared_I > 0) {
+    if ((st = check_shared_weights(*d, w)) != MOE_OK) return st;
+    if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    if (shared_gated(*d) && !shared_gate) return MOE_ERR_INVALID_ARG;
+  }
+  const Layout L = layout_of(*d);
+  if (d->shared_I > 0 && (!ws || ws_bytes < L.total)) return MOE_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return combine_impl(c, *d, y_slots, x, *w, shared_gate, out, ws, L);
+}
+
+moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, void* out, void* ws, size_t ws_bytes,
+                     moe_stream_t stream) {
+  moe_status st = check_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = check_router_args(*d, x, w)) != MOE_OK) return st;
+  if ((st = check_expert_weights(*d, w)) != MOE_OK) return st;
+  if ((st = check_shared_weights(*d, w)) != MOE_OK) return st;
+  if (!out || !aligned16(out) || out == x) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout_of(*d);
+  if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  float* logits = at<float>(ws, L.logits);
+  int32_t* ids = at<int32_t>(ws, L.ids);
+  float* tw = at<float>(ws, L.w);
+  float* sg = at<float>(ws, L.shared_gate);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* sorted_pairs = at<int32_t>(ws, L.sorted_pairs);
+  float* y_slots = at<float>(ws, L.y_slots);
+  if ((st = route_impl(c, *d, x, *w, logits, ids, tw, sg)) != MOE_OK) return st;
+  MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, at<int32_t>(ws, L.counts), offsets, sorted_pairs,
+                              at<int32_t>(ws, L.pair_pos)));
+  if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L)) != MOE_OK) return st;
+  return combine_impl(c, *d, y_slots, x, *w, sg, out, ws, L);
+}
+
+moe_status moe_layer_host(const moe_desc* d, const void* x_host, const moe_weights* w, void* out_host, void* x_dev,
+                          void* out_dev, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_desc(d);
+  if (st != MOE_OK) return st;
+  if (!x_host || !out_host || !x_dev || !out_dev) return MOE_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(d->T) * d->H * (d->act_dtype == MOE_F32 ? 4 : 2);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->T > 0 && cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((st = moe_layer(d, x_dev, w, out_dev, ws, ws_bytes, stream)) != MOE_OK) return st;
+  if (d->T > 0 && cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_q8_0_split(const void* blocks, int64_t rows, int64_t cols, int8_t* q, void* scales,
+                          moe_stream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 32) return MOE_ERR_INVALID_ARG;
+  if (rows * cols == 0) return MOE_OK;
+  if (!blocks || !q || !scales || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+    return MOE_ERR_INVALID_ARG;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return from_cuda(moe::launch_q8_0_split(c, blocks, rows, cols, q, scales));
+}
+
+moe_status moe_last_device_status(moe_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status>(v);
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+void moe_trace_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  g_trace_on = on != 0;
+  if (g_trace_on) g_trace_n = 0;
+}
+
+int moe_trace_read(const char** names, float* ms, int max) {
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  for (int i = 0; i < g_trace_n && i < max; ++i) {
+    float t = -1.f;
+    if (cudaEventSynchronize(g_trace[i].stop) == cudaSuccess) cudaEventElapsedTime(&t, g_trace[i].start, g_trace[i].stop);
+    if (names) names[i] = g_trace[i].name;
+    if (ms) ms[i] = t;
+  }
+  return g_trace_n;
+}
+
+void moe_debug_set_wait_limit(int64_t cycles) { g_wait_limit.store(cycles > 0 ? cycles : (1LL << 31)); }
+
+void moe_debug_set_skip_stage(int enable) { g_skip_stage.store(enable ? 1 : 0); }
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+"""The C-ABI library loads and exports every symbol include/moe.h declares, and the
+host-side checks reject bad arguments before touching CUDA (CPU only: no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from mixture_experts_ffn_07_b200 import _lib
+    return _lib.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    from mixture_experts_ffn_07_b200 import _lib
+    names = _declared()
+    assert len(names) >= 15
+    assert sorted(_lib.EXPORTS) == names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_struct_layouts_match_header(L):
+    from mixture_experts_ffn_07_b200 import _lib
+    src = open(HEADER).read()
+    desc_fields = re.search(r"typedef struct moe_desc \{(.*?)\} moe_desc;", src, re.S).group(1)
+    desc_fields = re.sub(r"/\*.*?\*/", "", desc_fields, flags=re.S)
+    n_desc = sum(len(line.split(";")[0].replace("int32_t", "").split(",")) for line in desc_fields.split("\n")
+                 if "int32_t" in line)
+    assert ctypes.sizeof(_lib.MoeDesc) == 4 * n_desc
+    w_fields = re.search(r"typedef struct moe_weights \{(.*?)\} moe_weights;", src, re.S).group(1)
+    assert ctypes.sizeof(_lib.MoeWeights) == 8 * w_fields.count(";")
+    assert [f[0] for f in _lib.MoeDesc._fields_] == re.findall(r"([A-Za-z_]+)\s*[,;]", desc_fields)
+
+
+def test_status_strings_and_version(L):
+    import mixture_experts_ffn_07_b200 as moe
+    assert moe.status_string(0) == "ok"
+    assert "timed out" in moe.status_string(moe.MOE_ERR_TIMEOUT)
+    assert "sm_100a" in moe.version()
+
+
+def test_workspace_bytes_host_only():
+    import mixture_experts_ffn_07_b200 as moe
+    d = moe.Desc(T=512, H=2048, E=64, I=1024, top_k=8)
+    n = moe.workspace_bytes(d)
+    P = 512 * 8
+    # routing + permutation + slots [P,H] f32 + gathered rows [P,H] bf16 + h [P,I] bf16
+    assert n >= P * 2048 * 4 + P * 2048 * 2 + P * 1024 * 2
+    assert n % 256 == 0
+    d2 = moe.Desc(T=1024, H=2048, E=64, I=1024, top_k=8)
+    d3 = moe.Desc(T=1536, H=2048, E=64, I=1024, top_k=8)
+    a, b, c = n, moe.workspace_bytes(d2), moe.workspace_bytes(d3)
+    assert abs((c - b) - (b - a)) <= 256 * 16      # affine in T up to region alignment
+    assert moe.workspace_bytes(moe.Desc(T=1, H=33, E=4, I=32, top_k=1)) == 0   # invalid -> 0
+
+
+@pytest.mark.parametrize("bad", [dict(E=0), dict(E=257), dict(top_k=0), dict(top_k=33, E=64), dict(top_k=5, E=4),
+                                 dict(T=-1), dict(H=0), dict(act=7), dict(renormalize=2), dict(act_dtype=2),
+                                 dict(w_dtype=5), dict(T=(1 << 20) + 1)])
+def test_invalid_descriptor_rejected_before_cuda(bad):
+    import mixture_experts_ffn_07_b200 as moe
+    from mixture_experts_ffn_07_b200 import _lib
+    d = _lib.MoeDesc(8, 64, 4, 64, 2, 0, 1, 1, 1, 1, 0, 0, 0)
+    for k, v in bad.items():
+        setattr(d, k, v)
+    w = _lib.MoeWeights()
+    rc = _lib.lib().moe_layer(ctypes.byref(d), None, ctypes.byref(w), None, None, 0, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+
+
+def test_unsupported_sizes_and_bad_pointers():
+    import mixture_experts_ffn_07_b200 as moe
+    from mixture_experts_ffn_07_b200 import _lib
+    L = _lib.lib()
+    d = _lib.MoeDesc(8, 48, 4, 64, 2, 0, 1, 1, 1, 1, 0, 0, 0)           # H not a multiple of 32
+    w = _lib.MoeWeights()
+    assert L.moe_layer(ctypes.byref(d), None, ctypes.byref(w), None, None, 0, None) == moe.MOE_ERR_UNSUPPORTED
+    d.H = 64
+    assert L.moe_layer(ctypes.byref(d), None, ctypes.byref(w), None, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    # misaligned x pointer (not 16-byte aligned) is rejected on the host
+    w.router = 0x1000
+    w.gate = w.up = w.down = 0x2000
+    assert L.moe_route(ctypes.byref(d), 0x1001, ctypes.byref(w), 0x3000, 0x4000, 0x5000, None, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    # workspace too small
+    assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, 16, None) == moe.MOE_ERR_WORKSPACE
+    # out aliasing x
+    assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x1000, 0x7000, 1 << 30, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    # Q8_0 without scale planes
+    d.w_dtype = moe.MOE_Q8_0
+    assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, 1 << 30, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_q8_0_split(None, 4, 48, None, None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op_without_cuda():
+    import mixture_experts_ffn_07_b200 as moe
+    from mixture_experts_ffn_07_b200 import _lib
+    d = _lib.MoeDesc(0, 64, 4, 64, 2, 0, 1, 1, 1, 1, 0, 0, 0)
+    w = _lib.MoeWeights(router=0x1000, gate=0x2000, up=0x2000, down=0x2000)
+    ws = moe.workspace_bytes(moe.Desc(T=0, H=64, E=4, I=64, top_k=2))
+    assert _lib.lib().moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, max(ws, 256), None) == \
+        moe.MOE_OK

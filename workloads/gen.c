@@ -14,12 +14,13 @@
  *   key(seed, s)    = mix64(seed + (s + 1) * GAMMA)
  *   bits(key, n)    = mix64(key + (n + 1) * GAMMA)
  *   uniform01(a)    = ((a >> 11) + 0.5) * 2^-53            in (0, 1)
- *   normal(i)       = sqrt(-2 ln u1) * cos(2 pi u2)        (Box-Muller, cosine
- *                     branch only), u1 = uniform01(bits(key, 2i)),
- *                     u2 = uniform01(bits(key, 2i + 1))
+ *   normal(2j)      = sqrt(-2 ln u1) * cos(2 pi u2)        (Box-Muller: both
+ *   normal(2j + 1)  = sqrt(-2 ln u1) * sin(2 pi u2)         outputs of pair j),
+ *                     u1 = uniform01(bits(key, 2j)), u2 = uniform01(bits(key, 2j + 1))
  * Samples are computed in double and rounded once to f32; bf16 and fp16 values
  * are then rounded to nearest-even from that f32 sample.
  */
+#define _GNU_SOURCE
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -42,11 +43,16 @@ static inline double uniform01(uint64_t key, uint64_t n) {
   return ((double)(a >> 11) + 0.5) * (1.0 / 9007199254740992.0);
 }
 
-static inline double normal_at(uint64_t key, uint64_t i) {
+/* Both Box-Muller outputs of pair j: z[0] = element 2j, z[1] = element 2j + 1. */
+static inline void normal_pair(uint64_t key, uint64_t j, double* z) {
   const double two_pi = 6.283185307179586476925286766559;
-  double u1 = uniform01(key, 2 * i);
-  double u2 = uniform01(key, 2 * i + 1);
-  return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
+  double u1 = uniform01(key, 2 * j);
+  double u2 = uniform01(key, 2 * j + 1);
+  double r = sqrt(-2.0 * log(u1));
+  double s, c;
+  sincos(two_pi * u2, &s, &c);
+  z[0] = r * c;
+  z[1] = r * s;
 }
 
 /* f32 -> bf16, round to nearest even (finite inputs only; NaN kept quiet). */
@@ -69,15 +75,24 @@ static inline uint16_t f32_to_f16_rne(float f) {
 void gen_normal_f32(uint64_t seed, uint64_t stream, double mean, double std, int64_t n, float* out) {
   uint64_t key = stream_key(seed, stream);
 #pragma omp parallel for schedule(static)
-  for (int64_t i = 0; i < n; ++i) out[i] = (float)(mean + std * normal_at(key, (uint64_t)i));
+  for (int64_t j = 0; j < (n + 1) / 2; ++j) {
+    double z[2];
+    normal_pair(key, (uint64_t)j, z);
+    out[2 * j] = (float)(mean + std * z[0]);
+    if (2 * j + 1 < n) out[2 * j + 1] = (float)(mean + std * z[1]);
+  }
 }
 
 /* n samples of N(mean, std): f32 sample, then bf16 (RNE) bit patterns. */
 void gen_normal_bf16(uint64_t seed, uint64_t stream, double mean, double std, int64_t n, uint16_t* out) {
   uint64_t key = stream_key(seed, stream);
 #pragma omp parallel for schedule(static)
-  for (int64_t i = 0; i < n; ++i)
-    out[i] = f32_to_bf16_rne((float)(mean + std * normal_at(key, (uint64_t)i)));
+  for (int64_t j = 0; j < (n + 1) / 2; ++j) {
+    double z[2];
+    normal_pair(key, (uint64_t)j, z);
+    out[2 * j] = f32_to_bf16_rne((float)(mean + std * z[0]));
+    if (2 * j + 1 < n) out[2 * j + 1] = f32_to_bf16_rne((float)(mean + std * z[1]));
+  }
 }
 
 /* n samples of U[lo, hi) as f32. */
