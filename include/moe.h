@@ -21,8 +21,8 @@
  *    past its time limit) do not trap: kernels record a status word that
  *    moe_last_device_status() reads.
  *  - Limits: 1 <= E <= 256, 1 <= K <= min(E, 32), H, I and Is multiples of 32,
- *    T <= 2^20.  T == 0 is valid and does nothing.  Every tensor pointer must
- *    be 16-byte aligned.  Outputs may not alias inputs.
+ *    T <= 2^20.  T == 0 is valid and does nothing (pointers may then be NULL).
+ *    Every tensor pointer must be 16-byte aligned.  Outputs may not alias inputs.
  *  - The library keeps no per-call state; it is safe to call from several host
  *    threads on different streams.
  *

@@ -339,10 +339,10 @@ moe_status moe_route(const moe_desc* d, const void* x, const moe_weights* w, flo
                      float* topk_w, float* shared_gate, moe_stream_t stream) {
   moe_status st = check_desc(d);
   if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
   if ((st = check_router_args(*d, x, w)) != MOE_OK) return st;
   if (!logits || !topk_ids || !topk_w || !aligned16(logits)) return MOE_ERR_INVALID_ARG;
   if (shared_gated(*d) && !shared_gate) return MOE_ERR_INVALID_ARG;
-  if (d->T == 0) return MOE_OK;
   moe::Ctx c;
   if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
   return route_impl(c, *d, x, *w, logits, topk_ids, topk_w, shared_gate);
@@ -352,6 +352,7 @@ moe_status moe_permute(const moe_desc* d, const int32_t* topk_ids, int32_t* coun
                        int32_t* sorted_pairs, int32_t* pair_pos, moe_stream_t stream) {
   moe_status st = check_desc(d);
   if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
   if (!topk_ids || !counts || !offsets || !sorted_pairs || !pair_pos) return MOE_ERR_INVALID_ARG;
   moe::Ctx c;
   if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
@@ -363,13 +364,13 @@ moe_status moe_expert_ffn(const moe_desc* d, const void* x, const moe_weights* w
                           size_t ws_bytes, moe_stream_t stream) {
   moe_status st = check_desc(d);
   if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
   if ((st = check_expert_weights(*d, w)) != MOE_OK) return st;
   if (!x || !aligned16(x) || !offsets || !sorted_pairs || !topk_w || !y_slots || !aligned16(y_slots))
     return MOE_ERR_INVALID_ARG;
   const Layout L = layout_of(*d);
   if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
-  if (d->T == 0) return MOE_OK;
   moe::Ctx c;
   if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
   return expert_impl(c, *d, x, *w, offsets, sorted_pairs, topk_w, y_slots, ws, L);
@@ -379,6 +380,7 @@ moe_status moe_combine(const moe_desc* d, const float* y_slots, const void* x, c
                        const float* shared_gate, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = check_desc(d);
   if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
   if (!y_slots || !out || !aligned16(y_slots) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (d->shared_I > 0) {
     if ((st = check_shared_weights(*d, w)) != MOE_OK) return st;
@@ -388,7 +390,6 @@ moe_status moe_combine(const moe_desc* d, const float* y_slots, const void* x, c
   const Layout L = layout_of(*d);
   if (d->shared_I > 0 && (!ws || ws_bytes < L.total)) return MOE_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return MOE_ERR_INVALID_ARG;
-  if (d->T == 0) return MOE_OK;
   moe::Ctx c;
   if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
   return combine_impl(c, *d, y_slots, x, *w, shared_gate, out, ws, L);
@@ -398,6 +399,7 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
                      moe_stream_t stream) {
   moe_status st = check_desc(d);
   if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
   if ((st = check_router_args(*d, x, w)) != MOE_OK) return st;
   if ((st = check_expert_weights(*d, w)) != MOE_OK) return st;
   if ((st = check_shared_weights(*d, w)) != MOE_OK) return st;
@@ -405,7 +407,6 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
   const Layout L = layout_of(*d);
   if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
-  if (d->T == 0) return MOE_OK;
   moe::Ctx c;
   if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
   float* logits = at<float>(ws, L.logits);
@@ -426,6 +427,7 @@ moe_status moe_layer_host(const moe_desc* d, const void* x_host, const moe_weigh
                           void* out_dev, void* ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = check_desc(d);
   if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
   if (!x_host || !out_host || !x_dev || !out_dev) return MOE_ERR_INVALID_ARG;
   const size_t bytes = static_cast<size_t>(d->T) * d->H * (d->act_dtype == MOE_F32 ? 4 : 2);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
