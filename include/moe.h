@@ -183,6 +183,29 @@ moe_status moe_layer_host(const moe_desc* d, const void* x_host, const moe_weigh
                           void* out_dev, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_layer for callers that cannot allocate device memory when they call the
+ * layer: for example a host whose HBM is already handed out to its own pool,
+ * code that must not pay cudaMalloc's implicit device synchronisation, or a
+ * plain C caller with no allocator at hand.  The pages have no counterpart of
+ * this entry point; it exists for such callers only.
+ *
+ * Same inputs, outputs and results as moe_layer, but the scratch is a static
+ * device array of MOE_NOALLOC_SCRATCH_BYTES (32 MiB) inside libmoe, present on
+ * every GPU that loads the library until the process exits; nothing is
+ * allocated or freed.  Descriptors with moe_workspace_bytes(d) above that size
+ * are rejected with MOE_ERR_WORKSPACE before anything is launched (every
+ * decode batch, T <= 64, of the layer shapes this library is measured on fits).
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.  All calls
+ * share the one array and it keeps the previous call's contents (nothing in
+ * it has to start at zero: each call writes every region before reading it),
+ * so calls that can overlap on the GPU -- other streams, other host threads --
+ * race on it: serialise them.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (32u << 20)
+moe_status moe_layer_noalloc(const moe_desc* d, const void* x, const moe_weights* w, void* out, moe_stream_t stream);
+
+/*
  * Split GGML Q8_0 blocks ({fp16 d; int8 q[32]}, 34 bytes, along the input
  * dimension) of a [rows, cols] matrix into int8 quants [rows, cols] and fp16
  * scales [rows, cols/32], the form moe_weights expects for MOE_Q8_0.  A

@@ -124,6 +124,16 @@ def layer(desc, x, w, out, ws, stream=None):
                                _stream(stream)), "moe_layer")
 
 
+def layer_noalloc(desc, x, w, out, stream=None):
+    """moe_layer with the library's static 32 MiB device scratch: for callers that cannot allocate.
+
+    Calls that may overlap on the GPU share that scratch and race; the first call on a device
+    looks up its address and should come before any stream capture."""
+    d, cw = desc.c(), w.c()
+    check(_lib.lib().moe_layer_noalloc(ctypes.byref(d), _ptr(x), ctypes.byref(cw), _ptr(out), _stream(stream)),
+          "moe_layer_noalloc")
+
+
 def layer_host(desc, x_host, w, out_host, x_dev, out_dev, ws, stream=None):
     """moe_layer with host x/out (pinned torch CPU tensors); copies are enqueued on `stream`."""
     d, cw = desc.c(), w.c()

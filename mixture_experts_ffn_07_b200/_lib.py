@@ -15,13 +15,14 @@ LIB_PATH = os.path.join(HERE, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
     MOE_ERR_DEVICE_INDEX = range(7)
 MOE_F32, MOE_BF16, MOE_Q8_0 = 0, 1, 2
+MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 MOE_ACT_SILU, MOE_ACT_GELU_TANH = 0, 1
 
 # every symbol include/moe.h declares
 EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
-           "moe_combine", "moe_layer", "moe_layer_host", "moe_q8_0_split", "moe_last_device_status",
-           "moe_launch_count", "moe_trace_enable", "moe_trace_read", "moe_debug_set_wait_limit",
-           "moe_debug_set_skip_stage")
+           "moe_combine", "moe_layer", "moe_layer_host", "moe_layer_noalloc", "moe_q8_0_split",
+           "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
+           "moe_debug_set_wait_limit", "moe_debug_set_skip_stage")
 
 
 class MoeDesc(ctypes.Structure):
@@ -64,10 +65,11 @@ def lib():
         L.moe_combine.argtypes = [DP, P, P, WP, P, P, P, S, P]
         L.moe_layer.argtypes = [DP, P, WP, P, P, S, P]
         L.moe_layer_host.argtypes = [DP, P, WP, P, P, P, P, S, P]
+        L.moe_layer_noalloc.argtypes = [DP, P, WP, P, P]
         L.moe_q8_0_split.argtypes = [P, I64, I64, P, P, P]
         L.moe_last_device_status.argtypes = [P]
         for f in (L.moe_route, L.moe_permute, L.moe_expert_ffn, L.moe_combine, L.moe_layer, L.moe_layer_host,
-                  L.moe_q8_0_split, L.moe_last_device_status):
+                  L.moe_layer_noalloc, L.moe_q8_0_split, L.moe_last_device_status):
             f.restype = I32
         L.moe_launch_count.restype = ctypes.c_uint64
         L.moe_trace_enable.argtypes = [I32]

@@ -478,6 +478,38 @@ int moe_trace_read(const char** names, float* ms, int max) {
   return g_trace_n;
 }
 
+// ---------------------------------------------------------------- moe_layer without allocation
+// The scratch of moe_layer_noalloc.  In host code this name is only a stand-in
+// for the device symbol; the kernels get the address that cudaGetSymbolAddress
+// returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+static void* g_noalloc_addr[kMaxDevices];
+static std::mutex g_noalloc_mu;
+
+// Device address of the static scratch on the current device, looked up once per device.
+static void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = p;
+  }
+  return g_noalloc_addr[dev];
+}
+
+moe_status moe_layer_noalloc(const moe_desc* d, const void* x, const moe_weights* w, void* out,
+                             moe_stream_t stream) {
+  moe_status st = check_desc(d);
+  if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
+  if (layout_of(*d).total > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  void* ws = noalloc_scratch();
+  if (!ws) return MOE_ERR_CUDA;
+  return moe_layer(d, x, w, out, ws, MOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 void moe_debug_set_wait_limit(int64_t cycles) { g_wait_limit.store(cycles > 0 ? cycles : (1LL << 31)); }
 
 void moe_debug_set_skip_stage(int enable) { g_skip_stage.store(enable ? 1 : 0); }
