@@ -105,9 +105,10 @@ const char* moe_status_string(moe_status s);
 const char* moe_version(void);
 
 /*
- * Bytes of caller-provided device workspace moe_layer needs for `d` (affine in
- * T for fixed sizes; 256-byte aligned regions).  Returns 0 for an invalid
- * descriptor.  moe_expert_ffn and moe_combine need no more than this.
+ * Bytes of caller-provided device workspace moe_layer needs for `d`: linear in
+ * T for fixed sizes, plus the bf16 router's split-K partial logits (at most
+ * 20480*E*4 bytes), in 256-byte aligned regions.  Returns 0 for an invalid
+ * descriptor.  moe_route, moe_expert_ffn and moe_combine need no more than this.
  */
 size_t moe_workspace_bytes(const moe_desc* d);
 
@@ -120,9 +121,14 @@ size_t moe_workspace_bytes(const moe_desc* d);
  *  topk_ids [T,K] int32 out: experts in order (logit desc, index asc)
  *  topk_w   [T,K] f32 out: exp(l - m) over the selected (renormalised) or over all E
  *  shared_gate [T] f32 out: sigmoid(w_s . x); required iff shared_I > 0 and has_shared_gate
+ *  ws, ws_bytes: optional workspace (NULL, or >= moe_workspace_bytes(d)).  With it,
+ *           a bf16 batch splits the logits GEMM over the hidden dimension into
+ *           partial sums added in a fixed order (the split moe_layer uses, so the
+ *           logits, and hence the selection, are identical to moe_layer's);
+ *           without it the GEMM is not split.
  */
 moe_status moe_route(const moe_desc* d, const void* x, const moe_weights* w, float* logits, int32_t* topk_ids,
-                     float* topk_w, float* shared_gate, moe_stream_t stream);
+                     float* topk_w, float* shared_gate, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Histogram, exclusive scan and stable permutation of the P pairs by expert

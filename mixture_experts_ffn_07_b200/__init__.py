@@ -93,10 +93,10 @@ def workspace_bytes(desc: Desc) -> int:
     return _lib.lib().moe_workspace_bytes(ctypes.byref(d))
 
 
-def route(desc, x, w, logits, topk_ids, topk_w, shared_gate=None, stream=None):
+def route(desc, x, w, logits, topk_ids, topk_w, shared_gate=None, ws=None, stream=None):
     d, cw = desc.c(), w.c()
     check(_lib.lib().moe_route(ctypes.byref(d), _ptr(x), ctypes.byref(cw), _ptr(logits), _ptr(topk_ids),
-                               _ptr(topk_w), _ptr(shared_gate), _stream(stream)), "moe_route")
+                               _ptr(topk_w), _ptr(shared_gate), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_route")
 
 
 def permute(desc, topk_ids, counts, offsets, sorted_pairs, pair_pos, stream=None):

@@ -59,7 +59,7 @@ def lib():
         L.moe_version.restype = ctypes.c_char_p
         L.moe_workspace_bytes.argtypes = [DP]
         L.moe_workspace_bytes.restype = S
-        L.moe_route.argtypes = [DP, P, WP, P, P, P, P, P]
+        L.moe_route.argtypes = [DP, P, WP, P, P, P, P, P, S, P]
         L.moe_permute.argtypes = [DP, P, P, P, P, P, P]
         L.moe_expert_ffn.argtypes = [DP, P, WP, P, P, P, P, P, S, P]
         L.moe_combine.argtypes = [DP, P, P, WP, P, P, P, S, P]

@@ -10,6 +10,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "../../include/moe.h"
 
@@ -22,7 +23,32 @@ struct Ctx {
   int num_sms;
   long long wait_limit;    // SM cycles a pipeline wait may spin before giving up
   int skip_stage;          // debug: grouped-GEMM producer skips one stage's loads
+  int pdl;                 // launch with programmatic stream serialization
 };
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per (kernel, device).
+cudaError_t allow_dynamic_smem(const void* kernel, int bytes);
+
+// Launch `kernel` on ctx.stream.  With ctx.pdl the launch may start while the
+// previous kernel on the stream is still running: every kernel here calls
+// pdl_wait() before it reads anything an earlier kernel wrote, and
+// pdl_trigger() once all of its CTAs have started.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(const Ctx& c, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = c.pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 // Marks one kernel launch for the launch counter and the optional event trace.
 struct KernelScope {
@@ -52,6 +78,11 @@ __device__ __forceinline__ void record_status(int* status, int code) {
 }
 
 // ---------------------------------------------------------------- PTX wrappers
+// Programmatic dependent launch: wait for the grids this one depends on (and
+// their memory), and allow the next grid on the stream to be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

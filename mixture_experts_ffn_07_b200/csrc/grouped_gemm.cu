@@ -12,21 +12,22 @@
 //  * persistent grid, one CTA per SM; work items (group, n-tile, m-tile) with
 //    the m-tile fastest so CTAs running at the same time share weight tiles
 //    in L2;
-//  * warp 0: TMA producer (one lane) into a 4-stage shared-memory ring of
-//    128x64 A tiles and 256x64 B tiles, 128-byte swizzle;
-//  * warp 1: allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=256,
+//  * warp 0: TMA producer (one lane) into a shared-memory ring of 128x64 A
+//    tiles and BNx64 B tiles, 128-byte swizzle (6 stages at BN = 128, 4 at 256);
+//  * warp 1: allocates 2*BN TMEM columns and issues tcgen05.mma (M=128, N=BN,
 //    K=16, bf16 in, f32 accumulate) from one lane; two accumulators so the
 //    epilogue of one tile overlaps the main loop of the next;
 //  * warps 2-5: epilogue, one TMEM lane (= output row) per thread;
-//  * dual mode (gate/up): the 256-row B tile is 128 rows of W_gate followed
-//    by the same 128 rows of W_up, so TMEM columns [0,128) hold x W_gate^T and
-//    [128,256) hold x W_up^T for the same outputs; the epilogue writes
+//  * dual mode (gate/up): the BN-row B tile is BN/2 rows of W_gate followed
+//    by the same BN/2 rows of W_up, so TMEM columns [0,BN/2) hold x W_gate^T and
+//    [BN/2,BN) hold x W_up^T for the same outputs; the epilogue writes
 //    act(g) * u as bf16;
 //  * single mode (down, router): the epilogue scales row r by row_scale and
 //    stores it at row row_map[r] in f32 (the slot row of the pair).
 //  * every mbarrier wait is bounded; on expiry the CTA records
 //    MOE_ERR_TIMEOUT, lets in-flight copies and MMAs land, frees TMEM and exits.
 #include <algorithm>
+#include <cmath>
 
 #include "kernels.h"
 
@@ -36,15 +37,21 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int BN_MMA = 256;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN_MMA * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr uint32_t TMEM_COLS = 2 * BN_MMA;
 constexpr int MAX_G = 256;
 constexpr int THREADS = 192;
 
+// Tile shape per instantiation: the MMA is M=128 x N=BN; the ring holds STAGES
+// (A 128x64, B BNx64) stage pairs, ~192 KB either way.
+template <int BN>
+struct Tile {
+  static constexpr int STAGES = BN == 128 ? 6 : 4;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+};
+
+template <int STAGES>
 struct Aux {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -58,11 +65,17 @@ struct Aux {
   int cnt[MAX_G];
 };
 
-constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(Aux);
+template <int BN>
+constexpr size_t smem_bytes() {
+  return 1024 + static_cast<size_t>(Tile<BN>::STAGES) * Tile<BN>::STAGE_BYTES + sizeof(Aux<Tile<BN>::STAGES>);
+}
 
 struct KParams {
   const int32_t* offsets;
   int G;
+  int ksplit;          // K ranges per output tile (plain f32 mode only)
+  int kb_per_split;    // k-blocks per range
+  size_t part_stride;  // elements between the f32 outputs of consecutive ranges
   int rows_single;
   int N;
   int Kdim;
@@ -86,7 +99,9 @@ __device__ __forceinline__ bool wait_cycles(uint64_t* bar, uint32_t parity, long
   return true;
 }
 
-__device__ __forceinline__ void decode_item(const Aux& aux, int G, int w, int& g, int& mt, int& nt) {
+template <typename AuxT>
+__device__ __forceinline__ void decode_item(const AuxT& aux, int G, int ksplit, int w, int& g, int& mt, int& nt,
+                                            int& ks) {
   int lo = 0, hi = G - 1;  // largest g with item_off[g] <= w
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -98,8 +113,10 @@ __device__ __forceinline__ void decode_item(const Aux& aux, int G, int w, int& g
   g = lo;
   const int tiles = (aux.cnt[g] + BM - 1) / BM;
   const int local = w - aux.item_off[g];
-  nt = local / tiles;
-  mt = local - nt * tiles;
+  ks = local % ksplit;
+  const int rest = local / ksplit;
+  nt = rest / tiles;
+  mt = rest - nt * tiles;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -107,22 +124,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <bool DUAL>
+template <bool DUAL, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                         const __grid_constant__ CUtensorMap mapB1, const KParams p) {
+  constexpr int STAGES = Tile<BN>::STAGES;
+  constexpr int STAGE_BYTES = Tile<BN>::STAGE_BYTES;
+  constexpr int B_BYTES = Tile<BN>::B_BYTES;
+  constexpr uint32_t TMEM_COLS = Tile<BN>::TMEM_COLS;
+  constexpr int BN_MMA = BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Aux& aux = *reinterpret_cast<Aux*>(smem + STAGES * STAGE_BYTES);
+  Aux<STAGES>& aux = *reinterpret_cast<Aux<STAGES>*>(smem + STAGES * STAGE_BYTES);
   volatile int* abort_flag = &aux.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int g = threadIdx.x; g < p.G; g += THREADS) {
-    const int r0 = p.offsets ? p.offsets[g] : 0;
-    const int r1 = p.offsets ? p.offsets[g + 1] : p.rows_single;
-    aux.row_off[g] = r0;
-    aux.cnt[g] = max(0, r1 - r0);
-  }
+  // prologue that reads nothing earlier kernels write: overlaps their tail under programmatic launch
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&aux.full[s], 1);
@@ -135,6 +152,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&aux.done, 1);
     aux.abort = 0;
     fence_mbar_init();
+  } else if (threadIdx.x == 32) {
+    prefetch_tensormap(&mapA);
+    prefetch_tensormap(&mapB0);
+    if (DUAL) prefetch_tensormap(&mapB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(&aux.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  pdl_wait();
+  for (int g = threadIdx.x; g < p.G; g += THREADS) {
+    const int r0 = p.offsets ? p.offsets[g] : 0;
+    const int r1 = p.offsets ? p.offsets[g + 1] : p.rows_single;
+    aux.row_off[g] = r0;
+    aux.cnt[g] = max(0, r1 - r0);
   }
   __syncthreads();
   if (warp == 0) {  // exclusive scan of work items per group; lane owns groups [8*lane, 8*lane+8)
@@ -142,7 +175,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int g = lane * 8 + i;
-      v[i] = g < p.G ? ((aux.cnt[g] + BM - 1) / BM) * p.n_tiles : 0;
+      v[i] = g < p.G ? ((aux.cnt[g] + BM - 1) / BM) * p.n_tiles * p.ksplit : 0;
       local += v[i];
     }
     int incl = local;
@@ -159,9 +192,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       run += v[i];
     }
     if (lane == 31) aux.item_off[p.G] = incl;
-  } else if (warp == 1) {
-    tmem_alloc(&aux.tmem_base, TMEM_COLS);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -175,17 +205,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
-      prefetch_tensormap(&mapA);
-      prefetch_tensormap(&mapB0);
-      if (DUAL) prefetch_tensormap(&mapB1);
       uint32_t kbg = 0, outstanding = 0, out_phase = 0;
       bool skipped = false;
       for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
-        int g, mt, nt;
-        decode_item(aux, p.G, w, g, mt, nt);
+        int g, mt, nt, ks;
+        decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
         const int a_row = aux.row_off[g] + mt * BM;
         const int b_row = g * p.N + nt * p.col_step;
-        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+        const int kb0 = ks * p.kb_per_split, kb1 = min(nkb, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
           const int s = kbg % STAGES;
           const uint32_t ph = (kbg / STAGES) & 1u;
           if (!mbar_wait_bounded(&aux.empty[s], ph ^ 1u, limit, abort_flag)) break;
@@ -220,13 +248,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t kbg = 0;
       int it = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+        int g, mt, nt, ks;
+        decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
+        const int kb0 = ks * p.kb_per_split, kb1 = min(nkb, kb0 + p.kb_per_split);
         const int acc = it & 1;
         const uint32_t acc_ph = (it >> 1) & 1u;
         if (!mbar_wait_bounded(&aux.tempty[acc], acc_ph ^ 1u, limit, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN_MMA;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+        for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
           const int s = kbg % STAGES;
           const uint32_t ph = (kbg / STAGES) & 1u;
           if (!mbar_wait_bounded(&aux.full[s], ph, limit, abort_flag)) {
@@ -240,7 +271,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                      (kb | kk) != 0 ? 1u : 0u);
+                      (kb > kb0 || kk > 0) ? 1u : 0u);
           umma_commit(&aux.empty[s]);
         }
         if (!ok) break;
@@ -255,8 +286,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int r = q * 32 + lane;
     int it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-      int g, mt, nt;
-      decode_item(aux, p.G, w, g, mt, nt);
+      int g, mt, nt, ks;
+      decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
       const int acc = it & 1;
       const uint32_t acc_ph = (it >> 1) & 1u;
       // every lane waits; the outcome is made warp-uniform because the TMEM loads below are .sync.aligned
@@ -306,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld_32x32b_x32(tbase + c, v);
           tmem_ld_wait();
           if (dest >= 0 && col0 + c < p.N) {
-            float* dst = p.out_f32 + static_cast<size_t>(dest) * p.N + col0 + c;
+            float* dst = p.out_f32 + ks * p.part_stride + static_cast<size_t>(dest) * p.N + col0 + c;
             if (col0 + c + 32 <= p.N) {
               float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
@@ -364,29 +395,15 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool DUAL>
-cudaError_t set_smem_attr() {
-  static int done_mask = 0;  // bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 31 && (done_mask & (1 << dev))) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(SMEM_BYTES));
-  if (e == cudaSuccess && dev < 31) done_mask |= 1 << dev;
-  return e;
-}
-
-}  // namespace
-
-cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
-  if (a.G <= 0 || a.max_rows <= 0 || a.N <= 0 || a.rows_A <= 0) return cudaSuccess;
-  if (a.G > MAX_G) return cudaErrorInvalidValue;
+template <bool DUAL, int BN>
+cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int max_items_per_sm_hint) {
+  (void)max_items_per_sm_hint;
   CUtensorMap mA, mB0, mB1;
-  const uint32_t brows = a.dual ? BN_MMA / 2 : BN_MMA;
+  const uint32_t brows = DUAL ? BN / 2 : BN;
   if (!make_map(&mA, a.A, static_cast<uint64_t>(a.rows_A), static_cast<uint64_t>(a.Kdim), BM) ||
       !make_map(&mB0, a.B0, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), brows))
     return cudaErrorInvalidValue;
-  if (a.dual) {
+  if (DUAL) {
     if (!make_map(&mB1, a.B1, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), brows))
       return cudaErrorInvalidValue;
   } else {
@@ -395,10 +412,14 @@ cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   KParams p;
   p.offsets = a.offsets;
   p.G = a.G;
+  const int nkb = (a.Kdim + BK - 1) / BK;
+  p.ksplit = effective_ksplit(a.ksplit, a.Kdim);
+  p.kb_per_split = (nkb + p.ksplit - 1) / p.ksplit;
+  p.part_stride = a.part_stride;
   p.rows_single = static_cast<int>(a.rows_A);
   p.N = a.N;
   p.Kdim = a.Kdim;
-  p.col_step = a.dual ? BN_MMA / 2 : BN_MMA;
+  p.col_step = DUAL ? BN / 2 : BN;
   p.n_tiles = (a.N + p.col_step - 1) / p.col_step;
   p.act = a.act;
   p.out_bf16 = a.out_bf16;
@@ -409,16 +430,43 @@ cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   p.wait_limit = c.wait_limit;
   p.skip_stage = c.skip_stage;
   const long long tiles_bound = static_cast<long long>(a.max_rows) / BM + std::min(a.G, a.max_rows);
-  const long long items_bound = tiles_bound * p.n_tiles;
+  const long long items_bound = tiles_bound * p.n_tiles * p.ksplit;
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(c.num_sms, items_bound)));
-  cudaError_t e = a.dual ? set_smem_attr<true>() : set_smem_attr<false>();
+  auto kern = grouped_gemm_kernel<DUAL, BN>;
+  const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem_bytes<BN>()));
   if (e != cudaSuccess) return e;
-  KernelScope ks(c, a.name ? a.name : (a.dual ? "grouped_gemm_dual" : "grouped_gemm"));
-  if (a.dual)
-    grouped_gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, c.stream>>>(mA, mB0, mB1, p);
-  else
-    grouped_gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, c.stream>>>(mA, mB0, mB1, p);
-  return cudaGetLastError();
+  KernelScope ks(c, a.name ? a.name : (DUAL ? "grouped_gemm_dual" : "grouped_gemm"));
+  return launch_kernel(c, kern, dim3(grid), dim3(THREADS), smem_bytes<BN>(), mA, mB0, mB1, p);
+}
+
+}  // namespace
+
+// Tail of the last wave when `items` equal work items run on `sms` persistent CTAs.
+double wave_waste(double items, int sms) {
+  const double waves = items / sms;
+  const double full = std::ceil(waves);
+  return full > 0 ? (full - waves) / full : 0.0;
+}
+
+// Narrow tiles (N = 128) for weight-streaming (memory-bound) shapes whose last
+// wave would leave many SMs idle with wide tiles; wide tiles (N = 256) for
+// compute-bound shapes, where they halve the A-tile traffic per flop.
+cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
+  if (a.G <= 0 || a.max_rows <= 0 || a.N <= 0 || a.rows_A <= 0) return cudaSuccess;
+  if (a.G > MAX_G) return cudaErrorInvalidValue;
+  const int groups = std::min(a.G, a.max_rows);
+  const double rows_per_group = static_cast<double>(a.max_rows) / groups;
+  // about half an M tile of padding per group
+  const double tiles = static_cast<double>(a.max_rows) / BM + 0.5 * groups;
+  const double cols_wide = a.dual ? 128.0 : 256.0;
+  const double items_wide = tiles * std::ceil(a.N / cols_wide);
+  const double items_narrow = tiles * std::ceil(a.N / (cols_wide / 2));
+  // weights are streamed once per group; rows per group sets flops per weight byte (ridge ~200)
+  const bool memory_bound = rows_per_group < 200.0;
+  const bool narrow =
+      memory_bound && wave_waste(items_wide, c.num_sms) - wave_waste(items_narrow, c.num_sms) > 0.03;
+  if (a.dual) return narrow ? launch_tiled<true, 128>(c, a, 0) : launch_tiled<true, 256>(c, a, 0);
+  return narrow ? launch_tiled<false, 128>(c, a, 0) : launch_tiled<false, 256>(c, a, 0);
 }
 
 }  // namespace moe

@@ -7,17 +7,20 @@
 
 namespace moe {
 
-// Router logits on CUDA cores: logits[t, r] = x[t] . W[r] for rows r in
-// [0, E) of the router and, when w_s != nullptr, shared_gate[t] =
-// sigmoid(x[t] . w_s).  rows_from_router = false computes only the w_s row.
-cudaError_t launch_router_logits(const Ctx& c, const void* x, int x_dtype, const void* W, const void* w_s,
-                                 int w_dtype, int T, int H, int E, bool rows_from_router, float* logits,
-                                 float* shared_gate);
+// Softmax + top-K (+renorm) per token from logits in global memory, one warp
+// per token.  Adds the optional bias to the logits in place; with w_s also
+// writes shared_gate[t] = sigmoid(w_s . x[t]).
+// `nparts` partial logit arrays of T*E floats, part_stride apart starting at
+// `parts`, are summed in order into `logits` first.
+cudaError_t launch_router_topk(const Ctx& c, const float* parts, int nparts, size_t part_stride, float* logits,
+                               const float* bias, int T, int E, int K, int renorm, int32_t* ids, float* w,
+                               const void* x, int x_dtype, const void* w_s, int w_dtype, int H, float* shared_gate);
 
-// Softmax + top-K (+renorm) per token, one warp per token.  Adds the optional
-// bias to the logits in place; writes ids and weights.
-cudaError_t launch_router_topk(const Ctx& c, float* logits, const float* bias, int T, int E, int K, int renorm,
-                               int32_t* ids, float* w);
+// Router in one launch for small batches: logits (+ the shared-gate row when
+// w_s != nullptr) by clusters of 8 CTAs, then softmax + top-K (+renorm) per token.
+cudaError_t launch_router_fused(const Ctx& c, const void* x, int x_dtype, const void* W, const void* w_s,
+                                int w_dtype, const float* bias, int T, int H, int E, int K, int renorm,
+                                float* logits, int32_t* ids, float* w, float* shared_gate);
 
 // Single-CTA stable counting sort of the P pair ids by expert.
 cudaError_t launch_permute(const Ctx& c, const int32_t* ids, int P, int E, int32_t* counts, int32_t* offsets,
@@ -50,8 +53,20 @@ struct GemmArgs {
   const int32_t* row_map;
   const float* row_scale;
   const char* name;        // trace label
+  int ksplit = 1;          // single mode without row_map/row_scale only: K split into ranges whose
+  size_t part_stride = 0;  // f32 results go to out_f32 + range * part_stride (summed by the caller)
 };
 cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a);
+
+// The number of K ranges a split request really produces for a reduction of
+// Kdim: at most one per 64-wide k-block, and no empty range.  The caller sums
+// exactly this many partial results.
+inline int effective_ksplit(int requested, int Kdim) {
+  const int nkb = (Kdim + 63) / 64;
+  const int want = std::max(1, std::min(requested, nkb));
+  const int per = (nkb + want - 1) / want;
+  return (nkb + per - 1) / per;
+}
 
 // Weight-streaming expert FFN (any T; f32/bf16 activations, f32/bf16/Q8_0 weights).
 // Groups as above (offsets == nullptr: one group of rows [0, T) with identity rows).

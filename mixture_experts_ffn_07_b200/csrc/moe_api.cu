@@ -8,6 +8,8 @@
 // touched expert's weights once and is the bandwidth-optimal form for small T.
 #include <atomic>
 #include <mutex>
+#include <tuple>
+#include <vector>
 
 #include "kernels.h"
 
@@ -61,6 +63,7 @@ bool make_ctx(cudaStream_t s, moe::Ctx* c) {
   c->stream = s;
   c->wait_limit = g_wait_limit.load();
   c->skip_stage = g_skip_stage.load();
+  c->pdl = 1;
   return true;
 }
 
@@ -72,6 +75,14 @@ bool tensor_path(const moe_desc& d) { return d.act_dtype == MOE_BF16 && d.w_dtyp
 
 bool tensor_router(const moe_desc& d) {
   return d.act_dtype == MOE_BF16 && d.router_dtype == MOE_BF16 && d.T > 64 && d.E % 32 == 0;
+}
+
+// Ranges the router GEMM splits the hidden dimension into, so that small batches
+// still occupy the GPU: about 160 CTAs over the 128-token tiles, at most 16.
+// A function of T alone, so logits do not depend on the device's SM count.
+int router_ksplit(const moe_desc& d) {
+  const int mtiles = (d.T + 127) / 128;
+  return std::max(1, std::min(16, 160 / std::max(1, mtiles)));
 }
 
 bool shared_gated(const moe_desc& d) { return d.shared_I > 0 && d.has_shared_gate; }
@@ -93,7 +104,8 @@ moe_status check_desc(const moe_desc* d) {
 }
 
 struct Layout {
-  size_t logits, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos, y_slots, x_perm, h, h_s, y_s, total;
+  size_t logits, logit_parts, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos, y_slots, x_perm, h, h_s,
+      y_s, total;
 };
 
 Layout layout_of(const moe_desc& d) {
@@ -107,6 +119,7 @@ Layout layout_of(const moe_desc& d) {
   const size_t T = d.T, H = d.H, E = d.E, I = d.I, P = T * d.top_k, Is = d.shared_I;
   const bool tc = tensor_path(d);
   L.logits = take(T * E * 4);
+  L.logit_parts = tensor_router(d) ? take(router_ksplit(d) * T * E * 4) : 0;
   L.ids = take(P * 4);
   L.w = take(P * 4);
   L.shared_gate = take(T * 4);
@@ -137,10 +150,12 @@ moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR
   } while (0)
 
 // ---------------------------------------------------------------- stages
+// parts: scratch for the split-K partial logits (nullptr: no split).
 moe_status route_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const moe_weights& w, float* logits,
-                      int32_t* ids, float* tw, float* shared_gate) {
+                      float* parts, int32_t* ids, float* tw, float* shared_gate) {
   const void* w_s = shared_gated(d) ? w.sh_gate_w : nullptr;
   if (tensor_router(d)) {
+    const int ksplit = parts ? moe::effective_ksplit(router_ksplit(d), d.H) : 1;
     moe::GemmArgs a{};
     a.A = static_cast<const __nv_bfloat16*>(x);
     a.rows_A = d.T;
@@ -150,18 +165,19 @@ moe_status route_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const
     a.G = 1;
     a.max_rows = d.T;
     a.dual = false;
-    a.out_f32 = logits;
+    a.out_f32 = ksplit > 1 ? parts : logits;
+    a.ksplit = ksplit;
+    a.part_stride = static_cast<size_t>(d.T) * d.E;
     a.name = "router_gemm";
     MOE_TRY(moe::launch_grouped_gemm(c, a));
-    if (w_s)
-      MOE_TRY(moe::launch_router_logits(c, x, d.act_dtype, w.router, w_s, d.router_dtype, d.T, d.H, d.E, false,
-                                        logits, shared_gate));
+    MOE_TRY(moe::launch_router_topk(c, parts, ksplit > 1 ? ksplit : 0, a.part_stride, logits,
+                                    d.has_router_bias ? w.router_bias : nullptr, d.T, d.E, d.top_k, d.renormalize, ids,
+                                    tw, x, d.act_dtype, w_s, d.router_dtype, d.H, shared_gate));
   } else {
-    MOE_TRY(moe::launch_router_logits(c, x, d.act_dtype, w.router, w_s, d.router_dtype, d.T, d.H, d.E, true, logits,
-                                      shared_gate));
+    MOE_TRY(moe::launch_router_fused(c, x, d.act_dtype, w.router, w_s, d.router_dtype,
+                                     d.has_router_bias ? w.router_bias : nullptr, d.T, d.H, d.E, d.top_k,
+                                     d.renormalize, logits, ids, tw, shared_gate));
   }
-  MOE_TRY(moe::launch_router_topk(c, logits, d.has_router_bias ? w.router_bias : nullptr, d.T, d.E, d.top_k,
-                                  d.renormalize, ids, tw));
   return MOE_OK;
 }
 
@@ -291,6 +307,19 @@ moe_status check_shared_weights(const moe_desc& d, const moe_weights* w) {
 // ---------------------------------------------------------------- instrumentation
 namespace moe {
 
+cudaError_t allow_dynamic_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::tuple<const void*, int, int>> done;  // (kernel, device, bytes)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  for (const auto& d : done)
+    if (std::get<0>(d) == kernel && std::get<1>(d) == dev && std::get<2>(d) >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.emplace_back(kernel, dev, bytes);
+  return e;
+}
+
 KernelScope::KernelScope(const Ctx& c, const char* name) : ctx(c), slot(-1) {
   g_launches.fetch_add(1);
   std::lock_guard<std::mutex> lk(g_trace_mu);
@@ -336,16 +365,20 @@ size_t moe_workspace_bytes(const moe_desc* d) {
 }
 
 moe_status moe_route(const moe_desc* d, const void* x, const moe_weights* w, float* logits, int32_t* topk_ids,
-                     float* topk_w, float* shared_gate, moe_stream_t stream) {
+                     float* topk_w, float* shared_gate, void* ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = check_desc(d);
   if (st != MOE_OK) return st;
   if (d->T == 0) return MOE_OK;
   if ((st = check_router_args(*d, x, w)) != MOE_OK) return st;
   if (!logits || !topk_ids || !topk_w || !aligned16(logits)) return MOE_ERR_INVALID_ARG;
   if (shared_gated(*d) && !shared_gate) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout_of(*d);
+  if (ws && ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return MOE_ERR_INVALID_ARG;
   moe::Ctx c;
   if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
-  return route_impl(c, *d, x, *w, logits, topk_ids, topk_w, shared_gate);
+  float* parts = (ws && L.logit_parts) ? at<float>(ws, L.logit_parts) : nullptr;
+  return route_impl(c, *d, x, *w, logits, parts, topk_ids, topk_w, shared_gate);
 }
 
 moe_status moe_permute(const moe_desc* d, const int32_t* topk_ids, int32_t* counts, int32_t* offsets,
@@ -416,7 +449,8 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* sorted_pairs = at<int32_t>(ws, L.sorted_pairs);
   float* y_slots = at<float>(ws, L.y_slots);
-  if ((st = route_impl(c, *d, x, *w, logits, ids, tw, sg)) != MOE_OK) return st;
+  float* parts = L.logit_parts ? at<float>(ws, L.logit_parts) : nullptr;
+  if ((st = route_impl(c, *d, x, *w, logits, parts, ids, tw, sg)) != MOE_OK) return st;
   MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, at<int32_t>(ws, L.counts), offsets, sorted_pairs,
                               at<int32_t>(ws, L.pair_pos)));
   if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L)) != MOE_OK) return st;

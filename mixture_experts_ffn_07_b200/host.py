@@ -74,6 +74,7 @@ def run_route(desc, w, x):
     ids = torch.empty((T, K), dtype=torch.int32, device="cuda")
     tw = torch.empty((T, K), dtype=torch.float32, device="cuda")
     sg = torch.empty((max(T, 1),), dtype=torch.float32, device="cuda")
-    route(desc, x, w, logits, ids, tw, sg if desc.has_shared_gate and desc.shared_I else None)
+    ws = torch.empty(max(workspace_bytes(desc), 256), dtype=torch.uint8, device="cuda")
+    route(desc, x, w, logits, ids, tw, sg if desc.has_shared_gate and desc.shared_I else None, ws)
     torch.cuda.synchronize()
     return logits, ids, tw, sg

@@ -60,10 +60,15 @@ def test_workspace_bytes_host_only():
     # routing + permutation + slots [P,H] f32 + gathered rows [P,H] bf16 + h [P,I] bf16
     assert n >= P * 2048 * 4 + P * 2048 * 2 + P * 1024 * 2
     assert n % 256 == 0
-    d2 = moe.Desc(T=1024, H=2048, E=64, I=1024, top_k=8)
-    d3 = moe.Desc(T=1536, H=2048, E=64, I=1024, top_k=8)
-    a, b, c = n, moe.workspace_bytes(d2), moe.workspace_bytes(d3)
-    assert abs((c - b) - (b - a)) <= 256 * 16      # affine in T up to region alignment
+    # affine in T without the tensor-core router; with it, plus at most 20480 * E * 4 bytes of split-K scratch
+    ts = (1024, 2048, 3072, 4096, 8192)
+    plain = [moe.workspace_bytes(moe.Desc(T=t, H=2048, E=64, I=1024, top_k=8, router_dtype="f32")) for t in ts]
+    step = (plain[1] - plain[0]) / 1024
+    for t, sz in zip(ts, plain):
+        assert abs(sz - plain[0] - step * (t - 1024)) <= 256 * 16
+    for t, sz in zip(ts, plain):
+        extra = moe.workspace_bytes(moe.Desc(T=t, H=2048, E=64, I=1024, top_k=8)) - sz
+        assert 0 < extra <= 20480 * 64 * 4 + 256
     assert moe.workspace_bytes(moe.Desc(T=1, H=33, E=4, I=32, top_k=1)) == 0   # invalid -> 0
 
 
@@ -93,7 +98,7 @@ def test_unsupported_sizes_and_bad_pointers():
     # misaligned x pointer (not 16-byte aligned) is rejected on the host
     w.router = 0x1000
     w.gate = w.up = w.down = 0x2000
-    assert L.moe_route(ctypes.byref(d), 0x1001, ctypes.byref(w), 0x3000, 0x4000, 0x5000, None, None) == \
+    assert L.moe_route(ctypes.byref(d), 0x1001, ctypes.byref(w), 0x3000, 0x4000, 0x5000, None, None, 0, None) == \
         moe.MOE_ERR_INVALID_ARG
     # workspace too small
     assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, 16, None) == moe.MOE_ERR_WORKSPACE

@@ -36,7 +36,8 @@ def make(s, seed=11, bias_values=None, router_std=None):
 
 ROUTE_CASES = {
     "f32_simt": (spec(5, 256, 16, 64, 4, dt="f32"), None),
-    "bf16_tensor_router": (spec(200, 512, 64, 64, 8), None),
+    "bf16_cluster_router": (spec(200, 512, 64, 64, 8), None),
+    "bf16_tensor_router_large": (spec(1100, 1024, 256, 64, 8, shared=32, gated=True), "bias"),
     "bf16_simt_router_bias_gated": (spec(130, 256, 48, 64, 6, shared=32, gated=True), "bias"),
     "bf16_tensor_no_renorm_E256": (spec(300, 256, 256, 64, 8, renorm=False), None),
     "K_equals_E": (spec(7, 128, 8, 64, 8, dt="f32"), None),
@@ -71,6 +72,8 @@ PERMUTE_CASES = {
     "empty_experts": (100, 2, 256, "few"),
     "tiny": (1, 1, 4, "uniform"),
     "large": (8192, 8, 256, "zipf"),
+    "two_ctas": (1250, 8, 64, "uniform"),
+    "beyond_cluster": (9000, 8, 256, "zipf"),
     "ragged": (77, 3, 5, "uniform"),
 }
 
@@ -171,6 +174,7 @@ LAYER_CASES = {
     "skew_all_to_two": (spec(300, 256, 8, 64, 2), dict(skew=True)),
     "no_renorm_gelu_tensor": (spec(150, 256, 32, 96, 4, act="gelu_tanh", renorm=False), {}),
     "K_equals_E_stream": (spec(3, 128, 4, 64, 4, dt="f32"), {}),
+    "stream_f32_wide_H_token_batches": (spec(20, 4096, 4, 64, 2, dt="f32", shared=32), {}),
 }
 
 
