@@ -171,7 +171,10 @@ moe_status moe_combine(const moe_desc* d, const float* y_slots, const void* x, c
 /*
  * The whole layer in one call: route, permute, experts, shared expert, combine.
  * Picks the tensor-core path (tcgen05 grouped GEMMs) when x and the expert
- * weights are bf16 and T > 64, else the weight-streaming path.
+ * weights are bf16 and T > 64, else the weight-streaming path.  The
+ * streaming path stages whole token rows in shared memory and returns
+ * MOE_ERR_UNSUPPORTED (also from moe_expert_ffn / moe_combine) when
+ * H * sizeof(act) > 65536 or I * 4 > 65536 or shared_I * 4 > 65536.
  *  x [T,H] act_dtype in, out [T,H] act_dtype out, ws >= moe_workspace_bytes(d).
  */
 moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, void* out, void* ws, size_t ws_bytes,

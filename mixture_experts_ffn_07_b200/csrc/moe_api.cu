@@ -286,7 +286,15 @@ moe_status check_router_args(const moe_desc& d, const void* x, const moe_weights
   return MOE_OK;
 }
 
+// The weight-streaming kernels stage whole token rows in shared memory:
+// x rows (H elements) and hidden rows (I or shared_I f32) of at most 64 KB.
+bool stream_rows_fit(const moe_desc& d, int inner) {
+  const long long xb = static_cast<long long>(d.H) * (d.act_dtype == MOE_F32 ? 4 : 2);
+  return xb <= 65536 && static_cast<long long>(inner) * 4 <= 65536;
+}
+
 moe_status check_expert_weights(const moe_desc& d, const moe_weights* w) {
+  if (!tensor_path(d) && !stream_rows_fit(d, d.I)) return MOE_ERR_UNSUPPORTED;
   if (!w || !w->gate || !w->up || !w->down) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w->gate) || !aligned16(w->up) || !aligned16(w->down)) return MOE_ERR_INVALID_ARG;
   if (d.w_dtype == MOE_Q8_0 && (!w->gate_scale || !w->up_scale || !w->down_scale)) return MOE_ERR_INVALID_ARG;
@@ -295,6 +303,7 @@ moe_status check_expert_weights(const moe_desc& d, const moe_weights* w) {
 
 moe_status check_shared_weights(const moe_desc& d, const moe_weights* w) {
   if (d.shared_I == 0) return MOE_OK;
+  if (!tensor_path(d) && !stream_rows_fit(d, d.shared_I)) return MOE_ERR_UNSUPPORTED;
   if (!w || !w->sh_gate || !w->sh_up || !w->sh_down) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w->sh_gate) || !aligned16(w->sh_up) || !aligned16(w->sh_down)) return MOE_ERR_INVALID_ARG;
   if (d.w_dtype == MOE_Q8_0 && (!w->sh_gate_scale || !w->sh_up_scale || !w->sh_down_scale))

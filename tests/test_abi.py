@@ -112,6 +112,31 @@ def test_unsupported_sizes_and_bad_pointers():
     assert L.moe_q8_0_split(None, 4, 48, None, None, None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_streaming_path_row_limit():
+    """The weight-streaming path stages whole token rows (<= 64 KB) in shared
+    memory; larger rows are rejected on the host, the tensor-core path is not."""
+    import mixture_experts_ffn_07_b200 as moe
+    from mixture_experts_ffn_07_b200 import _lib
+    L = _lib.lib()
+    w = _lib.MoeWeights(router=0x1000, gate=0x2000, up=0x2000, down=0x2000)
+    big = 1 << 34
+    # f32 x with H = 16416 (65664-byte rows) on the streaming path
+    d = _lib.MoeDesc(4, 16416, 4, 64, 2, 0, 1, moe.MOE_F32, moe.MOE_F32, moe.MOE_F32, 0, 0, 0)
+    assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, big, None) == \
+        moe.MOE_ERR_UNSUPPORTED
+    d.H = 16384  # exactly 64 KB passes validation (the call then fails only for want of a device)
+    assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, big, None) != \
+        moe.MOE_ERR_UNSUPPORTED
+    # hidden rows: I * 4 bytes
+    d.H, d.I = 64, 16416
+    assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, big, None) == \
+        moe.MOE_ERR_UNSUPPORTED
+    # the same sizes in bf16 with T > 64 take the tensor-core path: no row limit
+    d = _lib.MoeDesc(100, 16416, 4, 64, 2, 0, 1, moe.MOE_BF16, moe.MOE_BF16, moe.MOE_BF16, 0, 0, 0)
+    assert L.moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, big, None) != \
+        moe.MOE_ERR_UNSUPPORTED
+
+
 def test_empty_batch_is_a_no_op_without_cuda():
     import mixture_experts_ffn_07_b200 as moe
     from mixture_experts_ffn_07_b200 import _lib
