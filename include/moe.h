@@ -107,10 +107,27 @@ const char* moe_version(void);
 /*
  * Bytes of caller-provided device workspace moe_layer needs for `d`: linear in
  * T for fixed sizes, plus the bf16 router's split-K partial logits (at most
- * 20480*E*4 bytes), in 256-byte aligned regions.  Returns 0 for an invalid
+ * 20480*E*4 bytes) for T > 64, or for 1 <= T <= 64 on the streaming path the
+ * fused decode kernel's per-chunk partial logits (ceil(H/1024)*T*(E+1)*4
+ * bytes), in 256-byte aligned regions.  Returns 0 for an invalid
  * descriptor.  moe_route, moe_expert_ffn and moe_combine need no more than this.
  */
 size_t moe_workspace_bytes(const moe_desc* d);
+
+/*
+ * Where moe_layer leaves its routing inside the workspace: byte offsets from
+ * `ws` (each 256-byte aligned) of logits [T,E] f32 (with the bias),
+ * topk_ids [T,K] int32, topk_w [T,K] f32, shared_gate [T] f32 (written only
+ * when shared_I > 0 and has_shared_gate), counts [E] int32, offsets [E+1]
+ * int32, sorted_pairs [P] int32 and pair_pos [P] int32, with the meanings of
+ * moe_route and moe_permute.  Readable once the stream has passed the
+ * moe_layer call.  Host only.  MOE_ERR_INVALID_ARG for an invalid descriptor
+ * or r == NULL.
+ */
+typedef struct moe_ws_regions {
+  size_t logits, topk_ids, topk_w, shared_gate, counts, offsets, sorted_pairs, pair_pos;
+} moe_ws_regions;
+moe_status moe_workspace_regions(const moe_desc* d, moe_ws_regions* r);
 
 /*
  * Router: logits, softmax, top-K with renormalisation.
@@ -252,6 +269,15 @@ int moe_trace_read(const char** names, float* ms, int max);
  * Used by the failure-detection test; never set in normal use. */
 void moe_debug_set_wait_limit(int64_t cycles);
 void moe_debug_set_skip_stage(int enable);
+
+/* How moe_layer runs a batch of 1..64 tokens on the weight-streaming path:
+ * enable = 1 (default) as one cooperative kernel ("decode_layer": router,
+ * top-K, permutation, gate/up, down and combine as phases of one persistent
+ * grid, one CTA per SM); 0 as the step-by-step launches.  Both write the same
+ * workspace regions and `out`, and give the same routing.  If the cooperative
+ * grid cannot be made resident, moe_layer takes the step-by-step path by
+ * itself.  Process-wide; takes effect at the next call. */
+void moe_set_fused_decode(int enable);
 
 #ifdef __cplusplus
 }

@@ -93,6 +93,13 @@ def workspace_bytes(desc: Desc) -> int:
     return _lib.lib().moe_workspace_bytes(ctypes.byref(d))
 
 
+def workspace_regions(desc: Desc) -> dict:
+    """moe_workspace_regions: byte offsets of the routing results moe_layer leaves in the workspace."""
+    d, r = desc.c(), _lib.MoeWsRegions()
+    check(_lib.lib().moe_workspace_regions(ctypes.byref(d), ctypes.byref(r)), "moe_workspace_regions")
+    return {n: getattr(r, n) for n, _ in _lib.MoeWsRegions._fields_}
+
+
 def route(desc, x, w, logits, topk_ids, topk_w, shared_gate=None, ws=None, stream=None):
     d, cw = desc.c(), w.c()
     check(_lib.lib().moe_route(ctypes.byref(d), _ptr(x), ctypes.byref(cw), _ptr(logits), _ptr(topk_ids),
@@ -171,6 +178,12 @@ def debug_set_wait_limit(cycles: int) -> None:
 
 def debug_set_skip_stage(enable: bool) -> None:
     _lib.lib().moe_debug_set_skip_stage(int(enable))
+
+
+def set_fused_decode(enable: bool) -> None:
+    """moe_set_fused_decode: one cooperative kernel (True, default) or step-by-step
+    launches (False) for 1..64 tokens on the weight-streaming path."""
+    _lib.lib().moe_set_fused_decode(int(enable))
 
 
 def _nbytes(t) -> int:

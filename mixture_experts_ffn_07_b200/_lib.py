@@ -22,7 +22,8 @@ MOE_ACT_SILU, MOE_ACT_GELU_TANH = 0, 1
 EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_layer", "moe_layer_host", "moe_layer_noalloc", "moe_q8_0_split",
            "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
-           "moe_debug_set_wait_limit", "moe_debug_set_skip_stage")
+           "moe_debug_set_wait_limit", "moe_debug_set_skip_stage", "moe_set_fused_decode",
+           "moe_workspace_regions")
 
 
 class MoeDesc(ctypes.Structure):
@@ -35,6 +36,11 @@ class MoeWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("router", "router_bias", "gate", "up", "down", "sh_gate", "sh_up", "sh_down", "sh_gate_w",
                  "gate_scale", "up_scale", "down_scale", "sh_gate_scale", "sh_up_scale", "sh_down_scale")]
+
+
+class MoeWsRegions(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("logits", "topk_ids", "topk_w", "shared_gate", "counts", "offsets", "sorted_pairs", "pair_pos")]
 
 
 class MoeError(RuntimeError):
@@ -80,6 +86,10 @@ def lib():
         L.moe_debug_set_wait_limit.restype = None
         L.moe_debug_set_skip_stage.argtypes = [I32]
         L.moe_debug_set_skip_stage.restype = None
+        L.moe_set_fused_decode.argtypes = [I32]
+        L.moe_set_fused_decode.restype = None
+        L.moe_workspace_regions.argtypes = [DP, ctypes.POINTER(MoeWsRegions)]
+        L.moe_workspace_regions.restype = I32
         _lib = L
     return _lib
 

@@ -21,6 +21,7 @@ struct Ctx {
   cudaStream_t stream;
   int* status;             // device status word (first error wins)
   int num_sms;
+  int smem_optin;           // largest dynamic + static shared memory per block
   long long wait_limit;    // SM cycles a pipeline wait may spin before giving up
   int skip_stage;          // debug: grouped-GEMM producer skips one stage's loads
   int pdl;                 // launch with programmatic stream serialization

@@ -1,0 +1,537 @@
+// The whole MoE layer for a small batch (T <= 64) in one cooperative launch.
+//
+// Decode is bandwidth-bound on the touched experts' weights (a few hundred MB
+// at most), so the cost that remains after streaming them at full speed is the
+// chain of dependent launches: router, permutation, gate/up, down, combine,
+// each with its launch latency, pipeline ramp and tail.  Here one persistent
+// grid (one CTA per SM, all resident: cooperative launch) runs the steps as
+// phases separated by grid barriers:
+//   R  router logits: the (router row, hidden chunk, token group) dot products
+//      spread over every warp of the grid; partial sums per chunk go to the
+//      workspace.                                                  -- barrier
+//   S  every CTA adds the chunk partials in chunk order (the same arithmetic
+//      order as the router kernels, so logits and routing are bit-identical to
+//      moe_route), runs the warp top-K for all tokens and the stable counting
+//      sort of the pairs into shared memory.  CTA 0 also writes them out.
+//   G  gate/up of every touched expert (and the shared expert) by the
+//      weight-streaming GEMV of stream_core.cuh.                   -- barrier
+//   D  down, same GEMV, scaled by the routing weights (the shared expert by
+//      its gate).                                                  -- barrier
+//   C  combine: out[t] = sum_k y_slot[t, k] (+ y_shared[t]) in that order.
+//
+// The grid barrier is a counter in device memory: CTA 0 adds 2^31 - (G-1) and
+// the others add 1, so every complete barrier moves the counter by exactly
+// 2^31 (its top bit flips, its low bits come back to 0); a CTA waits for the
+// top bit to differ from the value it saw on arrival.  Waits are bounded; a
+// CTA that gives up still arrives at the later barriers, so every barrier of a
+// launch sees all G arrivals and the counter is consistent for the next launch.
+// Only one such grid can be resident on a device at a time (each takes every
+// SM), so one counter per device serves all launches.
+#include <atomic>
+
+#include "route_util.cuh"
+#include "stream_core.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace stream;
+
+constexpr int kTokGroup = 8;  // tokens per router work item
+constexpr int kDecodeTok = 4;  // token rows per expert batch in the GEMV phases
+constexpr int kMaxRouterRows = 257;
+constexpr int kRouterSteps = kRouterChunk / 256;  // 8-element steps of a lane per chunk
+
+__device__ unsigned g_decode_barrier;
+
+struct DecodeArgs {
+  const void* x;
+  const void* router;
+  int router_bf16;
+  const float* bias;
+  const void* w_s;  // shared-gate row (router dtype) or nullptr
+  int T, H, E, K, renorm, has_shared;
+  Phase g, d;       // gate/up and down; pairs and row scales are set in the kernel
+  int stage_bytes;  // dynamic shared memory before the pair arrays
+  float* parts;     // [nch, T, R] chunk partials of the logits
+  float* logits;    // [T, E] biased logits
+  int32_t* ids;
+  float* w;
+  float* shared_gate;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_pairs;
+  int32_t* pair_pos;
+  const float* y_slots;
+  const float* y_s;
+  void* out;
+  int* status;
+  long long wait_limit;
+};
+
+// One thread per CTA.  Returns false when the wait gave up (or wait == false).
+__device__ __forceinline__ bool grid_barrier(long long limit, const int* status, bool wait) {
+  __threadfence();
+  const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+  const unsigned old = atomicAdd(&g_decode_barrier, add);
+  if (!wait) return false;
+  const long long t0 = clock64();
+  while (true) {
+    unsigned cur;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(&g_decode_barrier) : "memory");
+    if ((cur ^ old) & 0x80000000u) break;
+    if (*reinterpret_cast<const volatile int*>(status) != 0 || clock64() - t0 > limit) return false;
+  }
+  __threadfence();
+  return true;
+}
+
+// All threads of the CTA; false once this CTA has given up on a barrier.
+__device__ __forceinline__ bool cta_grid_sync(const DecodeArgs& a, int* s_abort, int* s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!grid_barrier(a.wait_limit, a.status, *s_abort == 0)) *s_abort = 1;
+    *s_flag = *s_abort;
+  }
+  __syncthreads();
+  return *s_flag == 0;
+}
+
+// Partial logits of a block of router rows for one (hidden chunk, token group):
+// the CTA has staged the group's x chunk in shared memory as f32 (xs, rows of
+// kRouterChunk); warp w takes row r0 + w.  The chunk arithmetic is that of
+// route_util.cuh.  The row's chunk is requested whole before any product.
+template <typename WT>
+__device__ __forceinline__ void router_rows(const DecodeArgs& a, const float* xs, int r0, int ch, int t0, int nt,
+                                            int R) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = r0 + warp;
+  if (r >= R) return;
+  const int h0 = ch * kRouterChunk, hc = min(kRouterChunk, a.H - h0);
+  const WT* wrow = (r < a.E ? static_cast<const WT*>(a.router) + static_cast<size_t>(r) * a.H
+                            : static_cast<const WT*>(a.w_s)) +
+                   h0;
+  Raw8<WT> wr[kRouterSteps];
+#pragma unroll
+  for (int u = 0; u < kRouterSteps; ++u)
+    if (lane * 8 + 256 * u < hc) raw_load(wrow + lane * 8 + 256 * u, wr[u]);
+  float acc[kTokGroup];
+#pragma unroll
+  for (int c = 0; c < kTokGroup; ++c) acc[c] = 0.f;
+#pragma unroll
+  for (int u = 0; u < kRouterSteps; ++u) {
+    const int j = lane * 8 + 256 * u;
+    if (j < hc) {
+      float wv[8];
+      raw_decode(wr[u], wv);
+#pragma unroll
+      for (int c = 0; c < kTokGroup; ++c) {
+        if (c < nt) {
+          const float4 x0 = *reinterpret_cast<const float4*>(xs + c * kRouterChunk + j);
+          const float4 x1 = *reinterpret_cast<const float4*>(xs + c * kRouterChunk + j + 4);
+          const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[c] = fmaf(wv[q], xv[q], acc[c]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < kTokGroup; ++c) {
+    if (c < nt) {
+      const float v = warp_sum(acc[c]);
+      if (lane == 0) a.parts[(static_cast<size_t>(ch) * a.T + t0 + c) * R + r] = v;
+    }
+  }
+}
+
+// Stages x[t0 .. t0+nt) [h0 .. h0+hc) as f32 rows of kRouterChunk.  All threads.
+template <typename XT>
+__device__ __forceinline__ void router_stage_x(const DecodeArgs& a, float* xs, int ch, int t0, int nt) {
+  const int h0 = ch * kRouterChunk, hc = min(kRouterChunk, a.H - h0);
+  const int g8 = hc / 8;
+  for (int i = threadIdx.x; i < nt * g8; i += blockDim.x) {
+    const int c = i / g8, q = i - c * g8;
+    Raw8<XT> r;
+    raw_load(static_cast<const XT*>(a.x) + static_cast<size_t>(t0 + c) * a.H + h0 + 8 * q, r);
+    float v[8];
+    raw_decode(r, v);
+    float4* dst = reinterpret_cast<float4*>(xs + c * kRouterChunk + 8 * q);
+    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+template <typename XT, int WK>
+__global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int s_expert[kMaxGroups], s_first[kMaxGroups], s_count[kMaxGroups], s_poff[kMaxGroups + 1];
+  __shared__ long long s_coff[kMaxGroups + 1];
+  __shared__ int s_cnt[256], s_off[257];
+  __shared__ float s_sgate[kMaxDecodeT];
+  __shared__ Phase s_ph[2];
+  __shared__ int s_arow[kMaxTok], s_dest[kMaxTok];
+  __shared__ float s_scale[kMaxTok];
+  __shared__ float s_part[kMaxUnits * kMaxTok * 2];
+  __shared__ int s_warp[8];
+  __shared__ int s_n, s_flag, s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = a.T, E = a.E, K = a.K, P = T * K;
+  const int R = E + (a.w_s ? 1 : 0);
+  float* s_rows = reinterpret_cast<float*>(smem);  // phase S: one logit row per warp (stage area)
+  int32_t* s_ids = reinterpret_cast<int32_t*>(smem + a.stage_bytes);
+  float* s_w = reinterpret_cast<float*>(s_ids + P);
+  int32_t* s_sorted = reinterpret_cast<int32_t*>(s_w + P);
+  int32_t* s_rank = s_sorted + P;
+  const Smem sm{smem, s_arow, s_dest, s_scale, s_part};
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    s_ph[0] = a.g;
+    s_ph[1] = a.d;
+    s_ph[0].pairs = s_sorted;
+    s_ph[1].pairs = s_sorted;
+    s_ph[1].src[0].row_scale = s_w;
+    s_ph[1].src[1].row_scale = a.w_s ? s_sgate : nullptr;
+  }
+
+  // ---- R: partial router logits; a CTA item is (hidden chunk, token group, block of kWarps rows)
+  {
+    const int nch = (a.H + kRouterChunk - 1) / kRouterChunk;
+    const int ntg = (T + kTokGroup - 1) / kTokGroup;
+    const int nrb = (R + kWarps - 1) / kWarps;
+    const int items = nch * ntg * nrb;
+    float* xs = reinterpret_cast<float*>(smem);
+    int staged = -1;
+    for (int i = blockIdx.x; i < items; i += gridDim.x) {
+      const int rb = i % nrb, cg = i / nrb;  // consecutive items of a CTA share their x chunk when they can
+      const int ch = cg % nch, tg = cg / nch;
+      const int t0 = tg * kTokGroup, nt = min(kTokGroup, T - t0);
+      if (cg != staged) {
+        __syncthreads();
+        router_stage_x<XT>(a, xs, ch, t0, nt);
+        __syncthreads();
+        staged = cg;
+      }
+      if (a.router_bf16)
+        router_rows<__nv_bfloat16>(a, xs, rb * kWarps, ch, t0, nt, R);
+      else
+        router_rows<float>(a, xs, rb * kWarps, ch, t0, nt, R);
+    }
+  }
+  cta_grid_sync(a, &s_abort, &s_flag);
+
+  // ---- S: logits, top-K and the pair permutation, in every CTA
+  {
+    const int nch = (a.H + kRouterChunk - 1) / kRouterChunk;
+    for (int t = warp; t < T; t += kWarps) {
+      float* row = s_rows + warp * kMaxRouterRows;
+      float l[9];  // experts lane + 32 i; chunk partials requested together, added in chunk order
+#pragma unroll
+      for (int i = 0; i < 9; ++i) l[i] = 0.f;
+      for (int ch0 = 0; ch0 < nch; ch0 += 2) {
+        float v[2][9];
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int i = 0; i < 9; ++i)
+            v[j][i] = (ch0 + j < nch && lane + 32 * i < R)
+                          ? __ldcg(a.parts + (static_cast<size_t>(ch0 + j) * T + t) * R + lane + 32 * i)
+                          : 0.f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int i = 0; i < 9; ++i)
+            if (ch0 + j < nch) l[i] += v[j][i];
+      }
+#pragma unroll
+      for (int i = 0; i < 9; ++i)
+        if (lane + 32 * i < R) row[lane + 32 * i] = l[i];
+      __syncwarp();
+      float* lout = blockIdx.x == 0 ? a.logits + static_cast<size_t>(t) * E : row;
+      warp_topk(row, a.bias, E, K, a.renorm, lout, s_ids + t * K, s_w + t * K);
+      if (a.w_s && lane == 0) {
+        const float sg = 1.0f / (1.0f + expf(-row[E]));
+        s_sgate[t] = sg;
+        if (blockIdx.x == 0) a.shared_gate[t] = sg;
+      }
+      __syncwarp();
+    }
+    __syncthreads();
+    if (warp == 0) {  // stable counting sort: ranks within each expert in pair order
+      for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
+      __syncwarp();
+      for (int base = 0; base < P; base += 32) {
+        const int p = base + lane;
+        const int e = p < P ? s_ids[p] : -1;
+        const unsigned m = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(m & ((1u << lane) - 1u));
+        const int before = p < P ? s_cnt[e] : 0;
+        __syncwarp();
+        if (p < P) {
+          s_rank[p] = before + rank;
+          if (rank == 0) s_cnt[e] = before + __popc(m);
+        }
+        __syncwarp();
+      }
+      int loc[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        loc[i] = e < E ? s_cnt[e] : 0;
+        sum += loc[i];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int run = incl - sum;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        if (e < E) s_off[e] = run;
+        run += loc[i];
+      }
+      if (lane == 31) s_off[E] = incl;
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+      const int pos = s_off[s_ids[p]] + s_rank[p];
+      s_sorted[pos] = p;
+      if (blockIdx.x == 0) {
+        a.pair_pos[p] = pos;
+        a.sorted_pairs[pos] = p;
+        a.ids[p] = s_ids[p];
+        a.w[p] = s_w[p];
+      }
+    }
+    if (blockIdx.x == 0)
+      for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+        a.offsets[e] = s_off[e];
+        if (e < E) a.counts[e] = s_cnt[e];
+      }
+    // groups: touched experts in order, then the shared expert
+    if (threadIdx.x < 256) {
+      const int e = threadIdx.x;
+      const bool f = e < E && s_cnt[e] > 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, f);
+      if (lane == 0) s_warp[warp] = __popc(bal);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      int base = 0, n = 0;
+      for (int w = 0; w < 8; ++w) {
+        if (w < warp) base += s_warp[w];
+        n += s_warp[w];
+      }
+      if (f) {
+        const int i = base + __popc(bal & ((1u << lane) - 1u));
+        s_expert[i] = e;
+        s_first[i] = s_off[e];
+        s_count[i] = s_cnt[e];
+      }
+      if (threadIdx.x == 0) {
+        if (a.has_shared) {
+          s_expert[n] = -1;
+          s_first[n] = 0;
+          s_count[n] = T;
+          ++n;
+        }
+        s_n = n;
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- G: gate/up
+  {
+    const Tables tb{s_expert, s_first, s_count, s_poff, s_coff, s_n};
+    if (warp == 0) build_prefix(tb, s_ph[0]);
+    __syncthreads();
+    int p0, p1;
+    cta_pairs(tb, s_ph[0], p0, p1);
+    if (!s_abort) run_phase<XT, WK, true, kDecodeTok>(s_ph[0], tb, p0, p1, sm);
+  }
+  cta_grid_sync(a, &s_abort, &s_flag);
+
+  // ---- D: down
+  {
+    const Tables tb{s_expert, s_first, s_count, s_poff, s_coff, s_n};
+    if (warp == 0) build_prefix(tb, s_ph[1]);
+    __syncthreads();
+    int p0, p1;
+    cta_pairs(tb, s_ph[1], p0, p1);
+    if (!s_abort) run_phase<float, WK, false, kDecodeTok>(s_ph[1], tb, p0, p1, sm);
+  }
+  const bool ok = cta_grid_sync(a, &s_abort, &s_flag);
+
+  // ---- C: combine
+  if (ok) {
+    const int H4 = a.H / 4;
+    const long long total = static_cast<long long>(T) * H4;
+    const float4* ys = reinterpret_cast<const float4*>(a.y_slots);
+    const float4* sh = reinterpret_cast<const float4*>(a.y_s);
+    for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+      const long long t = idx / H4;
+      const int c = static_cast<int>(idx - t * H4);
+      float4 acc = __ldcg(ys + (t * K) * H4 + c);
+      for (int k = 1; k < K; ++k) {
+        const float4 v = __ldcg(ys + (t * K + k) * H4 + c);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      if (a.has_shared) {
+        const float4 v = __ldcg(sh + t * H4 + c);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      if constexpr (sizeof(XT) == 4) {
+        reinterpret_cast<float4*>(a.out)[idx] = acc;
+      } else {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(a.out)[idx] = pk;
+      }
+    }
+  }
+  if (threadIdx.x == 0 && s_abort) record_status(a.status, MOE_ERR_TIMEOUT);
+}
+
+// Static shared memory of a kernel instance (queried once).
+template <typename XT, int WK>
+int static_smem() {
+  static std::atomic<int> bytes{-1};
+  int b = bytes.load();
+  if (b < 0) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, decode_layer_kernel<XT, WK>) != cudaSuccess) return -1;
+    b = static_cast<int>(fa.sharedSizeBytes);
+    bytes.store(b);
+  }
+  return b;
+}
+
+template <typename XT, int WK>
+cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
+  auto kern = decode_layer_kernel<XT, WK>;
+  const int smem = a.stage_bytes + 16 * P;
+  const int st = static_smem<XT, WK>();
+  if (st < 0 || smem + st > c.smem_optin) return cudaErrorInvalidValue;
+  const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  KernelScope ks(c, "decode_layer");
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(c.num_sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace
+
+size_t decode_router_parts_floats(int T, int H, int E, bool shared_gate) {
+  const size_t nch = (static_cast<size_t>(H) + kRouterChunk - 1) / kRouterChunk;
+  return nch * T * (E + (shared_gate ? 1 : 0));
+}
+
+cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
+  if (L.T <= 0) return cudaSuccess;
+  const int P = L.T * L.K;
+  if (L.T > kMaxDecodeT || P > kMaxDecodePairs || L.E > 256 || (L.H % 4)) return cudaErrorInvalidValue;
+  const int wk = wk_of(L.w_dtype);
+  const int ab = L.x_dtype == MOE_F32 ? 4 : 2;
+  DecodeArgs a{};
+  // gate/up: routed experts read x rows through the pair list, the shared expert reads x row r
+  a.g.plan[0] = make_plan(wk, true, L.H, L.I, ab, L.T, kDecodeTok);
+  a.g.plan[1] = L.Is > 0 ? make_plan(wk, true, L.H, L.Is, ab, L.T, kDecodeTok) : a.g.plan[0];
+  a.d.plan[0] = make_plan(wk, false, L.I, L.H, 4, L.T, kDecodeTok);
+  a.d.plan[1] = L.Is > 0 ? make_plan(wk, false, L.Is, L.H, 4, L.T, kDecodeTok) : a.d.plan[0];
+  // phases R and S use the stage area for an f32 x chunk of a token group and one logit row per warp
+  int stage = std::max(kTokGroup * kRouterChunk * 4, kWarps * kMaxRouterRows * 4);
+  for (const Plan* p : {&a.g.plan[0], &a.g.plan[1], &a.d.plan[0], &a.d.plan[1]}) {
+    if (p->xrow_bytes > kMaxTokenRowBytes) return cudaErrorInvalidValue;
+    stage = std::max(stage, p->TS * p->xrow_bytes);
+  }
+  a.stage_bytes = (stage + 127) / 128 * 128;
+  a.x = L.x;
+  a.router = L.router;
+  a.router_bf16 = L.router_dtype == MOE_BF16;
+  a.bias = L.bias;
+  a.w_s = L.w_s;
+  a.T = L.T;
+  a.H = L.H;
+  a.E = L.E;
+  a.K = L.K;
+  a.renorm = L.renorm;
+  a.has_shared = L.Is > 0;
+  a.g.K = L.K;
+  a.g.act_fn = L.act;
+  GroupSrc& gr = a.g.src[0];
+  gr.w0 = static_cast<const uint8_t*>(L.gate);
+  gr.w1 = static_cast<const uint8_t*>(L.up);
+  gr.s0 = static_cast<const uint8_t*>(L.gate_scale);
+  gr.s1 = static_cast<const uint8_t*>(L.up_scale);
+  gr.act = static_cast<const uint8_t*>(L.x);
+  gr.out = L.h;
+  gr.act_via_pairs = 1;
+  GroupSrc& gs = a.g.src[1];
+  gs.w0 = static_cast<const uint8_t*>(L.sh_gate);
+  gs.w1 = static_cast<const uint8_t*>(L.sh_up);
+  gs.s0 = static_cast<const uint8_t*>(L.sh_gate_scale);
+  gs.s1 = static_cast<const uint8_t*>(L.sh_up_scale);
+  gs.act = static_cast<const uint8_t*>(L.x);
+  gs.out = L.h_s;
+  // down: routed rows go to their pair's slot scaled by its weight; the shared expert by its gate
+  a.d.K = 1;
+  GroupSrc& dr = a.d.src[0];
+  dr.w0 = static_cast<const uint8_t*>(L.down);
+  dr.s0 = static_cast<const uint8_t*>(L.down_scale);
+  dr.act = reinterpret_cast<const uint8_t*>(L.h);
+  dr.out = L.y_slots;
+  dr.out_via_pairs = 1;
+  dr.scale_via_pairs = 1;
+  GroupSrc& ds = a.d.src[1];
+  ds.w0 = static_cast<const uint8_t*>(L.sh_down);
+  ds.s0 = static_cast<const uint8_t*>(L.sh_down_scale);
+  ds.act = reinterpret_cast<const uint8_t*>(L.h_s);
+  ds.out = L.y_s;
+  a.parts = L.router_parts;
+  a.logits = L.logits;
+  a.ids = L.ids;
+  a.w = L.w;
+  a.shared_gate = L.shared_gate;
+  a.counts = L.counts;
+  a.offsets = L.offsets;
+  a.sorted_pairs = L.sorted_pairs;
+  a.pair_pos = L.pair_pos;
+  a.y_slots = L.y_slots;
+  a.y_s = L.y_s;
+  a.out = L.out;
+  a.status = c.status;
+  a.wait_limit = c.wait_limit;
+  if (L.x_dtype == MOE_F32) {
+    if (wk == WK_F32) return launch_fused<float, WK_F32>(c, a, P);
+    if (wk == WK_BF16) return launch_fused<float, WK_BF16>(c, a, P);
+    return launch_fused<float, WK_Q8>(c, a, P);
+  }
+  if (wk == WK_F32) return launch_fused<__nv_bfloat16, WK_F32>(c, a, P);
+  if (wk == WK_BF16) return launch_fused<__nv_bfloat16, WK_BF16>(c, a, P);
+  return launch_fused<__nv_bfloat16, WK_Q8>(c, a, P);
+}
+
+}  // namespace moe

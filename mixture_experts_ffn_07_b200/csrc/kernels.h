@@ -88,4 +88,40 @@ cudaError_t launch_combine(const Ctx& c, const float* y_slots, const float* y_sh
 cudaError_t launch_q8_0_split(const Ctx& c, const void* blocks, int64_t rows, int64_t cols, int8_t* q,
                               void* scales);
 
+
+// The whole layer for a small batch in one cooperative launch (decode_fused.cu):
+// router, top-K, permutation, gate/up, down and combine as phases of one
+// persistent grid separated by grid barriers.  Writes the same workspace
+// outputs as the step-by-step path (logits, ids, w, shared_gate, counts,
+// offsets, sorted_pairs, pair_pos, h, h_s, y_slots, y_s) and `out`.
+constexpr int kMaxDecodeT = 64;
+constexpr int kMaxDecodePairs = 2048;
+struct DecodeLayer {
+  const void* x;
+  int x_dtype;
+  const void* router;
+  int router_dtype;
+  const float* bias;   // router bias or nullptr
+  const void* w_s;     // shared-gate row or nullptr
+  int T, H, E, K, I, Is, act, renorm, w_dtype;
+  const void *gate, *up, *down, *gate_scale, *up_scale, *down_scale;
+  const void *sh_gate, *sh_up, *sh_down, *sh_gate_scale, *sh_up_scale, *sh_down_scale;
+  float* router_parts;  // decode_router_parts_floats(...) floats
+  float* logits;
+  int32_t* ids;
+  float* w;
+  float* shared_gate;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_pairs;
+  int32_t* pair_pos;
+  float* h;
+  float* h_s;
+  float* y_slots;
+  float* y_s;
+  void* out;
+};
+size_t decode_router_parts_floats(int T, int H, int E, bool shared_gate);
+cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L);
+
 }  // namespace moe

@@ -25,6 +25,7 @@ struct DeviceInfo {
   bool ready = false;
   int* status = nullptr;
   int num_sms = 0;
+  int smem_optin = 0;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -32,6 +33,7 @@ std::mutex g_dev_mu;
 std::atomic<uint64_t> g_launches{0};
 std::atomic<long long> g_wait_limit{1LL << 31};
 std::atomic<int> g_skip_stage{0};
+std::atomic<int> g_fused_decode{1};
 
 struct TraceRec {
   const char* name;
@@ -51,14 +53,17 @@ bool make_ctx(cudaStream_t s, moe::Ctx* c) {
     if (!d.ready) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return false;
-      int sms = 0;
+      int sms = 0, optin = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return false;
+      if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
       d.status = static_cast<int*>(p);
       d.num_sms = sms;
+      d.smem_optin = optin;
       d.ready = true;
     }
     c->status = d.status;
     c->num_sms = d.num_sms;
+    c->smem_optin = d.smem_optin;
   }
   c->stream = s;
   c->wait_limit = g_wait_limit.load();
@@ -75,6 +80,12 @@ bool tensor_path(const moe_desc& d) { return d.act_dtype == MOE_BF16 && d.w_dtyp
 
 bool tensor_router(const moe_desc& d) {
   return d.act_dtype == MOE_BF16 && d.router_dtype == MOE_BF16 && d.T > 64 && d.E % 32 == 0;
+}
+
+// The whole layer as one cooperative kernel (decode_fused.cu): the streaming
+// path with at most 64 tokens.
+bool fused_decode(const moe_desc& d) {
+  return !tensor_path(d) && d.T >= 1 && d.T <= moe::kMaxDecodeT && d.T * d.top_k <= moe::kMaxDecodePairs;
 }
 
 // Ranges the router GEMM splits the hidden dimension into, so that small batches
@@ -104,8 +115,8 @@ moe_status check_desc(const moe_desc* d) {
 }
 
 struct Layout {
-  size_t logits, logit_parts, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos, y_slots, x_perm, h, h_s,
-      y_s, total;
+  size_t logits, logit_parts, router_parts, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos, y_slots,
+      x_perm, h, h_s, y_s, total;
 };
 
 Layout layout_of(const moe_desc& d) {
@@ -120,6 +131,7 @@ Layout layout_of(const moe_desc& d) {
   const bool tc = tensor_path(d);
   L.logits = take(T * E * 4);
   L.logit_parts = tensor_router(d) ? take(router_ksplit(d) * T * E * 4) : 0;
+  L.router_parts = fused_decode(d) ? take(moe::decode_router_parts_floats(d.T, d.H, d.E, shared_gated(d)) * 4) : 0;
   L.ids = take(P * 4);
   L.w = take(P * 4);
   L.shared_gate = take(T * 4);
@@ -373,6 +385,20 @@ size_t moe_workspace_bytes(const moe_desc* d) {
   return layout_of(*d).total;
 }
 
+moe_status moe_workspace_regions(const moe_desc* d, moe_ws_regions* r) {
+  if (!r || check_desc(d) != MOE_OK) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout_of(*d);
+  r->logits = L.logits;
+  r->topk_ids = L.ids;
+  r->topk_w = L.w;
+  r->shared_gate = L.shared_gate;
+  r->counts = L.counts;
+  r->offsets = L.offsets;
+  r->sorted_pairs = L.sorted_pairs;
+  r->pair_pos = L.pair_pos;
+  return MOE_OK;
+}
+
 moe_status moe_route(const moe_desc* d, const void* x, const moe_weights* w, float* logits, int32_t* topk_ids,
                      float* topk_w, float* shared_gate, void* ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = check_desc(d);
@@ -459,6 +485,56 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
   int32_t* sorted_pairs = at<int32_t>(ws, L.sorted_pairs);
   float* y_slots = at<float>(ws, L.y_slots);
   float* parts = L.logit_parts ? at<float>(ws, L.logit_parts) : nullptr;
+  if (fused_decode(*d) && g_fused_decode.load()) {
+    moe::DecodeLayer f{};
+    f.x = x;
+    f.x_dtype = d->act_dtype;
+    f.router = w->router;
+    f.router_dtype = d->router_dtype;
+    f.bias = d->has_router_bias ? w->router_bias : nullptr;
+    f.w_s = shared_gated(*d) ? w->sh_gate_w : nullptr;
+    f.T = d->T;
+    f.H = d->H;
+    f.E = d->E;
+    f.K = d->top_k;
+    f.I = d->I;
+    f.Is = d->shared_I;
+    f.act = d->act;
+    f.renorm = d->renormalize;
+    f.w_dtype = d->w_dtype;
+    f.gate = w->gate;
+    f.up = w->up;
+    f.down = w->down;
+    f.gate_scale = w->gate_scale;
+    f.up_scale = w->up_scale;
+    f.down_scale = w->down_scale;
+    f.sh_gate = w->sh_gate;
+    f.sh_up = w->sh_up;
+    f.sh_down = w->sh_down;
+    f.sh_gate_scale = w->sh_gate_scale;
+    f.sh_up_scale = w->sh_up_scale;
+    f.sh_down_scale = w->sh_down_scale;
+    f.router_parts = at<float>(ws, L.router_parts);
+    f.logits = logits;
+    f.ids = ids;
+    f.w = tw;
+    f.shared_gate = sg;
+    f.counts = at<int32_t>(ws, L.counts);
+    f.offsets = offsets;
+    f.sorted_pairs = sorted_pairs;
+    f.pair_pos = at<int32_t>(ws, L.pair_pos);
+    f.h = at<float>(ws, L.h);
+    f.h_s = d->shared_I ? at<float>(ws, L.h_s) : nullptr;
+    f.y_slots = y_slots;
+    f.y_s = d->shared_I ? at<float>(ws, L.y_s) : nullptr;
+    f.out = out;
+    const cudaError_t e = moe::launch_decode_layer(c, f);
+    if (e == cudaSuccess) return MOE_OK;
+    // the grid cannot be made resident (or the shape does not fit one CTA per SM):
+    // clear the launch error and take the step-by-step path
+    if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorInvalidValue) return MOE_ERR_CUDA;
+    cudaGetLastError();
+  }
   if ((st = route_impl(c, *d, x, *w, logits, parts, ids, tw, sg)) != MOE_OK) return st;
   MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, at<int32_t>(ws, L.counts), offsets, sorted_pairs,
                               at<int32_t>(ws, L.pair_pos)));
@@ -556,5 +632,7 @@ moe_status moe_layer_noalloc(const moe_desc* d, const void* x, const moe_weights
 void moe_debug_set_wait_limit(int64_t cycles) { g_wait_limit.store(cycles > 0 ? cycles : (1LL << 31)); }
 
 void moe_debug_set_skip_stage(int enable) { g_skip_stage.store(enable ? 1 : 0); }
+
+void moe_set_fused_decode(int enable) { g_fused_decode.store(enable ? 1 : 0); }
 
 }  // extern "C"

@@ -19,7 +19,7 @@
 //    product of its token on the way when there is one.
 #include <cooperative_groups.h>
 
-#include "kernels.h"
+#include "route_util.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -37,46 +37,6 @@ __device__ __forceinline__ void smem8(const float* p, float (&v)[8]) {
   const float4 b = *reinterpret_cast<const float4*>(p + 4);
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void smem8(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 a = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-    v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-  }
-}
-
-template <typename T>
-struct Raw8;  // 8 elements as raw 16-byte words
-template <>
-struct Raw8<float> {
-  uint4 a, b;
-};
-template <>
-struct Raw8<__nv_bfloat16> {
-  uint4 a;
-};
-__device__ __forceinline__ void raw_load(const float* p, Raw8<float>& r) {
-  r.a = __ldg(reinterpret_cast<const uint4*>(p));
-  r.b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
-}
-__device__ __forceinline__ void raw_load(const __nv_bfloat16* p, Raw8<__nv_bfloat16>& r) {
-  r.a = __ldg(reinterpret_cast<const uint4*>(p));
-}
-__device__ __forceinline__ void raw_decode(const Raw8<float>& r, float (&v)[8]) {
-  v[0] = __uint_as_float(r.a.x); v[1] = __uint_as_float(r.a.y); v[2] = __uint_as_float(r.a.z);
-  v[3] = __uint_as_float(r.a.w); v[4] = __uint_as_float(r.b.x); v[5] = __uint_as_float(r.b.y);
-  v[6] = __uint_as_float(r.b.z); v[7] = __uint_as_float(r.b.w);
-}
-__device__ __forceinline__ void raw_decode(const Raw8<__nv_bfloat16>& r, float (&v)[8]) {
-  const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-    v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-  }
 }
 
 // acc[c] += W[row, h0 + j] . xs[c, j] for j in [0, hc) and tokens c < nt, where xs
@@ -113,77 +73,8 @@ __device__ __forceinline__ void row_dots_smem(const WT* __restrict__ wrow, const
   }
 }
 
-// Softmax + top-K (+ renormalisation) of one token, by one warp.  `row` holds the
-// E raw logits (global or shared memory); the biased logits go to logits_out.
-__device__ __forceinline__ void warp_topk(const float* row, const float* __restrict__ bias, int E, int K, int renorm,
-                                          float* __restrict__ logits_out, int32_t* __restrict__ ids,
-                                          float* __restrict__ wout) {
-  const int lane = threadIdx.x & 31;
-  float v[8];
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = -INFINITY;
-    if (e < E) {
-      float l = row[e];
-      if (bias) l += bias[e];
-      logits_out[e] = l;
-      v[i] = l;
-      m = fmaxf(m, l);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-
-  uint32_t taken = 0;
-  int my_e = 0;
-  float my_v = 0.f;
-  for (int k = 0; k < K; ++k) {
-    float bv = -INFINITY;
-    int be = 0x7FFFFFFF;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
-        bv = v[i];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == k) {
-      my_e = be;
-      my_v = bv;
-    }
-  }
-  const float ev = (lane < K) ? expf(my_v - m) : 0.f;
-  float denom;
-  if (renorm) {
-    denom = warp_sum(ev);
-  } else {
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (lane + 32 * i < E) s += expf(v[i] - m);
-    denom = warp_sum(s);
-  }
-  const float inv = denom > 1e-20f ? 1.0f / denom : (renorm ? 1.0f / K : 1.0f);
-  if (lane < K) {
-    ids[lane] = my_e;
-    wout[lane] = ev * inv;
-  }
-}
-
 constexpr int kStageBytes = 64 * 1024;  // x staging per chunk of the hidden dimension
+static_assert(kStageBytes / (kClusterTok * 4) == kRouterChunk, "router chunking must match route_util.cuh");
 
 template <typename XT, typename WT>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(256)

@@ -145,3 +145,23 @@ def test_empty_batch_is_a_no_op_without_cuda():
     ws = moe.workspace_bytes(moe.Desc(T=0, H=64, E=4, I=64, top_k=2))
     assert _lib.lib().moe_layer(ctypes.byref(d), 0x1000, ctypes.byref(w), 0x6000, 0x7000, max(ws, 256), None) == \
         moe.MOE_OK
+
+
+def test_workspace_regions_host_only():
+    import mixture_experts_ffn_07_b200 as moe
+    for d in (moe.Desc(T=1, H=2816, E=128, I=704, top_k=8, act_dtype="f32", w_dtype="f32", router_dtype="f32"),
+              moe.Desc(T=512, H=2048, E=64, I=1024, top_k=8),
+              moe.Desc(T=16, H=2048, E=128, I=768, top_k=8, act_dtype="f32", w_dtype="q8_0", router_dtype="f32",
+                       shared_I=64, has_shared_gate=1)):
+        r = moe.workspace_regions(d)
+        n = moe.workspace_bytes(d)
+        P = d.T * d.top_k
+        sizes = {"logits": d.T * d.E * 4, "topk_ids": P * 4, "topk_w": P * 4, "shared_gate": d.T * 4,
+                 "counts": d.E * 4, "offsets": (d.E + 1) * 4, "sorted_pairs": P * 4, "pair_pos": P * 4}
+        spans = sorted((r[k], r[k] + sizes[k]) for k in sizes)
+        for (a0, a1), (b0, _) in zip(spans, spans[1:]):
+            assert a1 <= b0  # disjoint
+        for k in sizes:
+            assert r[k] % 256 == 0 and r[k] + sizes[k] <= n
+    with pytest.raises(moe.MoeError):
+        moe.workspace_regions(moe.Desc(T=1, H=33, E=4, I=32, top_k=1))
