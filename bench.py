@@ -158,6 +158,23 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(dist, x: float, device) -> float:
+    """The largest of every rank's x (a device time in ms): the job's time.  Every
+    rank must call it at the same point."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: every replica runs `steps` layers of `tokens_per_step`
+    tokens; the job takes the slowest rank's `ms`."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def time_oracle(spec, wl, budget_s: float, max_tokens=None):
     """Oracle on host cores over a bounded token sample sized to ~budget_s seconds. Returns (tokens/s, info)."""
@@ -269,12 +286,9 @@ def run_ours(args, spec):
     torch.cuda.synchronize()
     moe.trace_enable(False)
     trace = moe.trace_read()
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(dist, ms, "cuda")
     ms_step = ms / args.steps
-    value = ws_n * T * args.steps / (ms / 1e3)
+    value = job_throughput(ws_n, T, args.steps, ms)
 
     # per-kernel durations (CUDA events around each launch on the launching stream)
     per = {}
@@ -323,10 +337,7 @@ def run_ours(args, spec):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(dist, e2e_ms, "cuda")
     io_bytes = T * H * x.element_size()
 
     cpu = None
@@ -341,7 +352,7 @@ def run_ours(args, spec):
             "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
                        "act": spec.act, "shared_I": spec.shared_I, "parallelism": f"replicas{ws_n}",
                        "l2": "no flush: inputs larger than L2 (expert weights streamed every step)"},
-            "e2e": {"value": ws_n * T * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
+            "e2e": {"value": job_throughput(ws_n, T, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
                     "d2h_bytes_per_step": io_bytes},
             "roofline": roofline, "layer_roofline": layer_roof, "cpu_baseline": cpu, "gpu_launches": n_launch,
             "clocks": clocks.summary(), "device_status": moe.status_string(status),

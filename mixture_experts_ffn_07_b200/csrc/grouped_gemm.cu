@@ -207,6 +207,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------------------------------------ TMA producer
       uint32_t kbg = 0, outstanding = 0, out_phase = 0;
       bool skipped = false;
+      const uint64_t pol_w = l2_policy_evict_first();  // weights: read once
+      const uint64_t pol_a = l2_policy_evict_last();   // activation rows: read by every column tile
       for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
         int g, mt, nt, ks;
         decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
@@ -225,12 +227,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t* sa = smem + s * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
           mbar_arrive_expect_tx(&aux.full[s], STAGE_BYTES);
-          tma_load_2d(sa, &mapA, &aux.full[s], kb * BK, a_row);
+          tma_load_2d_hint(sa, &mapA, &aux.full[s], kb * BK, a_row, pol_a);
           if (DUAL) {
-            tma_load_2d(sb, &mapB0, &aux.full[s], kb * BK, b_row);
-            tma_load_2d(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row);
+            tma_load_2d_hint(sb, &mapB0, &aux.full[s], kb * BK, b_row, pol_w);
+            tma_load_2d_hint(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row, pol_w);
           } else {
-            tma_load_2d(sb, &mapB0, &aux.full[s], kb * BK, b_row);
+            tma_load_2d_hint(sb, &mapB0, &aux.full[s], kb * BK, b_row, pol_w);
           }
           outstanding |= 1u << s;
           out_phase = (out_phase & ~(1u << s)) | (ph << s);
