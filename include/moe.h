@@ -107,9 +107,9 @@ const char* moe_version(void);
 /*
  * Bytes of caller-provided device workspace moe_layer needs for `d`: linear in
  * T for fixed sizes, plus the bf16 router's split-K partial logits (at most
- * 20480*E*4 bytes) for T > 64, or for 1 <= T <= 64 on the streaming path the
- * fused decode kernel's per-chunk partial logits (ceil(H/1024)*T*(E+1)*4
- * bytes), in 256-byte aligned regions.  Returns 0 for an invalid
+ * 20480*E*4 bytes) and 256*E*4 bytes of per-CTA expert counts for T > 64, or
+ * for 1 <= T <= 64 on the streaming path the fused decode kernel's per-chunk
+ * partial logits (ceil(H/1024)*T*(E+1)*4 bytes), in 256-byte aligned regions.  Returns 0 for an invalid
  * descriptor.  moe_route, moe_expert_ffn and moe_combine need no more than this.
  */
 size_t moe_workspace_bytes(const moe_desc* d);
@@ -278,6 +278,14 @@ void moe_debug_set_skip_stage(int enable);
  * grid cannot be made resident, moe_layer takes the step-by-step path by
  * itself.  Process-wide; takes effect at the next call. */
 void moe_set_fused_decode(int enable);
+
+/* How moe_layer runs the selection, permutation and row gather of the
+ * tensor-core path (bf16, T > 64, bf16 router with E % 32 == 0): enable = 1
+ * (default) as one cooperative kernel ("route_permute_gather") after the
+ * router GEMM; 0 as three launches (router_topk, permute, gather_rows).  Same
+ * values either way; if the cooperative grid cannot be made resident,
+ * moe_layer takes the three launches by itself.  Process-wide. */
+void moe_set_fused_front(int enable);
 
 #ifdef __cplusplus
 }

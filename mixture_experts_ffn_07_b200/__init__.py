@@ -180,6 +180,12 @@ def debug_set_skip_stage(enable: bool) -> None:
     _lib.lib().moe_debug_set_skip_stage(int(enable))
 
 
+def set_fused_front(enable: bool) -> None:
+    """moe_set_fused_front: selection + permutation + row gather of the tensor-core
+    path as one cooperative kernel (True, default) or three launches (False)."""
+    _lib.lib().moe_set_fused_front(int(enable))
+
+
 def set_fused_decode(enable: bool) -> None:
     """moe_set_fused_decode: one cooperative kernel (True, default) or step-by-step
     launches (False) for 1..64 tokens on the weight-streaming path."""

@@ -23,7 +23,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route
            "moe_combine", "moe_layer", "moe_layer_host", "moe_layer_noalloc", "moe_q8_0_split",
            "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
            "moe_debug_set_wait_limit", "moe_debug_set_skip_stage", "moe_set_fused_decode",
-           "moe_workspace_regions")
+           "moe_workspace_regions", "moe_set_fused_front")
 
 
 class MoeDesc(ctypes.Structure):
@@ -88,6 +88,8 @@ def lib():
         L.moe_debug_set_skip_stage.restype = None
         L.moe_set_fused_decode.argtypes = [I32]
         L.moe_set_fused_decode.restype = None
+        L.moe_set_fused_front.argtypes = [I32]
+        L.moe_set_fused_front.restype = None
         L.moe_workspace_regions.argtypes = [DP, ctypes.POINTER(MoeWsRegions)]
         L.moe_workspace_regions.restype = I32
         _lib = L

@@ -134,6 +134,44 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 
+// ---- grid barrier (cooperative launches only) ----
+// A barrier over every CTA of a grid that is resident as a whole (a
+// cooperative launch), on a counter in device memory: CTA 0 adds
+// 2^31 - (G-1) and the others add 1, so each complete barrier moves the
+// counter by exactly 2^31 (its top bit flips, its low bits come back); a CTA
+// waits for the top bit to differ from the value it saw on arrival.  The wait
+// is bounded and abandoned when the status word reports an error; a CTA that
+// gave up still arrives at the later barriers (wait == false), so every
+// barrier of a launch sees all G arrivals and the counter stays consistent.
+// One thread per CTA; returns false when it did not wait to completion.
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, long long limit, const int* status, bool wait) {
+  __threadfence();
+  const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+  const unsigned old = atomicAdd(bar, add);
+  if (!wait) return false;
+  const long long t0 = clock64();
+  while (true) {
+    unsigned cur;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
+    if ((cur ^ old) & 0x80000000u) break;
+    if (*reinterpret_cast<const volatile int*>(status) != 0 || clock64() - t0 > limit) return false;
+  }
+  __threadfence();
+  return true;
+}
+
+// All threads of the CTA; false once this CTA has given up on a barrier.
+__device__ __forceinline__ bool grid_sync(unsigned* bar, long long limit, const int* status, int* s_abort,
+                                          int* s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!grid_barrier(bar, limit, status, *s_abort == 0)) *s_abort = 1;
+    *s_flag = *s_abort;
+  }
+  __syncthreads();
+  return *s_flag == 0;
+}
+
 // 2D tiled TMA load of box {c0.., r0..} into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0) {
   asm volatile(

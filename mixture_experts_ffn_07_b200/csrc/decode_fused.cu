@@ -70,32 +70,8 @@ struct DecodeArgs {
   long long wait_limit;
 };
 
-// One thread per CTA.  Returns false when the wait gave up (or wait == false).
-__device__ __forceinline__ bool grid_barrier(long long limit, const int* status, bool wait) {
-  __threadfence();
-  const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
-  const unsigned old = atomicAdd(&g_decode_barrier, add);
-  if (!wait) return false;
-  const long long t0 = clock64();
-  while (true) {
-    unsigned cur;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(&g_decode_barrier) : "memory");
-    if ((cur ^ old) & 0x80000000u) break;
-    if (*reinterpret_cast<const volatile int*>(status) != 0 || clock64() - t0 > limit) return false;
-  }
-  __threadfence();
-  return true;
-}
-
-// All threads of the CTA; false once this CTA has given up on a barrier.
 __device__ __forceinline__ bool cta_grid_sync(const DecodeArgs& a, int* s_abort, int* s_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    if (!grid_barrier(a.wait_limit, a.status, *s_abort == 0)) *s_abort = 1;
-    *s_flag = *s_abort;
-  }
-  __syncthreads();
-  return *s_flag == 0;
+  return grid_sync(&g_decode_barrier, a.wait_limit, a.status, s_abort, s_flag);
 }
 
 // Partial logits of a block of router rows for one (hidden chunk, token group):

@@ -207,12 +207,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------------------------------------ TMA producer
       uint32_t kbg = 0, outstanding = 0, out_phase = 0;
       bool skipped = false;
-      const uint64_t pol_w = l2_policy_evict_first();  // weights: read once
+      const uint64_t pol_w = l2_policy_evict_first();  // weights of a group with one row tile: read once
       const uint64_t pol_a = l2_policy_evict_last();   // activation rows: read by every column tile
       for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
         int g, mt, nt, ks;
         decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
         const int a_row = aux.row_off[g] + mt * BM;
+        const bool one_mtile = aux.cnt[g] <= BM;
         const int b_row = g * p.N + nt * p.col_step;
         const int kb0 = ks * p.kb_per_split, kb1 = min(nkb, kb0 + p.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
@@ -228,11 +229,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t* sb = sa + A_BYTES;
           mbar_arrive_expect_tx(&aux.full[s], STAGE_BYTES);
           tma_load_2d_hint(sa, &mapA, &aux.full[s], kb * BK, a_row, pol_a);
-          if (DUAL) {
+          if (one_mtile) {  // the weight tile is not needed again
             tma_load_2d_hint(sb, &mapB0, &aux.full[s], kb * BK, b_row, pol_w);
-            tma_load_2d_hint(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row, pol_w);
-          } else {
-            tma_load_2d_hint(sb, &mapB0, &aux.full[s], kb * BK, b_row, pol_w);
+            if (DUAL) tma_load_2d_hint(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row, pol_w);
+          } else {  // the group's other row tiles read it again: default L2 policy
+            tma_load_2d(sb, &mapB0, &aux.full[s], kb * BK, b_row);
+            if (DUAL) tma_load_2d(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row);
           }
           outstanding |= 1u << s;
           out_phase = (out_phase & ~(1u << s)) | (ph << s);

@@ -124,4 +124,31 @@ struct DecodeLayer {
 size_t decode_router_parts_floats(int T, int H, int E, bool shared_gate);
 cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L);
 
+
+// Top-K selection (from the router GEMM's output), stable permutation and
+// x-row gather of the tensor-core path in one cooperative launch
+// (prefill_front.cu).  Writes the same workspace regions as
+// router_topk + permute + gather_rows, and the same values.
+constexpr int kMaxFrontCtas = 256;
+struct PrefillFront {
+  const float* parts;  // split-K partial logits (nparts > 0), part_stride apart; else logits already complete
+  int nparts;
+  size_t part_stride;
+  float* logits;
+  const float* bias;
+  int T, E, K, renorm, H;
+  int32_t* ids;
+  float* w;
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* w_s;  // shared-gate row or nullptr
+  float* shared_gate;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_pairs;
+  int32_t* pair_pos;
+  __nv_bfloat16* x_perm;
+  int32_t* hist;  // kMaxFrontCtas * E ints of scratch
+};
+cudaError_t launch_prefill_front(const Ctx& c, const PrefillFront& f);
+
 }  // namespace moe

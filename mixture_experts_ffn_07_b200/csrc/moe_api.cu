@@ -34,6 +34,7 @@ std::atomic<uint64_t> g_launches{0};
 std::atomic<long long> g_wait_limit{1LL << 31};
 std::atomic<int> g_skip_stage{0};
 std::atomic<int> g_fused_decode{1};
+std::atomic<int> g_fused_front{1};
 
 struct TraceRec {
   const char* name;
@@ -82,6 +83,10 @@ bool tensor_router(const moe_desc& d) {
   return d.act_dtype == MOE_BF16 && d.router_dtype == MOE_BF16 && d.T > 64 && d.E % 32 == 0;
 }
 
+// Selection, permutation and row gather as one cooperative kernel after the
+// tensor-core router GEMM (prefill_front.cu).
+bool fused_front(const moe_desc& d) { return tensor_path(d) && tensor_router(d); }
+
 // The whole layer as one cooperative kernel (decode_fused.cu): the streaming
 // path with at most 64 tokens.
 bool fused_decode(const moe_desc& d) {
@@ -115,8 +120,8 @@ moe_status check_desc(const moe_desc* d) {
 }
 
 struct Layout {
-  size_t logits, logit_parts, router_parts, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos, y_slots,
-      x_perm, h, h_s, y_s, total;
+  size_t logits, logit_parts, router_parts, front_hist, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos,
+      y_slots, x_perm, h, h_s, y_s, total;
 };
 
 Layout layout_of(const moe_desc& d) {
@@ -132,6 +137,7 @@ Layout layout_of(const moe_desc& d) {
   L.logits = take(T * E * 4);
   L.logit_parts = tensor_router(d) ? take(router_ksplit(d) * T * E * 4) : 0;
   L.router_parts = fused_decode(d) ? take(moe::decode_router_parts_floats(d.T, d.H, d.E, shared_gated(d)) * 4) : 0;
+  L.front_hist = fused_front(d) ? take(static_cast<size_t>(moe::kMaxFrontCtas) * E * 4) : 0;
   L.ids = take(P * 4);
   L.w = take(P * 4);
   L.shared_gate = take(T * 4);
@@ -163,6 +169,30 @@ moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR
 
 // ---------------------------------------------------------------- stages
 // parts: scratch for the split-K partial logits (nullptr: no split).
+// The tensor-core router GEMM: logits (or, with `parts`, split-K partials
+// that the selection adds in order).  Returns the number of partial arrays
+// (0: the logits are complete) through *nparts.
+moe_status router_gemm(const moe::Ctx& c, const moe_desc& d, const void* x, const moe_weights& w, float* logits,
+                       float* parts, int* nparts) {
+  const int ksplit = parts ? moe::effective_ksplit(router_ksplit(d), d.H) : 1;
+  moe::GemmArgs a{};
+  a.A = static_cast<const __nv_bfloat16*>(x);
+  a.rows_A = d.T;
+  a.Kdim = d.H;
+  a.B0 = static_cast<const __nv_bfloat16*>(w.router);
+  a.N = d.E;
+  a.G = 1;
+  a.max_rows = d.T;
+  a.dual = false;
+  a.out_f32 = ksplit > 1 ? parts : logits;
+  a.ksplit = ksplit;
+  a.part_stride = static_cast<size_t>(d.T) * d.E;
+  a.name = "router_gemm";
+  MOE_TRY(moe::launch_grouped_gemm(c, a));
+  *nparts = ksplit > 1 ? ksplit : 0;
+  return MOE_OK;
+}
+
 moe_status route_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const moe_weights& w, float* logits,
                       float* parts, int32_t* ids, float* tw, float* shared_gate) {
   const void* w_s = shared_gated(d) ? w.sh_gate_w : nullptr;
@@ -195,13 +225,14 @@ moe_status route_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const
 
 moe_status expert_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const moe_weights& w,
                        const int32_t* offsets, const int32_t* sorted_pairs, const float* tw, float* y_slots, void* ws,
-                       const Layout& L) {
+                       const Layout& L, bool rows_gathered = false) {
   const int P = d.T * d.top_k;
   if (tensor_path(d)) {
     __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.x_perm);
     __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
-    MOE_TRY(moe::launch_gather_rows(c, static_cast<const __nv_bfloat16*>(x), sorted_pairs, offsets, d.E, d.top_k, P,
-                                    d.H, xp));
+    if (!rows_gathered)
+      MOE_TRY(moe::launch_gather_rows(c, static_cast<const __nv_bfloat16*>(x), sorted_pairs, offsets, d.E, d.top_k,
+                                      P, d.H, xp));
     moe::GemmArgs a{};
     a.A = xp;
     a.rows_A = P;
@@ -535,6 +566,44 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
     if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorInvalidValue) return MOE_ERR_CUDA;
     cudaGetLastError();
   }
+  if (fused_front(*d) && g_fused_front.load()) {
+    int nparts = 0;
+    if ((st = router_gemm(c, *d, x, *w, logits, parts, &nparts)) != MOE_OK) return st;
+    moe::PrefillFront f{};
+    f.parts = parts;
+    f.nparts = nparts;
+    f.part_stride = static_cast<size_t>(d->T) * d->E;
+    f.logits = logits;
+    f.bias = d->has_router_bias ? w->router_bias : nullptr;
+    f.T = d->T;
+    f.E = d->E;
+    f.K = d->top_k;
+    f.renorm = d->renormalize;
+    f.H = d->H;
+    f.ids = ids;
+    f.w = tw;
+    f.x = static_cast<const __nv_bfloat16*>(x);
+    f.w_s = shared_gated(*d) ? static_cast<const __nv_bfloat16*>(w->sh_gate_w) : nullptr;
+    f.shared_gate = sg;
+    f.counts = at<int32_t>(ws, L.counts);
+    f.offsets = offsets;
+    f.sorted_pairs = sorted_pairs;
+    f.pair_pos = at<int32_t>(ws, L.pair_pos);
+    f.x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+    f.hist = at<int32_t>(ws, L.front_hist);
+    const cudaError_t e = moe::launch_prefill_front(c, f);
+    bool gathered = e == cudaSuccess;
+    if (!gathered) {  // the grid cannot be made resident: the three steps as separate launches
+      if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorInvalidValue) return MOE_ERR_CUDA;
+      cudaGetLastError();
+      const void* w_s = shared_gated(*d) ? w->sh_gate_w : nullptr;
+      MOE_TRY(moe::launch_router_topk(c, parts, nparts, f.part_stride, logits, f.bias, d->T, d->E, d->top_k,
+                                      d->renormalize, ids, tw, x, d->act_dtype, w_s, d->router_dtype, d->H, sg));
+      MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, f.counts, offsets, sorted_pairs, f.pair_pos));
+    }
+    if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L, gathered)) != MOE_OK) return st;
+    return combine_impl(c, *d, y_slots, x, *w, sg, out, ws, L);
+  }
   if ((st = route_impl(c, *d, x, *w, logits, parts, ids, tw, sg)) != MOE_OK) return st;
   MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, at<int32_t>(ws, L.counts), offsets, sorted_pairs,
                               at<int32_t>(ws, L.pair_pos)));
@@ -634,5 +703,7 @@ void moe_debug_set_wait_limit(int64_t cycles) { g_wait_limit.store(cycles > 0 ? 
 void moe_debug_set_skip_stage(int enable) { g_skip_stage.store(enable ? 1 : 0); }
 
 void moe_set_fused_decode(int enable) { g_fused_decode.store(enable ? 1 : 0); }
+
+void moe_set_fused_front(int enable) { g_fused_front.store(enable ? 1 : 0); }
 
 }  // extern "C"

@@ -1,0 +1,226 @@
+// Selection, permutation and row gather of the tensor-core path in one
+// cooperative launch, after the router GEMM.
+//
+// The three steps are the ones of router_topk_kernel, permute_kernel and
+// gather_rows_kernel (hf2q softmax_topk_renorm_cpu for the selection;
+// DS4Server gather_sort for the stable expert order and the gathered rows),
+// which as separate launches each pay a launch and a ramp for a few
+// microseconds of work.  Here CTA c owns a contiguous block of tokens:
+//   A  a warp per token adds the router GEMM's split-K partials in order and
+//      selects (topk_token, shared with router_topk_kernel, so the ids equal
+//      moe_route's bit for bit); the CTA counts its pairs per expert and
+//      publishes the counts in hist[c][*];                         -- barrier
+//   B  every CTA adds the published counts (totals, and the counts of the
+//      CTAs before it), scans them into expert offsets, places its own pairs
+//      in pair order (a stable counting sort, so the permutation is unique),
+//      writes sorted_pairs / pair_pos and copies each pair's x row into its
+//      place in x_perm.
+// The grid barrier is the bounded counter barrier of common.cuh on a counter
+// of its own; the kernel asks for more than half of an SM's shared memory so
+// that no two of these grids are ever resident on one device together.
+#include <atomic>
+
+#include "route_util.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+
+__device__ unsigned g_front_barrier;
+
+struct FrontArgs {
+  const float* parts;  // split-K partial logits (nparts > 0) or nullptr
+  int nparts;
+  size_t part_stride;
+  float* logits;  // [T, E]
+  const float* bias;
+  int T, E, K, renorm, H;
+  int32_t* ids;
+  float* w;
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* w_s;
+  float* shared_gate;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_pairs;
+  int32_t* pair_pos;
+  __nv_bfloat16* x_perm;
+  int32_t* hist;  // [gridDim.x, E]
+  int* status;
+  long long wait_limit;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
+  __shared__ int s_hist[256], s_run[256], s_tot[256], s_off[257];
+  __shared__ int s_abort, s_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x, E = a.E, K = a.K;
+  const int t0 = static_cast<int>(static_cast<long long>(a.T) * c / G);
+  const int t1 = static_cast<int>(static_cast<long long>(a.T) * (c + 1) / G);
+  const int p0 = t0 * K, p1 = t1 * K;
+  if (threadIdx.x == 0) s_abort = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  pdl_trigger();
+  pdl_wait();  // the router GEMM's logits are complete and visible
+
+  // ---- A: selection of this CTA's tokens, and its pair counts
+  for (int t = t0 + warp; t < t1; t += kWarps)
+    topk_token<__nv_bfloat16, __nv_bfloat16>(a.parts, a.nparts, a.part_stride, a.logits, a.bias, E, K, a.renorm,
+                                             a.ids, a.w, a.x, a.w_s, a.H, a.shared_gate, t);
+  __syncthreads();
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&s_hist[a.ids[p]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) a.hist[static_cast<size_t>(c) * E + e] = s_hist[e];
+  if (!grid_sync(&g_front_barrier, a.wait_limit, a.status, &s_abort, &s_flag)) {
+    // some CTA's counts may be missing: placing pairs could go out of range
+    if (threadIdx.x == 0) record_status(a.status, MOE_ERR_TIMEOUT);
+    return;
+  }
+
+  // ---- B: offsets, this CTA's pair positions and rows
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_run[e] = 0;
+  __syncthreads();
+  {  // totals and the counts of the CTAs before this one: all G x E counts requested 8 at a time
+    const int n = G * E;
+#pragma unroll 1
+    for (int i0 = threadIdx.x; i0 < n; i0 += blockDim.x * 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + j * blockDim.x;
+        v[j] = i < n ? __ldcg(a.hist + i) : 0;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + j * blockDim.x;
+        if (i < n && v[j]) {
+          const int cc = i / E, e = i - cc * E;
+          atomicAdd(&s_tot[e], v[j]);
+          if (cc < c) atomicAdd(&s_run[e], v[j]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the totals (E <= 256: 8 per lane)
+    int loc[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      loc[i] = e < E ? s_tot[e] : 0;
+      sum += loc[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      if (e < E) s_off[e] = run;
+      run += loc[i];
+    }
+    if (lane == 31) s_off[E] = incl;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    s_run[e] += s_off[e];  // where this CTA's first pair of expert e goes
+    if (c == 0) {
+      a.counts[e] = s_tot[e];
+      a.offsets[e] = s_off[e];
+    }
+  }
+  if (c == 0 && threadIdx.x == 0) a.offsets[E] = s_off[E];
+  __syncthreads();
+  if (warp == 0) {  // in pair order, 32 at a time; equal experts ranked by lane
+    for (int base = p0; base < p1; base += 32) {
+      const int p = base + lane;
+      const int e = p < p1 ? a.ids[p] : -1;
+      const unsigned m = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(m & ((1u << lane) - 1u));
+      const int before = p < p1 ? s_run[e] : 0;
+      __syncwarp();
+      if (p < p1) {
+        const int pos = before + rank;
+        a.sorted_pairs[pos] = p;
+        a.pair_pos[p] = pos;
+        if (rank == 0) s_run[e] = before + __popc(m);
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  const int n16 = a.H / 8;  // 16-byte groups of a bf16 row
+  const uint4* src = reinterpret_cast<const uint4*>(a.x);
+  uint4* dst = reinterpret_cast<uint4*>(a.x_perm);
+  for (int p = p0 + warp; p < p1; p += kWarps) {
+    const uint4* s = src + static_cast<size_t>(p / K) * n16;
+    uint4* d = dst + static_cast<size_t>(a.pair_pos[p]) * n16;
+    for (int o = lane; o < n16; o += 32 * 4) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (o + 32 * j < n16) v[j] = __ldg(s + o + 32 * j);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (o + 32 * j < n16) d[o + 32 * j] = v[j];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_front(const Ctx& c, const PrefillFront& f) {
+  if (f.T <= 0) return cudaSuccess;
+  if (f.E > 256 || (f.H % 8)) return cudaErrorInvalidValue;
+  FrontArgs a{};
+  a.parts = f.parts;
+  a.nparts = f.nparts;
+  a.part_stride = f.part_stride;
+  a.logits = f.logits;
+  a.bias = f.bias;
+  a.T = f.T;
+  a.E = f.E;
+  a.K = f.K;
+  a.renorm = f.renorm;
+  a.H = f.H;
+  a.ids = f.ids;
+  a.w = f.w;
+  a.x = f.x;
+  a.w_s = f.w_s;
+  a.shared_gate = f.shared_gate;
+  a.counts = f.counts;
+  a.offsets = f.offsets;
+  a.sorted_pairs = f.sorted_pairs;
+  a.pair_pos = f.pair_pos;
+  a.x_perm = f.x_perm;
+  a.hist = f.hist;
+  a.status = c.status;
+  a.wait_limit = c.wait_limit;
+  // more than half of an SM's shared memory: one CTA per SM, one such grid per device
+  const int smem = c.smem_optin / 2 + 1024;
+  const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(front_kernel), smem);
+  if (e != cudaSuccess) return e;
+  KernelScope ks(c, "route_permute_gather");
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(std::min(c.num_sms, kMaxFrontCtas));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the launch overlaps the router GEMM's tail
+  attr[1].val.programmaticStreamSerializationAllowed = c.pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, front_kernel, a);
+}
+
+}  // namespace moe

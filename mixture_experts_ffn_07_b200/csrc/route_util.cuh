@@ -118,5 +118,62 @@ __device__ __forceinline__ void warp_topk(const float* row, const float* __restr
   }
 }
 
+
+// Selection for token t by one warp, from logits in global memory: `nparts`
+// (<= 16) partial logit arrays of T*E floats, part_stride apart starting at `parts`,
+// are first added in order into logits[t] (nparts == 0: logits[t] already
+// holds them); then warp_topk with the bias in place.  With w_s the warp also
+// writes shared_gate[t] = sigmoid(w_s . x[t]) (lane l accumulates elements
+// 8l + 256u + q in order; warp_sum).
+template <typename XT, typename WT>
+__device__ __forceinline__ void topk_token(const float* parts, int nparts, size_t part_stride, float* logits,
+                                           const float* bias, int E, int K, int renorm, int32_t* ids, float* wout,
+                                           const XT* x, const WT* w_s, int H, float* shared_gate, int t) {
+  constexpr int kUnroll = 8;
+  const int lane = threadIdx.x & 31;
+  float* row = logits + static_cast<size_t>(t) * E;
+  if (nparts > 0) {  // all partials of an expert requested together, then added in range order
+    constexpr int kMaxParts = 16;
+    for (int e = lane; e < E; e += 32) {
+      const float* src = parts + static_cast<size_t>(t) * E + e;
+      float v[kMaxParts];
+#pragma unroll
+      for (int k = 0; k < kMaxParts; ++k) v[k] = k < nparts ? src[k * part_stride] : 0.f;
+      float sum = v[0];
+#pragma unroll
+      for (int k = 1; k < kMaxParts; ++k)
+        if (k < nparts) sum += v[k];
+      row[e] = sum;
+    }
+    __syncwarp();
+  }
+  warp_topk(row, bias, E, K, renorm, row, ids + static_cast<size_t>(t) * K, wout + static_cast<size_t>(t) * K);
+  if (w_s) {
+    const XT* xr = x + static_cast<size_t>(t) * H;
+    float acc = 0.f;
+    for (int base = lane * 8; base < H; base += 256 * kUnroll) {
+      Raw8<XT> xv[kUnroll];
+      Raw8<WT> wv[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (base + 256 * u < H) {
+          raw_load(xr + base + 256 * u, xv[u]);
+          raw_load(w_s + base + 256 * u, wv[u]);
+        }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (base + 256 * u < H) {
+          float a[8], b[8];
+          raw_decode(xv[u], a);
+          raw_decode(wv[u], b);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc = fmaf(a[q], b[q], acc);
+        }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) shared_gate[t] = 1.0f / (1.0f + expf(-acc));
+  }
+}
+
 }  // namespace
 }  // namespace moe

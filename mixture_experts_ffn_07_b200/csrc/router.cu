@@ -159,42 +159,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   pdl_wait();
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;
-  float* row = logits + static_cast<size_t>(t) * E;
-  if (nparts > 0) {
-    for (int e = lane; e < E; e += 32) {
-      const float* src = parts + static_cast<size_t>(t) * E + e;
-      float v = src[0];
-      for (int k = 1; k < nparts; ++k) v += src[k * part_stride];
-      row[e] = v;
-    }
-    __syncwarp();
-  }
-  warp_topk(row, bias, E, K, renorm, row, ids + static_cast<size_t>(t) * K, wout + static_cast<size_t>(t) * K);
-  if (w_s) {
-    const XT* xr = x + static_cast<size_t>(t) * H;
-    float acc = 0.f;
-    for (int base = lane * 8; base < H; base += 256 * kRowUnroll) {
-      Raw8<XT> xv[kRowUnroll];
-      Raw8<WT> wv[kRowUnroll];
-#pragma unroll
-      for (int u = 0; u < kRowUnroll; ++u)
-        if (base + 256 * u < H) {
-          raw_load(xr + base + 256 * u, xv[u]);
-          raw_load(w_s + base + 256 * u, wv[u]);
-        }
-#pragma unroll
-      for (int u = 0; u < kRowUnroll; ++u)
-        if (base + 256 * u < H) {
-          float a[8], b[8];
-          raw_decode(xv[u], a);
-          raw_decode(wv[u], b);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc = fmaf(a[q], b[q], acc);
-        }
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) shared_gate[t] = 1.0f / (1.0f + expf(-acc));
-  }
+  (void)lane;
+  topk_token(parts, nparts, part_stride, logits, bias, E, K, renorm, ids, wout, x, w_s, H, shared_gate, t);
 }
 
 template <typename XT, typename WT>
