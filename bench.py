@@ -74,6 +74,10 @@ def algorithmic(spec, counts):
         k["shared_down_gemm"] = dict(bytes=Is * H * wb + T * Is * hb + T * H * 4, flops=2.0 * T * H * Is)
     layer = dict(bytes=touched * 3 * I * H * wb + E * H * rb + (3 * Is * H * wb if Is else 0) + 2 * T * H * ab,
                  flops=2.0 * (T * E * H + P * 3 * H * I + T * 3 * H * Is))
+    # fused launches: the sum of the steps they replace
+    k["route_permute_gather"] = dict(bytes=sum(k[n]["bytes"] for n in ("router_topk", "permute", "gather_rows")),
+                                     flops=0)
+    k["decode_layer"] = dict(layer)  # the whole layer in one launch
     return k, layer, touched
 
 
@@ -145,9 +149,10 @@ def _traffic(kernel: str, workload: str):
     rec = d.get(f"{kernel}@{workload}")
     if not rec:
         return None
-    src = os.path.join(ROOT, "mixture_experts_ffn_07_b200", "csrc", rec["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha"]:
-        return None
+    for name, sha in rec["sources"].items():  # every source the kernel is built from, unchanged
+        src = os.path.join(ROOT, "mixture_experts_ffn_07_b200", "csrc", name)
+        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != sha:
+            return None
     return rec["bytes_per_launch"]
 
 
