@@ -40,7 +40,16 @@ class _Desc(ctypes.Structure):
                 ("K", ctypes.c_int64), ("act", ctypes.c_int32), ("renormalize", ctypes.c_int32),
                 ("act_dtype", ctypes.c_int32), ("w_dtype", ctypes.c_int32), ("router_dtype", ctypes.c_int32),
                 ("has_router_bias", ctypes.c_int32), ("shared_I", ctypes.c_int64),
-                ("has_shared_gate", ctypes.c_int32)]
+                ("has_shared_gate", ctypes.c_int32), ("gating", ctypes.c_int32), ("n_groups", ctypes.c_int64),
+                ("topk_groups", ctypes.c_int64)]
+
+
+class _Route(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int64), ("K", ctypes.c_int64), ("renorm", ctypes.c_int), ("gating", ctypes.c_int),
+                ("n_groups", ctypes.c_int64), ("topk_groups", ctypes.c_int64)]
+
+
+GATING = {"softmax": 0, "sigmoid": 1}
 
 
 class _Tensors(ctypes.Structure):
@@ -60,8 +69,8 @@ def bind(lib):
     lib.ora_act.restype = ctypes.c_double
     lib.ora_sigmoid.argtypes = [ctypes.c_double]
     lib.ora_sigmoid.restype = ctypes.c_double
-    lib.ora_select.argtypes = [p, i64, i64, i64, i32, p, p]
-    lib.ora_weights_for.argtypes = [p, i64, i64, i64, i32, p, p]
+    lib.ora_select.argtypes = [p, i64, p, p, p]
+    lib.ora_weights_for.argtypes = [p, i64, p, p, p]
     lib.ora_permute.argtypes = [p, i64, i64, p, p, p, p]
     lib.ora_permute.restype = i32
     lib.ora_expert.argtypes = [p, p, i64, i64, p]
@@ -109,11 +118,15 @@ class Layer:
     sh_up: np.ndarray | None = None
     sh_down: np.ndarray | None = None
     sh_gate_w: np.ndarray | None = None
+    gating: str = "softmax"
+    n_groups: int = 1
+    topk_groups: int = 1
 
     def _c(self):
         d = _Desc(self.T, self.H, self.E, self.I, self.K, ACT[self.act], int(self.renormalize),
                   DTYPE[self.act_dtype], DTYPE[self.w_dtype], DTYPE[self.router_dtype],
-                  int(self.bias is not None), self.shared_I, int(self.sh_gate_w is not None))
+                  int(self.bias is not None), self.shared_I, int(self.sh_gate_w is not None), GATING[self.gating],
+                  self.n_groups, self.topk_groups)
         keep = []
 
         def ptr(a, dt=None):
@@ -134,7 +147,8 @@ def from_workload(wl) -> Layer:
     return Layer(T=s.T, H=s.H, E=s.E, I=s.I, K=s.K, act=s.act, renormalize=s.renormalize, act_dtype=s.act_dtype,
                  w_dtype=s.w_dtype, router_dtype=s.router_dtype, x=wl.x, router=wl.router, gate=wl.gate, up=wl.up,
                  down=wl.down, bias=wl.router_bias, shared_I=s.shared_I, sh_gate=wl.sh_gate, sh_up=wl.sh_up,
-                 sh_down=wl.sh_down, sh_gate_w=wl.sh_gate_w)
+                 sh_down=wl.sh_down, sh_gate_w=wl.sh_gate_w, gating=getattr(s, "gating", "softmax"),
+                 n_groups=getattr(s, "n_groups", 1), topk_groups=getattr(s, "topk_groups", 1))
 
 
 def _tok(tokens, n_default):
@@ -173,23 +187,27 @@ def logits(L: Layer, tokens=None):
     return out, am
 
 
-def select(logit_rows: np.ndarray, K: int, renormalize: bool = True):
-    """Selection (l desc, e asc; first K) and weights from given logits [n,E] (any float dtype, widened exactly)."""
+def select(logit_rows: np.ndarray, K: int, renormalize: bool = True, gating: str = "softmax", n_groups: int = 1,
+           topk_groups: int = 1):
+    """Selection (l desc, e asc; first K, among the topk_groups best of n_groups groups) and weights from given
+    logits [n,E] (any float dtype, widened exactly)."""
     l = np.ascontiguousarray(logit_rows, np.float64)
     n, E = l.shape
     ids = np.zeros((n, K), np.int32)
     w = np.zeros((n, K), np.float64)
-    _lib().ora_select(l.ctypes.data, n, E, K, int(renormalize), ids.ctypes.data, w.ctypes.data)
+    r = _Route(E, K, int(renormalize), GATING[gating], n_groups, topk_groups)
+    _lib().ora_select(l.ctypes.data, n, ctypes.byref(r), ids.ctypes.data, w.ctypes.data)
     return ids, w
 
 
-def weights_for(logit_rows: np.ndarray, ids: np.ndarray, renormalize: bool = True):
+def weights_for(logit_rows: np.ndarray, ids: np.ndarray, renormalize: bool = True, gating: str = "softmax"):
     l = np.ascontiguousarray(logit_rows, np.float64)
     n, E = l.shape
     ids = np.ascontiguousarray(ids, np.int32)
     K = ids.shape[1]
     w = np.zeros((n, K), np.float64)
-    _lib().ora_weights_for(l.ctypes.data, n, E, K, int(renormalize), ids.ctypes.data, w.ctypes.data)
+    r = _Route(E, K, int(renormalize), GATING[gating], 1, 1)
+    _lib().ora_weights_for(l.ctypes.data, n, ctypes.byref(r), ids.ctypes.data, w.ctypes.data)
     return w
 
 

@@ -13,10 +13,19 @@
  *                ferrox-models decoder.rs, gpt_oss_ffn: bias added to logits)
  *   2. select   experts ordered by (l descending, e ascending); ids = first K
  *               (hf2q qwen35/gpu_ffn.rs, softmax_topk_renorm_cpu: full stable
- *                sort of all experts, then the first K)
- *   3. weights  p_e = exp(l_e - m) / sum_j exp(l_j - m), m = max_e l_e;
+ *                sort of all experts, then the first K).
+ *               Group-limited (ferrox-models decoder.rs calls
+ *               route_top_k_grouped(logits, n_groups, groups used, K, ...)
+ *               when the model has expert groups; its body is not printed):
+ *               the E experts form n_groups contiguous groups of E/n_groups;
+ *               a group's score is its largest logit; the topk_groups groups
+ *               with the highest scores (lower group index first on ties)
+ *               stay eligible and the K experts are chosen among them.
+ *   3. weights  softmax gating: p_e = exp(l_e - m) / sum_j exp(l_j - m),
+ *               m = max_e l_e; sigmoid gating (GatingFunction, the other
+ *               router the pages name): p_e = 1 / (1 + exp(-l_e));
  *               renormalised: w_k = p_id_k / sum_k' p_id_k'; else w_k = p_id_k
- *               (same function; its 1e-20 guards are kept)
+ *               (softmax_topk_renorm_cpu; its 1e-20 guards are kept)
  *   4. permute  counts[e], exclusive offsets, pair ids p = t K + k stably
  *               sorted by expert, and the inverse pair_pos
  *               (DS4Server qwen_mtplx.rs, gather_sort: argsort of the flat
@@ -47,6 +56,8 @@
 enum { ORA_F32 = 0, ORA_BF16 = 1, ORA_Q8_0 = 2 };
 enum { ORA_SILU = 0, ORA_GELU_TANH = 1 };
 
+enum { ORA_GATING_SOFTMAX = 0, ORA_GATING_SIGMOID = 1 };
+
 typedef struct {
   int64_t T, H, E, I, K;
   int32_t act, renormalize;
@@ -54,7 +65,16 @@ typedef struct {
   int32_t has_router_bias;
   int64_t shared_I;
   int32_t has_shared_gate;
+  int32_t gating;                /* ORA_GATING_* */
+  int64_t n_groups, topk_groups; /* group-limited selection when n_groups > 1 */
 } ora_desc;
+
+/* How one token's experts are chosen and weighted. */
+typedef struct {
+  int64_t E, K;
+  int renorm, gating;
+  int64_t n_groups, topk_groups;
+} ora_route;
 
 typedef struct {
   const void* x;          /* [T,H] act_dtype */
@@ -156,8 +176,12 @@ static int by_logit_desc_index_asc(const void* pa, const void* pb) {
   return (a->e > b->e) - (a->e < b->e);
 }
 
-/* Probabilities of all experts (max-subtracted softmax). */
-static void softmax_all(const double* l, int64_t E, double* p) {
+/* Gate values of all experts: max-subtracted softmax, or elementwise sigmoid. */
+static void gate_all(const double* l, int64_t E, int gating, double* p) {
+  if (gating == ORA_GATING_SIGMOID) {
+    for (int64_t e = 0; e < E; ++e) p[e] = 1.0 / (1.0 + exp(-l[e]));
+    return;
+  }
   double m = -INFINITY;
   for (int64_t e = 0; e < E; ++e)
     if (l[e] > m) m = l[e];
@@ -182,40 +206,77 @@ static void weights_of(const double* p, const int32_t* ids, int64_t K, int renor
   for (int64_t k = 0; k < K; ++k) w[k] = p[ids[k]] * inv;
 }
 
-static void select_one(const double* l, int64_t E, int64_t K, int renorm, ora_key* keys, double* p, int32_t* ids,
-                       double* w) {
-  for (int64_t e = 0; e < E; ++e) {
-    keys[e].l = l[e];
-    keys[e].e = (int32_t)e;
+/* keys[E] scratch; with groups, the experts of groups that are not among the
+ * topk_groups best are left out of the sort. */
+static void select_one(const double* l, const ora_route* r, ora_key* keys, double* p, int32_t* ids, double* w) {
+  const int64_t E = r->E, K = r->K;
+  int64_t n = 0;
+  if (r->n_groups > 1) {
+    const int64_t gs = E / r->n_groups;
+    ora_key* gkeys = keys; /* group scores first, in the same scratch */
+    for (int64_t g = 0; g < r->n_groups; ++g) {
+      double m = -INFINITY;
+      for (int64_t e = g * gs; e < (g + 1) * gs; ++e)
+        if (l[e] > m) m = l[e];
+      gkeys[g].l = m;
+      gkeys[g].e = (int32_t)g;
+    }
+    qsort(gkeys, (size_t)r->n_groups, sizeof(ora_key), by_logit_desc_index_asc);
+    char* keep = (char*)calloc((size_t)r->n_groups, 1);
+    for (int64_t i = 0; i < r->topk_groups; ++i) keep[gkeys[i].e] = 1;
+    for (int64_t e = 0; e < E; ++e)
+      if (keep[e / gs]) {
+        keys[n].l = l[e];
+        keys[n].e = (int32_t)e;
+        ++n;
+      }
+    free(keep);
+  } else {
+    for (int64_t e = 0; e < E; ++e) {
+      keys[e].l = l[e];
+      keys[e].e = (int32_t)e;
+    }
+    n = E;
   }
-  qsort(keys, (size_t)E, sizeof(ora_key), by_logit_desc_index_asc);
+  qsort(keys, (size_t)n, sizeof(ora_key), by_logit_desc_index_asc);
   for (int64_t k = 0; k < K; ++k) ids[k] = keys[k].e;
-  softmax_all(l, E, p);
-  weights_of(p, ids, K, renorm, w);
+  gate_all(l, E, r->gating, p);
+  weights_of(p, ids, K, r->renorm, w);
 }
 
 /* Selection + weights for n tokens from given logits [n,E] (e.g. the GPU's f32 logits widened to f64). */
-void ora_select(const double* logits, int64_t n, int64_t E, int64_t K, int renorm, int32_t* ids, double* w) {
+void ora_select(const double* logits, int64_t n, const ora_route* r, int32_t* ids, double* w) {
+  const int64_t E = r->E, K = r->K;
 #pragma omp parallel
   {
     ora_key* keys = (ora_key*)malloc(sizeof(ora_key) * E);
     double* p = (double*)malloc(sizeof(double) * E);
 #pragma omp for schedule(static)
-    for (int64_t t = 0; t < n; ++t) select_one(logits + t * E, E, K, renorm, keys, p, ids + t * K, w + t * K);
+    for (int64_t t = 0; t < n; ++t) select_one(logits + t * E, r, keys, p, ids + t * K, w + t * K);
     free(keys);
     free(p);
   }
 }
 
 /* Weights of a forced selection ids[n,K] from logits [n,E]. */
-void ora_weights_for(const double* logits, int64_t n, int64_t E, int64_t K, int renorm, const int32_t* ids,
-                     double* w) {
-  double* p = (double*)malloc(sizeof(double) * E);
+void ora_weights_for(const double* logits, int64_t n, const ora_route* r, const int32_t* ids, double* w) {
+  double* p = (double*)malloc(sizeof(double) * r->E);
   for (int64_t t = 0; t < n; ++t) {
-    softmax_all(logits + t * E, E, p);
-    weights_of(p, ids + t * K, K, renorm, w + t * K);
+    gate_all(logits + t * r->E, r->E, r->gating, p);
+    weights_of(p, ids + t * r->K, r->K, r->renorm, w + t * r->K);
   }
   free(p);
+}
+
+static ora_route route_of(const ora_desc* d) {
+  ora_route r;
+  r.E = d->E;
+  r.K = d->K;
+  r.renorm = d->renormalize;
+  r.gating = d->gating;
+  r.n_groups = d->n_groups;
+  r.topk_groups = d->topk_groups;
+  return r;
 }
 
 /* ---- step 4: stable permutation of pair ids by expert (counting sort) ---- */
@@ -283,6 +344,7 @@ void ora_layer(const ora_desc* d, const ora_tensors* w, const int64_t* tokens, i
                double* out, double* logits_out, int32_t* ids_out, double* w_out, double* gate_s_out,
                double* absmax_out) {
   const int64_t H = d->H, E = d->E, I = d->I, K = d->K, Is = d->shared_I;
+  const ora_route rt = route_of(d);
   int64_t big = H;
   if (I > big) big = I;
   if (Is > big) big = Is;
@@ -305,10 +367,10 @@ void ora_layer(const ora_desc* d, const ora_tensors* w, const int64_t* tokens, i
       logits_one(d, w, xt, row, l, &am);
       if (force_ids) {
         for (int64_t k = 0; k < K; ++k) ids[k] = force_ids[i * K + k];
-        softmax_all(l, E, p);
+        gate_all(l, E, d->gating, p);
         weights_of(p, ids, K, d->renormalize, wk);
       } else {
-        select_one(l, E, K, d->renormalize, keys, p, ids, wk);
+        select_one(l, &rt, keys, p, ids, wk);
       }
       double* o = out + i * H;
       for (int64_t j = 0; j < H; ++j) o[j] = 0.0;

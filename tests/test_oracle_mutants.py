@@ -28,6 +28,13 @@ MUTANTS = {
     "slot_weight_index": ("o[j] += wk[k] * y[j];", "o[j] += wk[0] * y[j];"),
     "up_reads_gate": ("load_row(Wu, dtype, row0 + i, Hin, row);", "load_row(Wg, dtype, row0 + i, Hin, row);"),
     "fp16_exponent_bias": ("ldexp(1024.0 + man, ex - 25)", "ldexp(1024.0 + man, ex - 24)"),
+    "sigmoid_gating_ignored": ("if (gating == ORA_GATING_SIGMOID) {", "if (0) {"),
+    "sigmoid_sign": ("for (int64_t e = 0; e < E; ++e) p[e] = 1.0 / (1.0 + exp(-l[e]));",
+                     "for (int64_t e = 0; e < E; ++e) p[e] = 1.0 / (1.0 + exp(l[e]));"),
+    "group_score_min": ("if (l[e] > m) m = l[e];\n      gkeys", "if (m == -INFINITY || l[e] < m) m = l[e];\n      gkeys"),
+    "groups_kept_off_by_one": ("for (int64_t i = 0; i < r->topk_groups; ++i) keep[gkeys[i].e] = 1;",
+                               "for (int64_t i = 0; i <= r->topk_groups && i < r->n_groups; ++i) keep[gkeys[i].e] = 1;"),
+    "groups_ignored": ("if (r->n_groups > 1) {", "if (0) {"),
 }
 
 BATTERY = [
@@ -39,6 +46,9 @@ BATTERY = [
     lambda g: pins.test_dense_special_case("silu", "f32"),
     lambda g: pins.test_layer_matches_numpy_restatement(48, True, True),
     pins.test_shared_gate_linearity,
+    lambda g: pins.test_sigmoid_gating_known_values(), lambda g: pins.test_sigmoid_gating_equals_two_way_softmax(),
+    lambda g: pins.test_sigmoid_gating_selects_like_softmax(), lambda g: pins.test_grouped_worked_example(),
+    lambda g: pins.test_grouped_special_cases_and_brute_force(),
 ]
 
 

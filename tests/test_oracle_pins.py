@@ -303,3 +303,76 @@ def test_ungated_shared_is_added_with_scale_one():
     Ls = _tiny(T=4, E=4, K=2, shared_I=0)
     routed = oracle.layer(Ls)["out"]
     assert np.max(np.abs(full - (routed + y_s))) < 1e-13 * np.max(np.abs(full))
+
+
+# ---------------------------------------------------------------- routing variants (SURVEY next rows f-1, f-2)
+def test_sigmoid_gating_known_values():
+    """sigma(0) = 1/2 exactly; equal logits renormalise to exactly 1/K."""
+    _, w = oracle.select(np.zeros((1, 4)), 1, False, gating="sigmoid")
+    assert w[0, 0] == 0.5
+    _, w = oracle.select(np.full((1, 6), 0.37), 3, True, gating="sigmoid")
+    assert np.all(np.abs(w - 1.0 / 3.0) < 1e-15)
+
+
+def test_sigmoid_gating_equals_two_way_softmax():
+    """sigma(a) = e^a / (e^a + e^0): the sigmoid weight of a logit equals the softmax
+    weight of the same logit against a single zero logit (an identity, not the formula)."""
+    rng = np.random.default_rng(7)
+    for a in rng.normal(0, 4, 20):
+        _, ws = oracle.select(np.array([[a, -50.0, -60.0]]), 1, False, gating="sigmoid")
+        _, wm = oracle.select(np.array([[a, 0.0]]), 2, False, gating="softmax")
+        p_a = wm[0, 0] if a >= 0 else wm[0, 1]  # slot of logit a in the softmax selection
+        assert abs(ws[0, 0] - p_a) < 1e-14
+
+
+def test_sigmoid_gating_selects_like_softmax():
+    """sigmoid is increasing: the chosen experts and their order are the softmax ones;
+    renormalised weights sum to 1 and follow the logit order."""
+    rng = np.random.default_rng(8)
+    l = rng.normal(0, 2, (40, 32))
+    l[:, 5] = l[:, 6]  # ties keep the lower index
+    ids_m, _ = oracle.select(l, 6, True)
+    ids_s, w_s = oracle.select(l, 6, True, gating="sigmoid")
+    assert np.array_equal(ids_m, ids_s)
+    assert np.all(np.abs(w_s.sum(axis=1) - 1.0) < 1e-12)
+    assert np.all(np.diff(w_s, axis=1) <= 0)
+    _, w_n = oracle.select(l, 6, False, gating="sigmoid")
+    assert np.all((w_n > 0) & (w_n < 1)) and np.all(np.diff(w_n, axis=1) <= 0)
+
+
+def _grouped_brute(l, K, n_groups, topk_groups):
+    """Independent statement: group maxima by reshape, groups ranked by (max desc, index asc),
+    eligible experts ranked by (logit desc, index asc)."""
+    E = l.size
+    gs = E // n_groups
+    gmax = l.reshape(n_groups, gs).max(axis=1)
+    order_g = sorted(range(n_groups), key=lambda g: (-gmax[g], g))[:topk_groups]
+    elig = [e for e in range(E) if e // gs in order_g]
+    return sorted(elig, key=lambda e: (-l[e], e))[:K]
+
+
+def test_grouped_worked_example():
+    """E=8 in 4 groups of 2, 2 groups kept: group maxima (10, 6, 4, 9) keep groups 0 and 3,
+    so the third expert is the weak partner of the best one, not the 6 of group 1."""
+    l = np.array([[10.0, -5.0, 6.0, 5.0, 4.0, 4.0, 9.0, -9.0]])
+    ids, _ = oracle.select(l, 3, True, n_groups=4, topk_groups=2)
+    assert ids[0].tolist() == [0, 6, 1]
+    ids, _ = oracle.select(l, 3, True)
+    assert ids[0].tolist() == [0, 6, 2]
+
+
+def test_grouped_special_cases_and_brute_force():
+    rng = np.random.default_rng(9)
+    l = rng.normal(0, 1, (60, 16))
+    base, _ = oracle.select(l, 4, True)
+    one, _ = oracle.select(l, 4, True, n_groups=1, topk_groups=1)     # one group: plain top-K
+    assert np.array_equal(base, one)
+    each, _ = oracle.select(l, 4, True, n_groups=16, topk_groups=4)  # a group per expert, K groups: plain top-K
+    assert np.array_equal(base, each)
+    ties = np.round(rng.normal(0, 1, (60, 16)) * 2) / 2               # many equal logits and equal group maxima
+    for n_groups, topk_groups, K in ((4, 2, 3), (8, 3, 5), (2, 1, 8), (4, 4, 6)):
+        for rows in (l, ties):
+            ids, w = oracle.select(rows, K, True, n_groups=n_groups, topk_groups=topk_groups)
+            for t in range(rows.shape[0]):
+                assert ids[t].tolist() == _grouped_brute(rows[t], K, n_groups, topk_groups)
+            assert np.all(np.abs(w.sum(axis=1) - 1.0) < 1e-12)

@@ -137,6 +137,9 @@ class Spec:
     router_bias: str | None = None     # None | "zipf1.1"
     router_std: float = 0.02
     name: str = "custom"
+    gating: str = "softmax"            # "softmax" | "sigmoid"
+    n_groups: int = 1                  # group-limited selection when > 1
+    topk_groups: int = 1
 
     @property
     def P(self) -> int:
@@ -153,6 +156,9 @@ CONFIGS = {
                               router_bias="zipf1.1", name="skewed_zipf_t8192"),
     "q8_0_decode_t16": Spec(T=16, H=2048, E=128, I=768, K=8, act_dtype=F32, w_dtype=Q8_0, router_dtype=F32,
                             name="q8_0_decode_t16"),
+    # routing variants on the prefill shapes: sigmoid gating, 8 groups of 8 experts, 4 groups kept
+    "grouped_sigmoid_t512": Spec(T=512, H=2048, E=64, I=1024, K=8, gating="sigmoid", n_groups=8, topk_groups=4,
+                                 name="grouped_sigmoid_t512"),
 }
 CONFIG_ORDER = list(CONFIGS)
 BASE_SEED = 0xB2000000
