@@ -58,16 +58,27 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_Q8_0 = 2 } moe_dtype;
  * (mlx-native moe_dispatch.rs, fused_gelu_mul and its test oracle cpu_gelu). */
 typedef enum { MOE_ACT_SILU = 0, MOE_ACT_GELU_TANH = 1 } moe_act;
 
+/* Gate values from the (biased) logits l_e: softmax over all E experts
+ * (hf2q softmax_topk_renorm_cpu), or sigmoid 1/(1+e^-l_e) per expert (the
+ * other GatingFunction ferrox-models decoder.rs passes to its routers). */
+typedef enum { MOE_GATING_SOFTMAX = 0, MOE_GATING_SIGMOID = 1 } moe_gating;
+
 typedef struct moe_desc {
   int32_t T, H, E, I, top_k;
   int32_t act;             /* moe_act, used by routed and shared experts */
-  int32_t renormalize;     /* 1: selected weights divided by their sum; 0: plain softmax probabilities */
+  int32_t renormalize;     /* 1: selected gate values divided by their sum; 0: the gate values themselves */
   int32_t act_dtype;       /* MOE_F32 | MOE_BF16: x and out */
   int32_t w_dtype;         /* MOE_F32 | MOE_BF16 | MOE_Q8_0: expert and shared projections */
   int32_t router_dtype;    /* MOE_F32 | MOE_BF16: router W and the shared-gate vector w_s */
   int32_t has_router_bias; /* 1: logits += b_e before selection (ferrox-models decoder.rs, gpt_oss_ffn) */
   int32_t shared_I;        /* 0: no shared expert */
   int32_t has_shared_gate; /* 1: shared output scaled by sigmoid(w_s . x); 0: scale 1 */
+  int32_t gating;          /* moe_gating (0: softmax) */
+  int32_t n_groups;        /* 0 or 1: plain top-K.  > 1: group-limited selection (ferrox-models decoder.rs,
+                              route_top_k_grouped): the experts form n_groups contiguous groups of E/n_groups,
+                              a group scores its largest logit and only the topk_groups best groups (lower
+                              index on ties) are eligible.  E % n_groups == 0, n_groups <= 32. */
+  int32_t topk_groups;     /* groups kept: 1 <= topk_groups <= n_groups, top_k <= topk_groups * E / n_groups */
 } moe_desc;
 
 /*
@@ -136,7 +147,8 @@ moe_status moe_workspace_regions(const moe_desc* d, moe_ws_regions* r);
  *  x        [T,H] act_dtype
  *  logits   [T,E] f32 out: x W_r^T (+ b), the values selection compared
  *  topk_ids [T,K] int32 out: experts in order (logit desc, index asc)
- *  topk_w   [T,K] f32 out: exp(l - m) over the selected (renormalised) or over all E
+ *  topk_w   [T,K] f32 out: the selected experts' gate values (moe_gating), divided by their sum
+ *           when renormalize
  *  shared_gate [T] f32 out: sigmoid(w_s . x); required iff shared_I > 0 and has_shared_gate
  *  ws, ws_bytes: optional workspace (NULL, or >= moe_workspace_bytes(d)).  With it,
  *           a bf16 batch splits the logits GEMM over the hidden dimension into

@@ -22,6 +22,7 @@ from ._lib import (MOE_ACT_GELU_TANH, MOE_ACT_SILU, MOE_BF16, MOE_ERR_CUDA, MOE_
 
 DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "q8_0": MOE_Q8_0}
 ACTS = {"silu": MOE_ACT_SILU, "gelu_tanh": MOE_ACT_GELU_TANH}
+GATINGS = {"softmax": 0, "sigmoid": 1}  # moe_gating
 
 
 @dataclass
@@ -39,11 +40,15 @@ class Desc:
     has_router_bias: bool = False
     shared_I: int = 0
     has_shared_gate: bool = False
+    gating: str = "softmax"
+    n_groups: int = 0
+    topk_groups: int = 0
 
     def c(self) -> _lib.MoeDesc:
         return _lib.MoeDesc(self.T, self.H, self.E, self.I, self.top_k, ACTS[self.act], int(self.renormalize),
                             DTYPES[self.act_dtype], DTYPES[self.w_dtype], DTYPES[self.router_dtype],
-                            int(self.has_router_bias), self.shared_I, int(self.has_shared_gate))
+                            int(self.has_router_bias), self.shared_I, int(self.has_shared_gate),
+                            GATINGS[self.gating], self.n_groups, self.topk_groups)
 
     @property
     def P(self) -> int:

@@ -29,7 +29,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route
 class MoeDesc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "H", "E", "I", "top_k", "act", "renormalize", "act_dtype", "w_dtype", "router_dtype",
-                 "has_router_bias", "shared_I", "has_shared_gate")]
+                 "has_router_bias", "shared_I", "has_shared_gate", "gating", "n_groups", "topk_groups")]
 
 
 class MoeWeights(ctypes.Structure):

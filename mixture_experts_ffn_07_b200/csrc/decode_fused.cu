@@ -52,6 +52,7 @@ struct DecodeArgs {
   const float* bias;
   const void* w_s;  // shared-gate row (router dtype) or nullptr
   int T, H, E, K, renorm, has_shared;
+  RouteCfg rc;
   Phase g, d;       // gate/up and down; pairs and row scales are set in the kernel
   int stage_bytes;  // dynamic shared memory before the pair arrays
   float* parts;     // [nch, T, R] chunk partials of the logits
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
         if (lane + 32 * i < R) row[lane + 32 * i] = l[i];
       __syncwarp();
       float* lout = blockIdx.x == 0 ? a.logits + static_cast<size_t>(t) * E : row;
-      warp_topk(row, a.bias, E, K, a.renorm, lout, s_ids + t * K, s_w + t * K);
+      warp_topk(row, a.bias, a.rc, lout, s_ids + t * K, s_w + t * K);
       if (a.w_s && lane == 0) {
         const float sg = 1.0f / (1.0f + expf(-row[E]));
         s_sgate[t] = sg;
@@ -454,6 +455,7 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
   a.E = L.E;
   a.K = L.K;
   a.renorm = L.renorm;
+  a.rc = L.rc;
   a.has_shared = L.Is > 0;
   a.g.K = L.K;
   a.g.act_fn = L.act;

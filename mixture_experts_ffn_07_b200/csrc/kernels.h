@@ -7,19 +7,28 @@
 
 namespace moe {
 
+// How a token's experts are chosen and weighted.
+struct RouteCfg {
+  int E, K, renorm;
+  int gating;       // MOE_GATING_SOFTMAX | MOE_GATING_SIGMOID
+  int n_groups;     // > 1: group-limited selection (E % n_groups == 0, n_groups <= 32)
+  int topk_groups;  // groups kept
+};
+
+
 // Softmax + top-K (+renorm) per token from logits in global memory, one warp
 // per token.  Adds the optional bias to the logits in place; with w_s also
 // writes shared_gate[t] = sigmoid(w_s . x[t]).
 // `nparts` partial logit arrays of T*E floats, part_stride apart starting at
 // `parts`, are summed in order into `logits` first.
 cudaError_t launch_router_topk(const Ctx& c, const float* parts, int nparts, size_t part_stride, float* logits,
-                               const float* bias, int T, int E, int K, int renorm, int32_t* ids, float* w,
+                               const float* bias, int T, const RouteCfg& rc, int32_t* ids, float* w,
                                const void* x, int x_dtype, const void* w_s, int w_dtype, int H, float* shared_gate);
 
 // Router in one launch for small batches: logits (+ the shared-gate row when
 // w_s != nullptr) by clusters of 8 CTAs, then softmax + top-K (+renorm) per token.
 cudaError_t launch_router_fused(const Ctx& c, const void* x, int x_dtype, const void* W, const void* w_s,
-                                int w_dtype, const float* bias, int T, int H, int E, int K, int renorm,
+                                int w_dtype, const float* bias, int T, int H, const RouteCfg& rc,
                                 float* logits, int32_t* ids, float* w, float* shared_gate);
 
 // Single-CTA stable counting sort of the P pair ids by expert.
@@ -104,6 +113,7 @@ struct DecodeLayer {
   const float* bias;   // router bias or nullptr
   const void* w_s;     // shared-gate row or nullptr
   int T, H, E, K, I, Is, act, renorm, w_dtype;
+  RouteCfg rc;  // E, K, renorm repeated with the gating and groups
   const void *gate, *up, *down, *gate_scale, *up_scale, *down_scale;
   const void *sh_gate, *sh_up, *sh_down, *sh_gate_scale, *sh_up_scale, *sh_down_scale;
   float* router_parts;  // decode_router_parts_floats(...) floats
@@ -137,6 +147,7 @@ struct PrefillFront {
   float* logits;
   const float* bias;
   int T, E, K, renorm, H;
+  RouteCfg rc;
   int32_t* ids;
   float* w;
   const __nv_bfloat16* x;

@@ -116,7 +116,25 @@ moe_status check_desc(const moe_desc* d) {
       (d->router_dtype != MOE_F32 && d->router_dtype != MOE_BF16))
     return MOE_ERR_INVALID_ARG;
   if (d->H % 32 || d->I % 32 || d->shared_I % 32) return MOE_ERR_UNSUPPORTED;
+  if (d->gating != MOE_GATING_SOFTMAX && d->gating != MOE_GATING_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (d->n_groups < 0 || d->n_groups > 32) return MOE_ERR_INVALID_ARG;
+  if (d->n_groups > 1) {
+    if (d->E % d->n_groups || d->topk_groups < 1 || d->topk_groups > d->n_groups ||
+        d->top_k > d->topk_groups * (d->E / d->n_groups))
+      return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
+}
+
+moe::RouteCfg route_cfg(const moe_desc& d) {
+  moe::RouteCfg r{};
+  r.E = d.E;
+  r.K = d.top_k;
+  r.renorm = d.renormalize;
+  r.gating = d.gating;
+  r.n_groups = d.n_groups > 1 ? d.n_groups : 1;
+  r.topk_groups = d.n_groups > 1 ? d.topk_groups : 1;
+  return r;
 }
 
 struct Layout {
@@ -213,12 +231,12 @@ moe_status route_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const
     a.name = "router_gemm";
     MOE_TRY(moe::launch_grouped_gemm(c, a));
     MOE_TRY(moe::launch_router_topk(c, parts, ksplit > 1 ? ksplit : 0, a.part_stride, logits,
-                                    d.has_router_bias ? w.router_bias : nullptr, d.T, d.E, d.top_k, d.renormalize, ids,
-                                    tw, x, d.act_dtype, w_s, d.router_dtype, d.H, shared_gate));
+                                    d.has_router_bias ? w.router_bias : nullptr, d.T, route_cfg(d), ids, tw, x,
+                                    d.act_dtype, w_s, d.router_dtype, d.H, shared_gate));
   } else {
     MOE_TRY(moe::launch_router_fused(c, x, d.act_dtype, w.router, w_s, d.router_dtype,
-                                     d.has_router_bias ? w.router_bias : nullptr, d.T, d.H, d.E, d.top_k,
-                                     d.renormalize, logits, ids, tw, shared_gate));
+                                     d.has_router_bias ? w.router_bias : nullptr, d.T, d.H, route_cfg(d), logits, ids,
+                                     tw, shared_gate));
   }
   return MOE_OK;
 }
@@ -532,6 +550,7 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
     f.Is = d->shared_I;
     f.act = d->act;
     f.renorm = d->renormalize;
+    f.rc = route_cfg(*d);
     f.w_dtype = d->w_dtype;
     f.gate = w->gate;
     f.up = w->up;
@@ -580,6 +599,7 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
     f.K = d->top_k;
     f.renorm = d->renormalize;
     f.H = d->H;
+    f.rc = route_cfg(*d);
     f.ids = ids;
     f.w = tw;
     f.x = static_cast<const __nv_bfloat16*>(x);
@@ -597,8 +617,8 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
       if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorInvalidValue) return MOE_ERR_CUDA;
       cudaGetLastError();
       const void* w_s = shared_gated(*d) ? w->sh_gate_w : nullptr;
-      MOE_TRY(moe::launch_router_topk(c, parts, nparts, f.part_stride, logits, f.bias, d->T, d->E, d->top_k,
-                                      d->renormalize, ids, tw, x, d->act_dtype, w_s, d->router_dtype, d->H, sg));
+      MOE_TRY(moe::launch_router_topk(c, parts, nparts, f.part_stride, logits, f.bias, d->T, f.rc, ids, tw, x,
+                                      d->act_dtype, w_s, d->router_dtype, d->H, sg));
       MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, f.counts, offsets, sorted_pairs, f.pair_pos));
     }
     if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L, gathered)) != MOE_OK) return st;

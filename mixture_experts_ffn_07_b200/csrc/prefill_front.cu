@@ -38,6 +38,7 @@ struct FrontArgs {
   float* logits;  // [T, E]
   const float* bias;
   int T, E, K, renorm, H;
+  RouteCfg rc;
   int32_t* ids;
   float* w;
   const __nv_bfloat16* x;
@@ -68,8 +69,8 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
 
   // ---- A: selection of this CTA's tokens, and its pair counts
   for (int t = t0 + warp; t < t1; t += kWarps)
-    topk_token<__nv_bfloat16, __nv_bfloat16>(a.parts, a.nparts, a.part_stride, a.logits, a.bias, E, K, a.renorm,
-                                             a.ids, a.w, a.x, a.w_s, a.H, a.shared_gate, t);
+    topk_token<__nv_bfloat16, __nv_bfloat16>(a.parts, a.nparts, a.part_stride, a.logits, a.bias, a.rc, a.ids, a.w,
+                                             a.x, a.w_s, a.H, a.shared_gate, t);
   __syncthreads();
   for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&s_hist[a.ids[p]], 1);
   __syncthreads();
@@ -190,6 +191,7 @@ cudaError_t launch_prefill_front(const Ctx& c, const PrefillFront& f) {
   a.K = f.K;
   a.renorm = f.renorm;
   a.H = f.H;
+  a.rc = f.rc;
   a.ids = f.ids;
   a.w = f.w;
   a.x = f.x;

@@ -48,12 +48,17 @@ __device__ __forceinline__ void raw_decode(const Raw8<__nv_bfloat16>& r, float (
   }
 }
 
-// Softmax + top-K (+ renormalisation) of one token, by one warp.  `row` holds the
-// E raw logits (global or shared memory); the biased logits go to logits_out.
-__device__ __forceinline__ void warp_topk(const float* row, const float* __restrict__ bias, int E, int K, int renorm,
+// Top-K (+ renormalisation) of one token, by one warp.  `row` holds the E raw
+// logits (global or shared memory); the biased logits go to logits_out.  With
+// n_groups > 1 the experts form n_groups contiguous groups, a group scores its
+// largest logit, and only the topk_groups best groups (lower index on ties)
+// are eligible.  Weights: softmax gate values over all E experts, or sigmoid
+// gate values; renormalised over the K selected when asked.
+__device__ __forceinline__ void warp_topk(const float* row, const float* __restrict__ bias, const RouteCfg& rc,
                                           float* __restrict__ logits_out, int32_t* __restrict__ ids,
                                           float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
+  const int E = rc.E, K = rc.K;
   float v[8];
   float m = -INFINITY;
 #pragma unroll
@@ -71,7 +76,43 @@ __device__ __forceinline__ void warp_topk(const float* row, const float* __restr
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
 
-  uint32_t taken = 0;
+  uint32_t taken = 0;  // bit i: v[i] chosen, or not eligible
+  if (rc.n_groups > 1) {
+    const int gs = E / rc.n_groups;
+    float my_gs = -INFINITY;  // lane g: score of group g
+    for (int g = 0; g < rc.n_groups; ++g) {
+      float gm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && e / gs == g) gm = fmaxf(gm, v[i]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+      if (lane == g) my_gs = gm;
+    }
+    uint32_t kept = 0;
+    for (int j = 0; j < rc.topk_groups; ++j) {
+      float bv = ((kept >> lane) & 1u) || lane >= rc.n_groups ? -INFINITY : my_gs;
+      int bg = ((kept >> lane) & 1u) || lane >= rc.n_groups ? 0x7FFFFFFF : lane;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int og = __shfl_xor_sync(0xffffffffu, bg, o);
+        if (ov > bv || (ov == bv && og < bg)) {
+          bv = ov;
+          bg = og;
+        }
+      }
+      kept |= 1u << bg;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((kept >> (e / gs)) & 1u)) taken |= 1u << i;
+    }
+  }
+
   int my_e = 0;
   float my_v = 0.f;
   for (int k = 0; k < K; ++k) {
@@ -100,18 +141,23 @@ __device__ __forceinline__ void warp_topk(const float* row, const float* __restr
       my_v = bv;
     }
   }
-  const float ev = (lane < K) ? expf(my_v - m) : 0.f;
-  float denom;
-  if (renorm) {
-    denom = warp_sum(ev);
+  float ev, denom;
+  if (rc.gating == MOE_GATING_SIGMOID) {
+    ev = (lane < K) ? 1.0f / (1.0f + expf(-my_v)) : 0.f;
+    denom = rc.renorm ? warp_sum(ev) : 1.0f;
   } else {
-    float s = 0.f;
+    ev = (lane < K) ? expf(my_v - m) : 0.f;
+    if (rc.renorm) {
+      denom = warp_sum(ev);
+    } else {
+      float s = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (lane + 32 * i < E) s += expf(v[i] - m);
-    denom = warp_sum(s);
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) s += expf(v[i] - m);
+      denom = warp_sum(s);
+    }
   }
-  const float inv = denom > 1e-20f ? 1.0f / denom : (renorm ? 1.0f / K : 1.0f);
+  const float inv = denom > 1e-20f ? 1.0f / denom : (rc.renorm ? 1.0f / K : 1.0f);
   if (lane < K) {
     ids[lane] = my_e;
     wout[lane] = ev * inv;
@@ -127,10 +173,11 @@ __device__ __forceinline__ void warp_topk(const float* row, const float* __restr
 // 8l + 256u + q in order; warp_sum).
 template <typename XT, typename WT>
 __device__ __forceinline__ void topk_token(const float* parts, int nparts, size_t part_stride, float* logits,
-                                           const float* bias, int E, int K, int renorm, int32_t* ids, float* wout,
+                                           const float* bias, const RouteCfg& rc, int32_t* ids, float* wout,
                                            const XT* x, const WT* w_s, int H, float* shared_gate, int t) {
   constexpr int kUnroll = 8;
   const int lane = threadIdx.x & 31;
+  const int E = rc.E, K = rc.K;
   float* row = logits + static_cast<size_t>(t) * E;
   if (nparts > 0) {  // all partials of an expert requested together, then added in range order
     constexpr int kMaxParts = 16;
@@ -147,7 +194,7 @@ __device__ __forceinline__ void topk_token(const float* parts, int nparts, size_
     }
     __syncwarp();
   }
-  warp_topk(row, bias, E, K, renorm, row, ids + static_cast<size_t>(t) * K, wout + static_cast<size_t>(t) * K);
+  warp_topk(row, bias, rc, row, ids + static_cast<size_t>(t) * K, wout + static_cast<size_t>(t) * K);
   if (w_s) {
     const XT* xr = x + static_cast<size_t>(t) * H;
     float acc = 0.f;

@@ -79,9 +79,10 @@ static_assert(kStageBytes / (kClusterTok * 4) == kRouterChunk, "router chunking 
 template <typename XT, typename WT>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(256)
     router_cluster_kernel(const XT* __restrict__ x, const WT* __restrict__ W, const WT* __restrict__ w_s,
-                          const float* __restrict__ bias, int T, int H, int E, int K, int renorm,
+                          const float* __restrict__ bias, int T, int H, const RouteCfg rc,
                           float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
                           float* __restrict__ shared_gate) {
+  const int E = rc.E, K = rc.K;
   constexpr int kHc = kStageBytes / (kClusterTok * 4);                // hidden elements per chunk (f32 staging)
   constexpr int kRowsPerCta = (kMaxRows + kCluster - 1) / kCluster;  // 33
   extern __shared__ __align__(16) uint8_t x_stage_raw[];
@@ -136,7 +137,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(256)
   if (rank != 0) return;
   for (int tt = warp; tt < nt; tt += 8) {
     const size_t t = static_cast<size_t>(t0 + tt);
-    warp_topk(s_logits + tt * kMaxRows, bias, E, K, renorm, logits + t * E, ids + t * K, wout + t * K);
+    warp_topk(s_logits + tt * kMaxRows, bias, rc, logits + t * E, ids + t * K, wout + t * K);
     if (w_s && lane == 0) shared_gate[t] = 1.0f / (1.0f + expf(-s_logits[tt * kMaxRows + E]));
   }
 }
@@ -149,8 +150,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(256)
 template <typename XT, typename WT>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ parts, int nparts,
                                                           size_t part_stride, float* __restrict__ logits,
-                                                          const float* __restrict__ bias, int T, int E, int K,
-                                                          int renorm, int32_t* __restrict__ ids,
+                                                          const float* __restrict__ bias, int T,
+                                                          const RouteCfg rc, int32_t* __restrict__ ids,
                                                           float* __restrict__ wout, const XT* __restrict__ x,
                                                           const WT* __restrict__ w_s, int H,
                                                           float* __restrict__ shared_gate) {
@@ -160,12 +161,12 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;
   (void)lane;
-  topk_token(parts, nparts, part_stride, logits, bias, E, K, renorm, ids, wout, x, w_s, H, shared_gate, t);
+  topk_token(parts, nparts, part_stride, logits, bias, rc, ids, wout, x, w_s, H, shared_gate, t);
 }
 
 template <typename XT, typename WT>
 cudaError_t cluster_typed(const Ctx& c, const void* x, const void* W, const void* w_s, const float* bias, int T,
-                          int H, int E, int K, int renorm, float* logits, int32_t* ids, float* w,
+                          int H, const RouteCfg& rc, float* logits, int32_t* ids, float* w,
                           float* shared_gate) {
   const int clusters = (T + kClusterTok - 1) / kClusterTok;
   const cudaError_t e =
@@ -174,51 +175,51 @@ cudaError_t cluster_typed(const Ctx& c, const void* x, const void* W, const void
   KernelScope ks(c, "router_fused");
   return launch_kernel(c, router_cluster_kernel<XT, WT>, dim3(clusters * kCluster), dim3(256), kStageBytes,
                        static_cast<const XT*>(x), static_cast<const WT*>(W), static_cast<const WT*>(w_s), bias, T,
-                       H, E, K, renorm, logits, ids, w, shared_gate);
+                       H, rc, logits, ids, w, shared_gate);
 }
 
 }  // namespace
 
 template <typename XT, typename WT>
 cudaError_t topk_typed(const Ctx& c, const float* parts, int nparts, size_t part_stride, float* logits,
-                       const float* bias, int T, int E, int K, int renorm, int32_t* ids, float* w, const void* x,
+                       const float* bias, int T, const RouteCfg& rc, int32_t* ids, float* w, const void* x,
                        const void* w_s, int H, float* shared_gate) {
   KernelScope ks(c, "router_topk");
   return launch_kernel(c, router_topk_kernel<XT, WT>, dim3((T + 7) / 8), dim3(256), 0, parts, nparts, part_stride,
-                       logits, bias, T, E, K, renorm, ids, w, static_cast<const XT*>(x), static_cast<const WT*>(w_s),
+                       logits, bias, T, rc, ids, w, static_cast<const XT*>(x), static_cast<const WT*>(w_s),
                        H, shared_gate);
 }
 
 cudaError_t launch_router_topk(const Ctx& c, const float* parts, int nparts, size_t part_stride, float* logits,
-                               const float* bias, int T, int E, int K, int renorm, int32_t* ids, float* w,
+                               const float* bias, int T, const RouteCfg& rc, int32_t* ids, float* w,
                                const void* x, int x_dtype, const void* w_s, int w_dtype, int H, float* shared_gate) {
   if (T == 0) return cudaSuccess;
   if (x_dtype == MOE_F32 && w_dtype == MOE_F32)
-    return topk_typed<float, float>(c, parts, nparts, part_stride, logits, bias, T, E, K, renorm, ids, w, x, w_s, H,
+    return topk_typed<float, float>(c, parts, nparts, part_stride, logits, bias, T, rc, ids, w, x, w_s, H,
                                     shared_gate);
   if (x_dtype == MOE_F32 && w_dtype == MOE_BF16)
-    return topk_typed<float, __nv_bfloat16>(c, parts, nparts, part_stride, logits, bias, T, E, K, renorm, ids, w, x,
+    return topk_typed<float, __nv_bfloat16>(c, parts, nparts, part_stride, logits, bias, T, rc, ids, w, x,
                                             w_s, H, shared_gate);
   if (x_dtype == MOE_BF16 && w_dtype == MOE_F32)
-    return topk_typed<__nv_bfloat16, float>(c, parts, nparts, part_stride, logits, bias, T, E, K, renorm, ids, w, x,
+    return topk_typed<__nv_bfloat16, float>(c, parts, nparts, part_stride, logits, bias, T, rc, ids, w, x,
                                             w_s, H, shared_gate);
-  return topk_typed<__nv_bfloat16, __nv_bfloat16>(c, parts, nparts, part_stride, logits, bias, T, E, K, renorm, ids,
+  return topk_typed<__nv_bfloat16, __nv_bfloat16>(c, parts, nparts, part_stride, logits, bias, T, rc, ids,
                                                   w, x, w_s, H, shared_gate);
 }
 
 cudaError_t launch_router_fused(const Ctx& c, const void* x, int x_dtype, const void* W, const void* w_s,
-                                int w_dtype, const float* bias, int T, int H, int E, int K, int renorm,
+                                int w_dtype, const float* bias, int T, int H, const RouteCfg& rc,
                                 float* logits, int32_t* ids, float* w, float* shared_gate) {
   if (T == 0) return cudaSuccess;
   if (x_dtype == MOE_F32 && w_dtype == MOE_F32)
-    return cluster_typed<float, float>(c, x, W, w_s, bias, T, H, E, K, renorm, logits, ids, w, shared_gate);
+    return cluster_typed<float, float>(c, x, W, w_s, bias, T, H, rc, logits, ids, w, shared_gate);
   if (x_dtype == MOE_F32 && w_dtype == MOE_BF16)
-    return cluster_typed<float, __nv_bfloat16>(c, x, W, w_s, bias, T, H, E, K, renorm, logits, ids, w,
+    return cluster_typed<float, __nv_bfloat16>(c, x, W, w_s, bias, T, H, rc, logits, ids, w,
                                                shared_gate);
   if (x_dtype == MOE_BF16 && w_dtype == MOE_F32)
-    return cluster_typed<__nv_bfloat16, float>(c, x, W, w_s, bias, T, H, E, K, renorm, logits, ids, w,
+    return cluster_typed<__nv_bfloat16, float>(c, x, W, w_s, bias, T, H, rc, logits, ids, w,
                                                shared_gate);
-  return cluster_typed<__nv_bfloat16, __nv_bfloat16>(c, x, W, w_s, bias, T, H, E, K, renorm, logits, ids, w,
+  return cluster_typed<__nv_bfloat16, __nv_bfloat16>(c, x, W, w_s, bias, T, H, rc, logits, ids, w,
                                                      shared_gate);
 }
 

@@ -36,7 +36,8 @@ def upload(src):
     desc = Desc(T=s.T, H=s.H, E=s.E, I=s.I, top_k=s.K, act=s.act, renormalize=s.renormalize,
                 act_dtype=s.act_dtype, w_dtype=s.w_dtype, router_dtype=s.router_dtype,
                 has_router_bias=src.router_bias is not None, shared_I=s.shared_I,
-                has_shared_gate=src.sh_gate_w is not None)
+                has_shared_gate=src.sh_gate_w is not None, gating=getattr(s, "gating", "softmax"),
+                n_groups=getattr(s, "n_groups", 1), topk_groups=getattr(s, "topk_groups", 1))
     w = Weights(router=to_device(src.router, s.router_dtype))
     if src.router_bias is not None:
         w.router_bias = torch.from_numpy(np.asarray(src.router_bias, np.float32)).cuda()

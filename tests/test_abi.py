@@ -75,7 +75,9 @@ def test_workspace_bytes_host_only():
 
 @pytest.mark.parametrize("bad", [dict(E=0), dict(E=257), dict(top_k=0), dict(top_k=33, E=64), dict(top_k=5, E=4),
                                  dict(T=-1), dict(H=0), dict(act=7), dict(renormalize=2), dict(act_dtype=2),
-                                 dict(w_dtype=5), dict(T=(1 << 20) + 1)])
+                                 dict(w_dtype=5), dict(T=(1 << 20) + 1), dict(gating=2), dict(n_groups=-1),
+                                 dict(n_groups=33, E=66), dict(n_groups=3), dict(n_groups=2, topk_groups=0),
+                                 dict(n_groups=2, topk_groups=3), dict(n_groups=4, topk_groups=1, top_k=2)])
 def test_invalid_descriptor_rejected_before_cuda(bad):
     import mixture_experts_ffn_07_b200 as moe
     from mixture_experts_ffn_07_b200 import _lib
@@ -85,6 +87,14 @@ def test_invalid_descriptor_rejected_before_cuda(bad):
     w = _lib.MoeWeights()
     rc = _lib.lib().moe_layer(ctypes.byref(d), None, ctypes.byref(w), None, None, 0, None)
     assert rc == moe.MOE_ERR_INVALID_ARG
+
+
+def test_routing_options_accepted():
+    """Valid gating / group settings pass validation (moe_workspace_bytes returns 0 only for invalid descriptors)."""
+    from mixture_experts_ffn_07_b200 import _lib
+    for gating, n_groups, topk_groups, K in ((1, 0, 0, 2), (0, 1, 7, 2), (1, 2, 1, 2), (0, 4, 2, 2), (1, 4, 4, 4)):
+        d = _lib.MoeDesc(8, 64, 4, 64, K, 0, 1, 1, 1, 1, 0, 0, 0, gating, n_groups, topk_groups)
+        assert _lib.lib().moe_workspace_bytes(ctypes.byref(d)) > 0, (gating, n_groups, topk_groups, K)
 
 
 def test_unsupported_sizes_and_bad_pointers():

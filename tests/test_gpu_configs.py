@@ -20,7 +20,7 @@ import workloads  # noqa: E402
 from tests import _gpu  # noqa: E402
 
 SAMPLE = {"decode_f32_t1": 1, "prefill_bf16_t512": 48, "routed_shared_t4096": 24, "skewed_zipf_t8192": 8,
-          "q8_0_decode_t16": 16}
+          "q8_0_decode_t16": 16, "grouped_sigmoid_t512": 32}
 
 
 @pytest.mark.parametrize("name", workloads.CONFIG_ORDER)
@@ -34,7 +34,8 @@ def test_full_size_config(name):
 
     # routing on every token: bit-exact against the oracle's selection of the GPU's logits
     gl = logits.cpu().numpy().astype(np.float64)
-    ref_ids, ref_w = oracle.select(gl, spec.K, spec.renormalize)
+    ref_ids, ref_w = oracle.select(gl, spec.K, spec.renormalize, gating=spec.gating, n_groups=spec.n_groups,
+                                   topk_groups=spec.topk_groups)
     gids = ids.cpu().numpy()
     assert np.array_equal(gids, ref_ids)
     assert np.max(np.abs(tw.cpu().numpy() - ref_w)) < 2e-6
