@@ -79,10 +79,15 @@ def bind(lib):
     lib.ora_shared.argtypes = [p, p, p, i64, p, p]
     lib.ora_load_rows.argtypes = [p, i32, i64, i64, i64, p]
     lib.ora_act_array.argtypes = [i32, p, i64, p]
+    lib.ora_act_grad.argtypes = [i32, ctypes.c_double]
+    lib.ora_act_grad.restype = ctypes.c_double
+    lib.ora_combine_backward.argtypes = [p, p, p, i64, i64, i64, p, p]
+    lib.ora_act_up_backward.argtypes = [i32, p, p, i64, i64, p]
     lib.ora_threads.restype = i32
     lib.ora_set_threads.argtypes = [i32]
     for f in (lib.ora_select, lib.ora_weights_for, lib.ora_expert, lib.ora_layer, lib.ora_logits,
-              lib.ora_shared, lib.ora_load_rows, lib.ora_act_array, lib.ora_set_threads):
+              lib.ora_shared, lib.ora_load_rows, lib.ora_act_array, lib.ora_set_threads, lib.ora_combine_backward,
+              lib.ora_act_up_backward):
         f.restype = None
     return lib
 
@@ -258,6 +263,37 @@ def act(name: str, g) -> np.ndarray:
     g = np.ascontiguousarray(np.atleast_1d(g), np.float64)
     out = np.zeros_like(g)
     _lib().ora_act_array(ACT[name], g.ctypes.data, g.size, out.ctypes.data)
+    return out
+
+
+def act_grad(name: str, g: float) -> float:
+    """Derivative of the activation at g (backward of act * up)."""
+    return _lib().ora_act_grad(ACT[name], g)
+
+
+def combine_backward(y: np.ndarray, w: np.ndarray, d_out: np.ndarray):
+    """Backward of out[t] = sum_k w[t,k] y[t,k]: y[T,K,H], w[T,K], d_out[T,H] (f32) -> d_y[T,K,H], d_w[T,K] (f64)."""
+    y = np.ascontiguousarray(y, np.float32)
+    w = np.ascontiguousarray(w, np.float32)
+    d_out = np.ascontiguousarray(d_out, np.float32)
+    T, K, H = y.shape
+    assert w.shape == (T, K) and d_out.shape == (T, H)
+    d_y = np.zeros((T, K, H), np.float64)
+    d_w = np.zeros((T, K), np.float64)
+    _lib().ora_combine_backward(y.ctypes.data, w.ctypes.data, d_out.ctypes.data, T, K, H, d_y.ctypes.data,
+                                d_w.ctypes.data)
+    return d_y, d_w
+
+
+def act_up_backward(act_name: str, gate_up: np.ndarray, d_h: np.ndarray) -> np.ndarray:
+    """Backward of h = act(gate) * up: gate_up[P, 2I] ([gate | up]), d_h[P, I] (f32) -> d_gate_up[P, 2I] (f64)."""
+    gu = np.ascontiguousarray(gate_up, np.float32)
+    dh = np.ascontiguousarray(d_h, np.float32)
+    P, I2 = gu.shape
+    I = I2 // 2
+    assert I2 == 2 * I and dh.shape == (P, I)
+    out = np.zeros((P, 2 * I), np.float64)
+    _lib().ora_act_up_backward(ACT[act_name], gu.ctypes.data, dh.ctypes.data, P, I, out.ctypes.data)
     return out
 
 

@@ -41,6 +41,16 @@
  *               out[t] += s * W_sdown (act(W_sgate x) * (W_sup x))
  *               (hf2q qwen35/gpu_ffn.rs, build_moe_ffn_layer_gpu, shared expert)
  *
+ * Backward of two steps (mlx-native moe_dispatch.rs, the backward kernels of
+ * moe_weighted_sum_seq and moe_swiglu_seq), for a loss L with dL/dout given:
+ *   combine     out[t,d] = sum_k y[t,k,d] w[t,k]:
+ *               d_y[t,k,d] = w[t,k] d_out[t,d];  d_w[t,k] = sum_d y[t,k,d] d_out[t,d]
+ *   act * up    h[p,i] = act(g[p,i]) u[p,i], gate_up rows [g | u] of 2I:
+ *               d_g = d_h u act'(g);  d_u = d_h act(g)
+ *               act'(g) for SiLU: s (1 + g (1 - s)), s = 1/(1+e^-g);
+ *               for the tanh GELU with z = c (g + a g^3), c = sqrt(2/pi),
+ *               a = 0.044715: 0.5 (1 + tanh z) + 0.5 g (1 - tanh^2 z) c (1 + 3 a g^2)
+ *
  * Storage formats read (converted exactly to f64): f32; bf16 (upper half of an
  * f32); Q8_0 GGML blocks {fp16 d; int8 q[32]} along the input dimension, value
  * = fp16(d) * q.
@@ -455,6 +465,49 @@ void ora_shared(const ora_desc* d, const ora_tensors* w, const int64_t* tokens, 
     free(xt);
     free(row);
     free(a);
+  }
+}
+
+/* Derivative of the activation (step "act * up" of the backward, header). */
+double ora_act_grad(int act, double g) {
+  if (act == ORA_SILU) {
+    const double s = 1.0 / (1.0 + exp(-g));
+    return s * (1.0 + g * (1.0 - s));
+  }
+  const double c = sqrt(2.0 / M_PI), a = 0.044715;
+  const double th = tanh(c * (g + a * g * g * g));
+  return 0.5 * (1.0 + th) + 0.5 * g * (1.0 - th * th) * c * (1.0 + 3.0 * a * g * g);
+}
+
+/* Backward of the combine: y[T,K,H], w[T,K], d_out[T,H] (f32, as stored) ->
+ * d_y[T,K,H], d_w[T,K] in f64. */
+void ora_combine_backward(const float* y, const float* w, const float* d_out, int64_t T, int64_t K, int64_t H,
+                          double* d_y, double* d_w) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t k = 0; k < K; ++k) {
+      const int64_t p = t * K + k;
+      double s = 0.0;
+      for (int64_t d = 0; d < H; ++d) {
+        d_y[p * H + d] = (double)w[p] * (double)d_out[t * H + d];
+        s += (double)y[p * H + d] * (double)d_out[t * H + d];
+      }
+      d_w[p] = s;
+    }
+  }
+}
+
+/* Backward of act(gate) * up: gate_up[P, 2I] (gate in columns [0, I), up in
+ * [I, 2I)), d_h[P, I] (f32) -> d_gate_up[P, 2I] in f64, same layout. */
+void ora_act_up_backward(int act, const float* gate_up, const float* d_h, int64_t P, int64_t I,
+                         double* d_gate_up) {
+#pragma omp parallel for schedule(static)
+  for (int64_t p = 0; p < P; ++p) {
+    for (int64_t i = 0; i < I; ++i) {
+      const double g = gate_up[p * 2 * I + i], u = gate_up[p * 2 * I + I + i], dh = d_h[p * I + i];
+      d_gate_up[p * 2 * I + i] = dh * u * ora_act_grad(act, g);
+      d_gate_up[p * 2 * I + I + i] = dh * ora_act(act, g);
+    }
   }
 }
 

@@ -35,6 +35,15 @@ MUTANTS = {
     "groups_kept_off_by_one": ("for (int64_t i = 0; i < r->topk_groups; ++i) keep[gkeys[i].e] = 1;",
                                "for (int64_t i = 0; i <= r->topk_groups && i < r->n_groups; ++i) keep[gkeys[i].e] = 1;"),
     "groups_ignored": ("if (r->n_groups > 1) {", "if (0) {"),
+    "gelu_grad_tanh_term_dropped": (" + 0.5 * g * (1.0 - th * th) * c * (1.0 + 3.0 * a * g * g);", ";"),
+    "silu_grad_sign": ("return s * (1.0 + g * (1.0 - s));", "return s * (1.0 - g * (1.0 - s));"),
+    "d_up_uses_gate": ("d_gate_up[p * 2 * I + I + i] = dh * ora_act(act, g);", "d_gate_up[p * 2 * I + I + i] = dh * g;"),
+    "d_gate_drops_up": ("d_gate_up[p * 2 * I + i] = dh * u * ora_act_grad(act, g);",
+                        "d_gate_up[p * 2 * I + i] = dh * ora_act_grad(act, g);"),
+    "d_w_slots_transposed": ("s += (double)y[p * H + d] * (double)d_out[t * H + d];",
+                             "s += (double)y[(k * T + t) * H + d] * (double)d_out[t * H + d];"),
+    "d_y_first_slot_weight": ("d_y[p * H + d] = (double)w[p] * (double)d_out[t * H + d];",
+                              "d_y[p * H + d] = (double)w[t * K] * (double)d_out[t * H + d];"),
 }
 
 BATTERY = [
@@ -49,6 +58,11 @@ BATTERY = [
     lambda g: pins.test_sigmoid_gating_known_values(), lambda g: pins.test_sigmoid_gating_equals_two_way_softmax(),
     lambda g: pins.test_sigmoid_gating_selects_like_softmax(), lambda g: pins.test_grouped_worked_example(),
     lambda g: pins.test_grouped_special_cases_and_brute_force(),
+    lambda g: pins.test_backward_canonical_values("gelu_tanh", g), lambda g: pins.test_backward_canonical_values("silu", g),
+    lambda g: pins.test_act_grad_matches_finite_difference("gelu_tanh"),
+    lambda g: pins.test_act_grad_matches_finite_difference("silu"),
+    lambda g: pins.test_act_up_backward_finite_difference("gelu_tanh"),
+    lambda g: pins.test_combine_backward_finite_difference(), lambda g: pins.test_combine_backward_special_cases(),
 ]
 
 

@@ -376,3 +376,97 @@ def test_grouped_special_cases_and_brute_force():
             for t in range(rows.shape[0]):
                 assert ids[t].tolist() == _grouped_brute(rows[t], K, n_groups, topk_groups)
             assert np.all(np.abs(w.sum(axis=1) - 1.0) < 1e-12)
+
+
+# ---------------------------------------------------------------- backward (act * up, combine)
+# Inputs of the finite-difference falsifiers on the page (mlx-native
+# moe_dispatch.rs, backward_*_finite_difference_falsifier tests).
+
+def _page_seq(n, a, b, c, fn):
+    i = np.arange(n, dtype=np.float32)
+    return (np.float32(a) + i * np.float32(b) - fn(i * np.float32(c))).astype(np.float32)
+
+
+def _act_up_forward(act, gu, I):
+    g, u = gu[:, :I].astype(np.float64), gu[:, I:].astype(np.float64)
+    return oracle.act(act, g.reshape(-1)).reshape(g.shape) * u
+
+
+@pytest.mark.parametrize("act", ["gelu_tanh", "silu"])
+def test_backward_canonical_values(act, golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "backward_canonical.json")))
+    gu = np.array([g["gate_up"]], np.float32)
+    d = oracle.act_up_backward(act, gu, np.array([g["d_h"]], np.float32))[0]
+    for v, e, tol in zip(d, g["expected_d_gate_up"], g["tol"]):
+        assert abs(v - e) <= tol, (act, v, e)
+
+
+@pytest.mark.parametrize("act", ["gelu_tanh", "silu"])
+def test_act_grad_matches_finite_difference(act):
+    h = 1e-5
+    for g in np.linspace(-9, 9, 721):
+        fd = (oracle.act(act, g + h)[0] - oracle.act(act, g - h)[0]) / (2 * h)
+        assert abs(oracle.act_grad(act, g) - fd) < 1e-8, (act, g)
+
+
+@pytest.mark.parametrize("act", ["gelu_tanh", "silu"])
+def test_act_up_backward_finite_difference(act):
+    T, K, I = 2, 3, 5
+    P = T * K
+    gu = _page_seq(P * 2 * I, 0.5, 0.07, 0.013, np.sin).reshape(P, 2 * I)
+    seed = _page_seq(P * I, 0.3, 0.05, 0.011, np.cos).reshape(P, I)
+    d = oracle.act_up_backward(act, gu, seed)
+    base = gu.astype(np.float64)
+    h = 1e-4
+    for idx in range(base.size):
+        r, c = divmod(idx, 2 * I)
+        gp, gm = base.copy(), base.copy()
+        gp[r, c] += h
+        gm[r, c] -= h
+        fd = (np.sum(_act_up_forward(act, gp, I) * seed) - np.sum(_act_up_forward(act, gm, I) * seed)) / (2 * h)
+        assert abs(d[r, c] - fd) < 1e-7 * max(1.0, abs(fd)), (act, idx)
+
+
+def test_combine_backward_finite_difference():
+    T, K, H = 3, 4, 7
+    y = _page_seq(T * K * H, 0.1, 0.013, 0.004, np.sin).reshape(T, K, H)
+    w = (np.float32(0.2) + np.arange(T * K, dtype=np.float32) * np.float32(0.07)).reshape(T, K)
+    seed = _page_seq(T * H, 0.3, 0.05, 0.011, np.cos).reshape(T, H)
+    d_y, d_w = oracle.combine_backward(y, w, seed)
+
+    def loss(yy, ww):
+        out = np.einsum("tkd,tk->td", yy, ww)
+        return np.sum(out * seed)
+
+    Y, W = y.astype(np.float64), w.astype(np.float64)
+    h = 1e-3
+    for idx in np.ndindex(T, K, H):
+        yp, ym = Y.copy(), Y.copy()
+        yp[idx] += h
+        ym[idx] -= h
+        fd = (loss(yp, W) - loss(ym, W)) / (2 * h)
+        assert abs(d_y[idx] - fd) < 1e-9 * max(1.0, abs(fd)), idx
+    for idx in np.ndindex(T, K):
+        wp, wm = W.copy(), W.copy()
+        wp[idx] += h
+        wm[idx] -= h
+        fd = (loss(Y, wp) - loss(Y, wm)) / (2 * h)
+        assert abs(d_w[idx] - fd) < 1e-9 * max(1.0, abs(fd)), idx
+
+
+def test_combine_backward_special_cases():
+    rng = np.random.default_rng(5)
+    T, K, H = 4, 3, 6
+    y = rng.standard_normal((T, K, H)).astype(np.float32)
+    w = rng.random((T, K)).astype(np.float32)
+    d_y, d_w = oracle.combine_backward(y, w, np.zeros((T, H), np.float32))
+    assert not d_y.any() and not d_w.any()
+    # one-hot d_out picks out single elements: d_w[t,k] = y[t,k,j], d_y[t,k,:] = w[t,k] e_j
+    for t, j in [(0, 0), (2, 5), (3, 2)]:
+        dout = np.zeros((T, H), np.float32)
+        dout[t, j] = 1.0
+        d_y, d_w = oracle.combine_backward(y, w, dout)
+        for k in range(K):
+            assert d_w[t, k] == y[t, k, j]
+            assert d_y[t, k, j] == w[t, k] and np.count_nonzero(d_y[t, k]) == (w[t, k] != 0)
+        assert not np.delete(d_w, t, axis=0).any()
