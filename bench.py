@@ -11,6 +11,9 @@ the max over ranks and `value` counts the tokens of all ranks.
 
 --impl reference times the f64 CPU oracle on the host cores instead (rank 0
 only), on bounded token samples of the same workload.
+
+--op backward times the backward of the combine and of act*up (one launch of
+each per step, f32) on the workload's T, K, H, I instead of the forward layer.
 """
 from __future__ import annotations
 
@@ -371,6 +374,166 @@ def run_ours(args, spec):
     return 0
 
 
+# ------------------------------------------------------------------ backward of combine and act * up
+BWD_METRIC = "MoE backward (combine + act*up) tokens/s at 1 B200; % of HBM BW"
+
+
+def backward_bytes(T, K, H, I):
+    """Algorithmic bytes of one launch of each backward kernel: every input read once, every output written once."""
+    P = T * K
+    return {"combine_backward": 4 * (T * H + 2 * P * H + 2 * P), "act_up_backward": 4 * P * I * 5}
+
+
+def _backward_host_inputs(spec, seed=11):
+    T, K, H, I = spec.T, spec.K, spec.H, spec.I
+    P = T * K
+    rng = np.random.default_rng(seed)
+    return {"y": rng.standard_normal((T, K, H), np.float32), "w": rng.random((T, K), np.float32),
+            "d_out": rng.standard_normal((T, H), np.float32),
+            "gate_up": (3 * rng.standard_normal((P, 2 * I))).astype(np.float32),
+            "d_h": rng.standard_normal((P, I), np.float32)}
+
+
+def _time_oracle_backward(spec, hin, budget_s):
+    import oracle
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.combine_backward(hin["y"], hin["w"], hin["d_out"])
+        oracle.act_up_backward(spec.act, hin["gate_up"], hin["d_h"])
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or reps >= 1000:
+            break
+    return spec.T * reps / dt, dict(cores=oracle.threads(), sample=f"all {spec.T} tokens x {reps} passes, f64")
+
+
+def run_backward(args, spec):
+    """--op backward: one step = moe_combine_backward + moe_act_up_backward over one batch of the workload's slots."""
+    T, K, H, I = spec.T, spec.K, spec.H, spec.I
+    P = T * K
+    ws_n, rank, local = _dist()
+    hin = _backward_host_inputs(spec)
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        v, info = _time_oracle_backward(spec, hin, budget_s=min(args.cpu_budget, 5.0))
+        print(json.dumps({"impl": "reference", "metric": BWD_METRIC, "value": v, "unit": UNIT, "n_gpus": ws_n,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * T / v,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": {"workload": spec.name + "/backward", "T": T, "K": K,
+                                                          "H": H, "I": I, "act": spec.act},
+                          "cpu_baseline": {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                                           "sample": info["sample"]},
+                          "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return 0
+    import torch
+    torch.cuda.set_device(local)
+    import mixture_experts_ffn_07_b200 as moe
+    dev = {k: torch.from_numpy(v).cuda() for k, v in hin.items()}
+    alg = backward_bytes(T, K, H, I)
+    set_bytes = sum(alg.values())
+    nsets = max(1, min(8, -(-400_000_000 // set_bytes)))  # rotate buffer sets: > 3x L2 between reuses
+    sets = []
+    for i in range(nsets):
+        d = dev if i == 0 else {k: v.clone() for k, v in dev.items()}
+        d = dict(d, d_y=torch.empty((T, K, H), device="cuda"), d_w=torch.empty((T, K), device="cuda"),
+                 d_gu=torch.empty((P, 2 * I), device="cuda"))
+        sets.append(d)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        b = sets[i % nsets]
+        moe.combine_backward(b["y"], b["w"], b["d_out"], b["d_y"], b["d_w"])
+        moe.act_up_backward(spec.act, b["gate_up"], b["d_h"], b["d_gu"])
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    clocks.start()
+    n0 = moe.launch_count()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    n_launch = moe.launch_count() - n0
+    clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    # per-kernel durations: each kernel alone, back to back over the rotating sets, between one event pair
+    # (an event pair around every launch would add the launch gap to these ~10 us kernels)
+    one = {"combine_backward": lambda b: moe.combine_backward(b["y"], b["w"], b["d_out"], b["d_y"], b["d_w"]),
+           "act_up_backward": lambda b: moe.act_up_backward(spec.act, b["gate_up"], b["d_h"], b["d_gu"])}
+    kernels = {}
+    for name, fn in one.items():
+        for i in range(3):
+            fn(sets[i % nsets])
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        for i in range(args.steps):
+            fn(sets[i % nsets])
+        k1.record(stream)
+        torch.cuda.synchronize()
+        t = k0.elapsed_time(k1)
+        kernels[name] = {"launches": args.steps, "avg_ms": t / args.steps, "total_ms": t}
+    tot = sum(k["total_ms"] for k in kernels.values()) or 1.0
+    dom = max(kernels, key=lambda n: kernels[n]["total_ms"])
+    peaks, peak_src = _peaks()
+    ach = {n: alg[n] / (kernels[n]["avg_ms"] / 1e3) / 1e9 for n in kernels}
+    roofline = {"bound": "hbm", "achieved": ach[dom], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach[dom] / peaks["hbm_gbs"], "traffic": _traffic(dom, spec.name + "/backward"), "kernel": dom,
+                "algorithmic_bytes_per_launch": alg[dom], "peak_source": f"{peak_src} (hbm_gbs)",
+                "per_kernel_frac": {n: ach[n] / peaks["hbm_gbs"] for n in kernels}}
+    # end to end: inputs from pinned host memory, both kernels, outputs back, every step
+    pin = {k: torch.from_numpy(v).pin_memory() for k, v in hin.items()}
+    outs = {"d_y": torch.empty((T, K, H)).pin_memory(), "d_w": torch.empty((T, K)).pin_memory(),
+            "d_gu": torch.empty((P, 2 * I)).pin_memory()}
+    b = sets[0]
+
+    def e2e_step():
+        for k in hin:
+            b[k].copy_(pin[k], non_blocking=True)
+        moe.combine_backward(b["y"], b["w"], b["d_out"], b["d_y"], b["d_w"])
+        moe.act_up_backward(spec.act, b["gate_up"], b["d_h"], b["d_gu"])
+        for k in outs:
+            outs[k].copy_(b[k], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(1, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    cpu = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        v, info = _time_oracle_backward(spec, hin, budget_s=min(args.cpu_budget, 5.0))
+        cpu = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle", "sample": info["sample"]}
+    line = {"metric": BWD_METRIC, "value": job_throughput(1, T, args.steps, ms), "unit": UNIT, "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": spec.name + "/backward", "T": T, "K": K, "H": H, "I": I, "act": spec.act,
+                       "l2": f"no flush: {nsets} rotating input sets of {set_bytes / 1e6:.0f} MB"},
+            "e2e": {"value": job_throughput(1, T, e_steps, e2e_ms), "unit": UNIT,
+                    "h2d_bytes_per_step": int(sum(v.nbytes for v in hin.values())),
+                    "d2h_bytes_per_step": int(4 * (P * H + P + 2 * P * I))},
+            "roofline": roofline, "cpu_baseline": cpu, "gpu_launches": n_launch, "clocks": clocks.summary(),
+            "device_status": moe.status_string(moe.last_device_status()),
+            "kernels": {n: {"launches": k["launches"], "avg_us": 1e3 * k["avg_ms"],
+                            "share": round(k["total_ms"] / tot, 4), "timing": "alone, back to back"}
+                        for n, k in kernels.items()}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -380,8 +543,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="layer", choices=["layer", "backward"],
+                    help="backward: the combine and act*up backward kernels on the workload's slots")
     args = ap.parse_args()
     spec = workloads.CONFIGS[args.config]
+    if args.op == "backward":
+        return run_backward(args, spec)
     if args.impl == "reference":
         return run_reference(args, spec)
     return run_ours(args, spec)

@@ -254,6 +254,42 @@ moe_status moe_q8_0_split(const void* blocks, int64_t rows, int64_t cols, int8_t
                           moe_stream_t stream);
 
 /*
+ * Backward of the routing-weighted combine out[t,:] = sum_k w[t,k] y[t,k,:],
+ * for a loss L with d_out = dL/dout given (mlx-native moe_dispatch.rs, the
+ * backward kernels of moe_weighted_sum_seq):
+ *   d_y[t,k,:] = w[t,k] d_out[t,:]          d_w[t,k] = sum_h y[t,k,h] d_out[t,h]
+ *  y     [T,K,H] f32 device: the expert outputs BEFORE weighting (row t*K+k);
+ *        moe_expert_ffn's y_slots are already weighted by topk_w
+ *  w     [T,K]   f32 device: the routing weights
+ *  d_out [T,H]   f32 device
+ *  d_y   [T,K,H] f32 device out;  d_w [T,K] f32 device out
+ * d_w is summed in a fixed order (the same bits on every run).  T == 0 does
+ * nothing.  MOE_ERR_INVALID_ARG: T < 0, K < 1, H < 1, T or K > 2^31-1,
+ * T*K > 2^33-1, a null pointer, or an output range that overlaps an input range.  Caller-owned
+ * memory; asynchronous on `stream`.
+ */
+moe_status moe_combine_backward(int64_t T, int64_t K, int64_t H, const float* y, const float* w, const float* d_out,
+                                float* d_y, float* d_w, moe_stream_t stream);
+
+/*
+ * Backward of h = act(gate) * up (mlx-native moe_dispatch.rs, the backward
+ * kernel of moe_swiglu_seq, which writes both gradients into one buffer laid
+ * out like its input):
+ *   d_gate = d_h * up * act'(gate)          d_up = d_h * act(gate)
+ *   act'(g) = s (1 + g (1 - s)), s = 1/(1+e^-g), for MOE_ACT_SILU;
+ *   0.5 (1 + tanh z) + 0.5 g (1 - tanh^2 z) sqrt(2/pi) (1 + 3 * 0.044715 g^2),
+ *   z = sqrt(2/pi) (g + 0.044715 g^3), for MOE_ACT_GELU_TANH
+ *  gate_up   [P, 2I] f32 device: row p = [gate (I values) | up (I values)]
+ *  d_h       [P, I]  f32 device
+ *  d_gate_up [P, 2I] f32 device out: row p = [d_gate | d_up]
+ * P == 0 does nothing.  MOE_ERR_INVALID_ARG: P < 0, I < 1, an unknown act, a
+ * null pointer, or an output range that overlaps an input range.
+ * Caller-owned memory; asynchronous on `stream`.
+ */
+moe_status moe_act_up_backward(int64_t P, int64_t I, int32_t act, const float* gate_up, const float* d_h,
+                               float* d_gate_up, moe_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device (MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_INDEX), or
  * MOE_ERR_CUDA if the synchronisation failed.

@@ -158,6 +158,20 @@ def q8_0_split(blocks, rows, cols, q, scales, stream=None):
           "moe_q8_0_split")
 
 
+def combine_backward(y, w, d_out, d_y, d_w, stream=None):
+    """moe_combine_backward: y [T,K,H] (unweighted expert outputs), w [T,K], d_out [T,H] -> d_y, d_w (all f32)."""
+    T, K, H = y.shape
+    check(_lib.lib().moe_combine_backward(T, K, H, _ptr(y), _ptr(w), _ptr(d_out), _ptr(d_y), _ptr(d_w),
+                                          _stream(stream)), "moe_combine_backward")
+
+
+def act_up_backward(act, gate_up, d_h, d_gate_up, stream=None):
+    """moe_act_up_backward: gate_up [P,2I] ([gate | up]), d_h [P,I] -> d_gate_up [P,2I] (all f32)."""
+    P, I = d_h.shape
+    check(_lib.lib().moe_act_up_backward(P, I, ACTS[act] if isinstance(act, str) else act, _ptr(gate_up), _ptr(d_h),
+                                         _ptr(d_gate_up), _stream(stream)), "moe_act_up_backward")
+
+
 def last_device_status(stream=None) -> int:
     return _lib.lib().moe_last_device_status(_stream(stream))
 

@@ -23,7 +23,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route
            "moe_combine", "moe_layer", "moe_layer_host", "moe_layer_noalloc", "moe_q8_0_split",
            "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
            "moe_debug_set_wait_limit", "moe_debug_set_skip_stage", "moe_set_fused_decode",
-           "moe_workspace_regions", "moe_set_fused_front")
+           "moe_workspace_regions", "moe_set_fused_front", "moe_combine_backward", "moe_act_up_backward")
 
 
 class MoeDesc(ctypes.Structure):
@@ -74,8 +74,11 @@ def lib():
         L.moe_layer_noalloc.argtypes = [DP, P, WP, P, P]
         L.moe_q8_0_split.argtypes = [P, I64, I64, P, P, P]
         L.moe_last_device_status.argtypes = [P]
+        L.moe_combine_backward.argtypes = [I64, I64, I64, P, P, P, P, P, P]
+        L.moe_act_up_backward.argtypes = [I64, I64, I32, P, P, P, P]
         for f in (L.moe_route, L.moe_permute, L.moe_expert_ffn, L.moe_combine, L.moe_layer, L.moe_layer_host,
-                  L.moe_layer_noalloc, L.moe_q8_0_split, L.moe_last_device_status):
+                  L.moe_layer_noalloc, L.moe_q8_0_split, L.moe_last_device_status, L.moe_combine_backward,
+                  L.moe_act_up_backward):
             f.restype = I32
         L.moe_launch_count.restype = ctypes.c_uint64
         L.moe_trace_enable.argtypes = [I32]

@@ -17,7 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OUT_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["moe_api.cu", "router.cu", "permute.cu", "grouped_gemm.cu", "stream_gemv.cu", "stream_ffn.cu", "decode_fused.cu", "prefill_front.cu"]
+SOURCES = ["moe_api.cu", "router.cu", "permute.cu", "grouped_gemm.cu", "stream_gemv.cu", "stream_ffn.cu", "decode_fused.cu", "prefill_front.cu",
+           "backward.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
          "-cudart", "static", f"-I{os.path.join(ROOT, 'include')}"]

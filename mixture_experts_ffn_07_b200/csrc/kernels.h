@@ -94,6 +94,11 @@ cudaError_t launch_combine(const Ctx& c, const float* y_slots, const float* y_sh
                            void* out, int out_dtype);
 
 // GGML Q8_0 blocks -> int8 plane + fp16 scale plane.
+// Backward of the combine and of act(gate) * up (backward.cu).
+cudaError_t launch_combine_backward(const Ctx& c, const float* y, const float* w, const float* d_out, long long T,
+                                    int K, long long H, float* d_y, float* d_w);
+cudaError_t launch_act_up_backward(const Ctx& c, const float* gate_up, const float* d_h, long long P, long long I,
+                                   int act, float* d_gate_up);
 cudaError_t launch_q8_0_split(const Ctx& c, const void* blocks, int64_t rows, int64_t cols, int8_t* q,
                               void* scales);
 

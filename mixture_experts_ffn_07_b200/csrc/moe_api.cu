@@ -658,6 +658,44 @@ moe_status moe_q8_0_split(const void* blocks, int64_t rows, int64_t cols, int8_t
   return from_cuda(moe::launch_q8_0_split(c, blocks, rows, cols, q, scales));
 }
 
+namespace {
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+}  // namespace
+
+moe_status moe_combine_backward(int64_t T, int64_t K, int64_t H, const float* y, const float* w, const float* d_out,
+                                float* d_y, float* d_w, moe_stream_t stream) {
+  if (T < 0 || K < 1 || H < 1 || T > 0x7fffffffLL || K > 0x7fffffffLL || T * K > 0x1ffffffffLL)
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!y || !w || !d_out || !d_y || !d_w) return MOE_ERR_INVALID_ARG;
+  const size_t ny = static_cast<size_t>(T) * K * H * 4, nw = static_cast<size_t>(T) * K * 4,
+               nd = static_cast<size_t>(T) * H * 4;
+  for (const void* out : {static_cast<const void*>(d_y), static_cast<const void*>(d_w)}) {
+    const size_t no = out == d_y ? ny : nw;
+    if (overlaps(out, no, y, ny) || overlaps(out, no, w, nw) || overlaps(out, no, d_out, nd))
+      return MOE_ERR_INVALID_ARG;
+  }
+  if (overlaps(d_y, ny, d_w, nw)) return MOE_ERR_INVALID_ARG;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return from_cuda(moe::launch_combine_backward(c, y, w, d_out, T, static_cast<int>(K), H, d_y, d_w));
+}
+
+moe_status moe_act_up_backward(int64_t P, int64_t I, int32_t act, const float* gate_up, const float* d_h,
+                               float* d_gate_up, moe_stream_t stream) {
+  if (P < 0 || I < 1 || (act != MOE_ACT_SILU && act != MOE_ACT_GELU_TANH)) return MOE_ERR_INVALID_ARG;
+  if (P == 0) return MOE_OK;
+  if (!gate_up || !d_h || !d_gate_up) return MOE_ERR_INVALID_ARG;
+  const size_t ng = static_cast<size_t>(P) * 2 * I * 4, nh = static_cast<size_t>(P) * I * 4;
+  if (overlaps(d_gate_up, ng, gate_up, ng) || overlaps(d_gate_up, ng, d_h, nh)) return MOE_ERR_INVALID_ARG;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return from_cuda(moe::launch_act_up_backward(c, gate_up, d_h, P, I, act, d_gate_up));
+}
+
 moe_status moe_last_device_status(moe_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
   int v = 0;

@@ -176,3 +176,27 @@ def test_workspace_regions_host_only():
             assert r[k] % 256 == 0 and r[k] + sizes[k] <= n
     with pytest.raises(moe.MoeError):
         moe.workspace_regions(moe.Desc(T=1, H=33, E=4, I=32, top_k=1))
+
+
+def test_backward_argument_checks_host_only(L):
+    """Invalid sizes, null pointers and overlapping outputs are rejected before any CUDA call."""
+    from mixture_experts_ffn_07_b200 import _lib as moe
+    inv = moe.MOE_ERR_INVALID_ARG
+    a, b, c, d, e = 1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20  # disjoint fake addresses, never dereferenced
+    assert L.moe_combine_backward(-1, 8, 16, a, b, c, d, e, None) == inv
+    assert L.moe_combine_backward(4, 0, 16, a, b, c, d, e, None) == inv
+    assert L.moe_combine_backward(4, 8, 0, a, b, c, d, e, None) == inv
+    assert L.moe_combine_backward(1 << 31, 1, 1, a, b, c, d, e, None) == inv
+    assert L.moe_combine_backward(1 << 20, 1 << 14, 1, a, b, c, d, e, None) == inv  # T*K beyond the grid
+    assert L.moe_combine_backward(4, 8, 16, None, b, c, d, e, None) == inv
+    assert L.moe_combine_backward(4, 8, 16, a, b, c, a, e, None) == inv  # d_y over y
+    assert L.moe_combine_backward(4, 8, 16, a, b, c, d, c + 4, None) == inv  # d_w inside d_out
+    assert L.moe_combine_backward(4, 8, 16, a, b, c, d, d + 64, None) == inv  # d_w inside d_y
+    assert L.moe_combine_backward(0, 8, 16, None, None, None, None, None, None) == moe.MOE_OK
+    assert L.moe_act_up_backward(-1, 16, 0, a, b, c, None) == inv
+    assert L.moe_act_up_backward(4, 0, 0, a, b, c, None) == inv
+    assert L.moe_act_up_backward(4, 16, 7, a, b, c, None) == inv
+    assert L.moe_act_up_backward(4, 16, 0, a, None, c, None) == inv
+    assert L.moe_act_up_backward(4, 16, 0, a, b, a + 8, None) == inv  # d_gate_up over gate_up
+    assert L.moe_act_up_backward(4, 16, 1, a, b, b, None) == inv  # d_gate_up over d_h
+    assert L.moe_act_up_backward(0, 16, 0, None, None, None, None) == moe.MOE_OK
