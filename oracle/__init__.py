@@ -22,7 +22,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SO = os.path.join(_HERE, "liboracle.so")
 _SRC = os.path.join(_HERE, "oracle.c")
 
-DTYPE = {"f32": 0, "bf16": 1, "q8_0": 2}
+DTYPE = {"f32": 0, "bf16": 1, "q8_0": 2, "q4_k": 3, "q4_k_q6_k": 4, "q6_k": 5}
+# bytes of one stored block and the values it holds, for the block formats
+BLOCK = {"q8_0": (34, 32), "q4_k": (144, 256), "q6_k": (210, 256)}
 ACT = {"silu": 0, "gelu_tanh": 1}
 
 
@@ -250,10 +252,14 @@ def shared(L: Layer, tokens=None):
 
 
 def load_rows(a: np.ndarray, dtype: str, cols: int, r0: int = 0, n: int | None = None) -> np.ndarray:
-    """Rows of a stored matrix widened to f64 (dequantising Q8_0 blocks)."""
+    """Rows of a stored matrix widened to f64 (dequantising Q8_0, Q4_K or Q6_K blocks)."""
     a = np.ascontiguousarray(a)
     if n is None:
-        n = (a.nbytes // (cols // 32 * 34)) if dtype == "q8_0" else a.size // cols
+        if dtype in BLOCK:
+            nb, nv = BLOCK[dtype]
+            n = a.nbytes // (cols // nv * nb)
+        else:
+            n = a.size // cols
     out = np.zeros((n, cols), np.float64)
     _lib().ora_load_rows(a.ctypes.data, DTYPE[dtype], r0, n, cols, out.ctypes.data)
     return out

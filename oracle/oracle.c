@@ -53,7 +53,21 @@
  *
  * Storage formats read (converted exactly to f64): f32; bf16 (upper half of an
  * f32); Q8_0 GGML blocks {fp16 d; int8 q[32]} along the input dimension, value
- * = fp16(d) * q.
+ * = fp16(d) * q.  The k-quant stacks of the pages' Metal MoE providers
+ * (ferrum-kernels vnext MoE: Q4_K and Q6_K blocks of 256 values, 144 and 210
+ * bytes; their byte layout is GGML's, which the pages name but do not print):
+ *   Q4_K {fp16 d; fp16 dmin; u8 scales[12]; u8 qs[128]}: eight sub-blocks of
+ *     32 values, sub-block j with a 6-bit scale s_j and 6-bit min m_j packed in
+ *     scales[] (j < 4: s = scales[j] & 63, m = scales[j+4] & 63; j >= 4:
+ *     s = (scales[j+4] & 15) | (scales[j-4] >> 6) << 4,
+ *     m = (scales[j+4] >> 4) | (scales[j] >> 6) << 4); value 32j + l is the
+ *     low nibble of qs[32 (j/2) + l] for even j, the high nibble for odd j;
+ *     value = d s_j q - dmin m_j.
+ *   Q6_K {u8 ql[128]; u8 qh[64]; i8 scales[16]; fp16 d}: two halves of 128
+ *     values; in half n, value 128n + 32i + l (i = 0..3, l = 0..31) has low
+ *     four bits from ql[64n + l + 32 (i & 1)] (low nibble for i < 2, high for
+ *     i >= 2) and high two bits (qh[32n + l] >> 2i) & 3; value =
+ *     d scales[8n + (32i + l)/16] (q - 32).
  */
 #include <math.h>
 #include <stdint.h>
@@ -63,7 +77,9 @@
 #include <omp.h>
 #endif
 
-enum { ORA_F32 = 0, ORA_BF16 = 1, ORA_Q8_0 = 2 };
+/* Storage formats.  ORA_Q4_K_Q6_K is a layer format: gate/up rows in Q4_K,
+ * down rows in Q6_K.  ORA_Q6_K is a row format only. */
+enum { ORA_F32 = 0, ORA_BF16 = 1, ORA_Q8_0 = 2, ORA_Q4_K = 3, ORA_Q4_K_Q6_K = 4, ORA_Q6_K = 5 };
 enum { ORA_SILU = 0, ORA_GELU_TANH = 1 };
 
 enum { ORA_GATING_SOFTMAX = 0, ORA_GATING_SIGMOID = 1 };
@@ -128,6 +144,52 @@ static void load_row(const void* base, int dtype, int64_t r, int64_t cols, doubl
   } else if (dtype == ORA_BF16) {
     const uint16_t* p = (const uint16_t*)base + r * cols;
     for (int64_t c = 0; c < cols; ++c) out[c] = bf16_to_double(p[c]);
+  } else if (dtype == ORA_Q4_K) {
+    const uint8_t* p = (const uint8_t*)base + r * (cols / 256) * 144;
+    for (int64_t b = 0; b < cols / 256; ++b) {
+      const uint8_t* blk = p + b * 144;
+      uint16_t db, mb;
+      memcpy(&db, blk, 2);
+      memcpy(&mb, blk + 2, 2);
+      const double d = ora_fp16_to_double(db), dmin = ora_fp16_to_double(mb);
+      const uint8_t* sc = blk + 4;
+      const uint8_t* qs = blk + 16;
+      for (int j = 0; j < 8; ++j) {
+        int s, m;
+        if (j < 4) {
+          s = sc[j] & 63;
+          m = sc[j + 4] & 63;
+        } else {
+          s = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4);
+          m = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4);
+        }
+        for (int l = 0; l < 32; ++l) {
+          const uint8_t byte = qs[32 * (j / 2) + l];
+          const int q = (j % 2 == 0) ? (byte & 15) : (byte >> 4);
+          out[b * 256 + 32 * j + l] = d * s * q - dmin * m;
+        }
+      }
+    }
+  } else if (dtype == ORA_Q6_K) {
+    const uint8_t* p = (const uint8_t*)base + r * (cols / 256) * 210;
+    for (int64_t b = 0; b < cols / 256; ++b) {
+      const uint8_t* ql = p + b * 210;
+      const uint8_t* qh = ql + 128;
+      const int8_t* sc = (const int8_t*)(ql + 192);
+      uint16_t db;
+      memcpy(&db, ql + 208, 2);
+      const double d = ora_fp16_to_double(db);
+      for (int n = 0; n < 2; ++n)
+        for (int i = 0; i < 4; ++i)
+          for (int l = 0; l < 32; ++l) {
+            const uint8_t lowb = ql[64 * n + l + 32 * (i & 1)];
+            const int lo = i < 2 ? (lowb & 15) : (lowb >> 4);
+            const int hi = (qh[32 * n + l] >> (2 * i)) & 3;
+            const int q = lo | (hi << 4);
+            const int j = 32 * i + l;
+            out[b * 256 + 128 * n + j] = d * sc[8 * n + j / 16] * (q - 32);
+          }
+    }
   } else { /* Q8_0: 34-byte blocks, 32 values each */
     const uint8_t* p = (const uint8_t*)base + r * (cols / 32) * 34;
     for (int64_t b = 0; b < cols / 32; ++b) {
@@ -292,6 +354,7 @@ static ora_route route_of(const ora_desc* d) {
 /* ---- step 4: stable permutation of pair ids by expert (counting sort) ---- */
 int ora_permute(const int32_t* ids, int64_t P, int64_t E, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
                 int32_t* pair_pos) {
+  if (E < 1 || P < 0) return -1;
   for (int64_t e = 0; e < E; ++e) counts[e] = 0;
   for (int64_t p = 0; p < P; ++p) {
     if (ids[p] < 0 || ids[p] >= E) return -1;
@@ -312,17 +375,22 @@ int ora_permute(const int32_t* ids, int64_t P, int64_t E, int32_t* counts, int32
 
 /* ---- step 5/6 building block: one gated FFN on one token ---- */
 /* y[Hout] = Wd (act(Wg xt) * (Wu xt)); Wg, Wu are [F, Hin] rows at row0, Wd is [Hout, F] rows at drow0. */
-static void ffn_one(int act, int dtype, const void* Wg, const void* Wu, const void* Wd, int64_t row0, int64_t drow0,
+/* Row formats of the gate/up and of the down projections of a layer format. */
+static int gu_format(int w_dtype) { return w_dtype == ORA_Q4_K_Q6_K ? ORA_Q4_K : w_dtype; }
+static int down_format(int w_dtype) { return w_dtype == ORA_Q4_K_Q6_K ? ORA_Q6_K : w_dtype; }
+
+static void ffn_one(int act, int w_dtype, const void* Wg, const void* Wu, const void* Wd, int64_t row0, int64_t drow0,
                     int64_t F, int64_t Hin, int64_t Hout, const double* xt, double* a, double* row, double* y) {
+  const int gf = gu_format(w_dtype), df = down_format(w_dtype);
   for (int64_t i = 0; i < F; ++i) {
-    load_row(Wg, dtype, row0 + i, Hin, row);
+    load_row(Wg, gf, row0 + i, Hin, row);
     double g = dot(row, xt, Hin);
-    load_row(Wu, dtype, row0 + i, Hin, row);
+    load_row(Wu, gf, row0 + i, Hin, row);
     double u = dot(row, xt, Hin);
     a[i] = ora_act(act, g) * u;
   }
   for (int64_t j = 0; j < Hout; ++j) {
-    load_row(Wd, dtype, drow0 + j, F, row);
+    load_row(Wd, df, drow0 + j, F, row);
     y[j] = dot(row, a, F);
   }
 }

@@ -19,14 +19,14 @@ MUTANTS = {
     "renorm_dropped": ("double inv = sum_sel > 1e-20 ? 1.0 / sum_sel : 1.0 / (double)K;", "double inv = 1.0;"),
     "gelu_cubic_coefficient": ("0.044715 * g * g * g", "0.44715 * g * g * g"),
     "silu_sign": ("return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));"),
-    "down_row_base": ("load_row(Wd, dtype, drow0 + j, F, row);", "load_row(Wd, dtype, row0 + j, F, row);"),
+    "down_row_base": ("load_row(Wd, df, drow0 + j, F, row);", "load_row(Wd, df, row0 + j, F, row);"),
     "shared_gate_ignored": ("for (int64_t j = 0; j < H; ++j) o[j] += s * y[j];",
                             "for (int64_t j = 0; j < H; ++j) o[j] += y[j];"),
     "router_bias_dropped": ("s += (double)w->bias[e];", "s += 0.0;"),
     "permutation_unstable": ("int32_t pos = offsets[e] + fill[e]++;", "int32_t pos = offsets[e + 1] - 1 - fill[e]++;"),
     "q8_unsigned": ("d * (double)(int8_t)p[b * 34 + 2 + j]", "d * (double)(uint8_t)p[b * 34 + 2 + j]"),
     "slot_weight_index": ("o[j] += wk[k] * y[j];", "o[j] += wk[0] * y[j];"),
-    "up_reads_gate": ("load_row(Wu, dtype, row0 + i, Hin, row);", "load_row(Wg, dtype, row0 + i, Hin, row);"),
+    "up_reads_gate": ("load_row(Wu, gf, row0 + i, Hin, row);", "load_row(Wg, gf, row0 + i, Hin, row);"),
     "fp16_exponent_bias": ("ldexp(1024.0 + man, ex - 25)", "ldexp(1024.0 + man, ex - 24)"),
     "sigmoid_gating_ignored": ("if (gating == ORA_GATING_SIGMOID) {", "if (0) {"),
     "sigmoid_sign": ("for (int64_t e = 0; e < E; ++e) p[e] = 1.0 / (1.0 + exp(-l[e]));",
@@ -42,6 +42,16 @@ MUTANTS = {
                         "d_gate_up[p * 2 * I + i] = dh * ora_act_grad(act, g);"),
     "d_w_slots_transposed": ("s += (double)y[p * H + d] * (double)d_out[t * H + d];",
                              "s += (double)y[(k * T + t) * H + d] * (double)d_out[t * H + d];"),
+    "q4_k_nibbles_swapped": ("const int q = (j % 2 == 0) ? (byte & 15) : (byte >> 4);",
+                             "const int q = (j % 2 == 0) ? (byte >> 4) : (byte & 15);"),
+    "q4_k_high_scale_bits": ("s = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4);", "s = (sc[j + 4] & 15) | ((sc[j] >> 6) << 4);"),
+    "q4_k_min_added": ("out[b * 256 + 32 * j + l] = d * s * q - dmin * m;", "out[b * 256 + 32 * j + l] = d * s * q + dmin * m;"),
+    "q6_k_not_centred": ("out[b * 256 + 128 * n + j] = d * sc[8 * n + j / 16] * (q - 32);",
+                         "out[b * 256 + 128 * n + j] = d * sc[8 * n + j / 16] * q;"),
+    "q6_k_high_bits_shift": ("const int hi = (qh[32 * n + l] >> (2 * i)) & 3;", "const int hi = (qh[32 * n + l] >> i) & 3;"),
+    "q6_k_scale_group": ("d * sc[8 * n + j / 16]", "d * sc[8 * n + j / 32]"),
+    "q6_down_read_as_q4": ("static int down_format(int w_dtype) { return w_dtype == ORA_Q4_K_Q6_K ? ORA_Q6_K : w_dtype; }",
+                           "static int down_format(int w_dtype) { return w_dtype == ORA_Q4_K_Q6_K ? ORA_Q4_K : w_dtype; }"),
     "d_y_first_slot_weight": ("d_y[p * H + d] = (double)w[p] * (double)d_out[t * H + d];",
                               "d_y[p * H + d] = (double)w[t * K] * (double)d_out[t * H + d];"),
 }
@@ -63,6 +73,9 @@ BATTERY = [
     lambda g: pins.test_act_grad_matches_finite_difference("silu"),
     lambda g: pins.test_act_up_backward_finite_difference("gelu_tanh"),
     lambda g: pins.test_combine_backward_finite_difference(), lambda g: pins.test_combine_backward_special_cases(),
+    lambda g: pins.test_kquant_rows_match_gguf("q4_k"), lambda g: pins.test_kquant_rows_match_gguf("q6_k"),
+    lambda g: pins.test_q4_k_single_sub_block_probes(), lambda g: pins.test_q6_k_single_scale_probes(),
+    lambda g: pins.test_kquant_dense_special_case("q4_k_q6_k"),
 ]
 
 

@@ -470,3 +470,121 @@ def test_combine_backward_special_cases():
             assert d_w[t, k] == y[t, k, j]
             assert d_y[t, k, j] == w[t, k] and np.count_nonzero(d_y[t, k]) == (w[t, k] != 0)
         assert not np.delete(d_w, t, axis=0).any()
+
+
+# ---------------------------------------------------------------- k-quant stacks (Q4_K, Q6_K)
+# ferrum-kernels vnext MoE names Q4_K and Q6_K blocks of 256 values in 144 and
+# 210 bytes; the byte layout is GGML's.  The gguf package's numpy dequantiser
+# (a library routine, independent of the oracle) pins the decoding.
+
+def _kq_blocks(fmt, nblocks, seed, d=0.01, dmin=0.02):
+    rng = np.random.default_rng(seed)
+    nb = oracle.BLOCK[fmt][0]
+    b = rng.integers(0, 256, (nblocks, nb), dtype=np.uint8)
+    if fmt == "q4_k":
+        b[:, 0:2] = np.frombuffer(np.full(nblocks, d, np.float16).tobytes(), np.uint8).reshape(-1, 2)
+        b[:, 2:4] = np.frombuffer(np.full(nblocks, dmin, np.float16).tobytes(), np.uint8).reshape(-1, 2)
+    else:
+        b[:, 208:210] = np.frombuffer(np.full(nblocks, d, np.float16).tobytes(), np.uint8).reshape(-1, 2)
+    return b
+
+
+def test_kquant_block_sizes_from_the_pages():
+    gguf = pytest.importorskip("gguf")
+    T = gguf.constants.GGMLQuantizationType
+    assert oracle.BLOCK["q4_k"] == (144, 256) == gguf.constants.GGML_QUANT_SIZES[T.Q4_K][::-1]
+    assert oracle.BLOCK["q6_k"] == (210, 256) == gguf.constants.GGML_QUANT_SIZES[T.Q6_K][::-1]
+
+
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+def test_kquant_rows_match_gguf(fmt):
+    gguf = pytest.importorskip("gguf")
+    qt = {"q4_k": gguf.constants.GGMLQuantizationType.Q4_K, "q6_k": gguf.constants.GGMLQuantizationType.Q6_K}[fmt]
+    for seed, (d, dmin) in enumerate([(0.01, 0.02), (1.5e-4, 1e-3), (3e-5, 2e-5), (-0.5, 0.25), (7.0, -3.0)]):
+        rows, cols = 3, 768
+        b = _kq_blocks(fmt, rows * cols // 256, seed, d, dmin)
+        ref = gguf.quants.dequantize(b.reshape(-1), qt).reshape(rows, cols)
+        got = oracle.load_rows(b.reshape(rows, -1), fmt, cols)
+        # every term is exact in f64 and gguf rounds once to f32
+        assert np.array_equal(got.astype(np.float32), ref), (fmt, seed)
+
+
+def test_q4_k_single_sub_block_probes():
+    """One sub-block scale (or min) at a time: only that sub-block's 32 values move."""
+    for j in range(8):
+        b = np.zeros(144, np.uint8)
+        b[0:2] = np.frombuffer(np.float16(0.5).tobytes(), np.uint8)
+        b[2:4] = np.frombuffer(np.float16(0.25).tobytes(), np.uint8)
+        b[16:] = (np.arange(128) * 37 % 256).astype(np.uint8)  # varied nibbles
+        # 6-bit scale 5 and min 3 for sub-block j only
+        if j < 4:
+            b[4 + j] = 5
+            b[8 + j] = 3
+        else:
+            b[8 + j] = 5 | (3 << 4)
+        v = oracle.load_rows(b.reshape(1, -1), "q4_k", 256)[0]
+        qs = b[16:]
+        for jj in range(8):
+            byte = qs[32 * (jj // 2):32 * (jj // 2) + 32]
+            q = (byte & 15) if jj % 2 == 0 else (byte >> 4)
+            exp = 0.5 * 5 * q - 0.25 * 3 if jj == j else np.zeros(32)
+            assert np.array_equal(v[32 * jj:32 * jj + 32], exp), (j, jj)
+    # the high bits of scales[j-4] and scales[j] extend sub-block j >= 4 to 6 bits
+    b = np.zeros(144, np.uint8)
+    b[0:2] = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+    b[2:4] = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+    b[4 + 1] = 0xC0  # high bits of scales[1]: scale of sub-block 5 gets 48
+    b[4 + 5] = 0x80  # high bits of scales[5]: min of sub-block 5 gets 32
+    b[16:] = 0x11
+    v = oracle.load_rows(b.reshape(1, -1), "q4_k", 256)[0]
+    assert np.all(v[160:192] == 48 * 1 - 32)
+    assert np.all(v[32:64] == 0) and np.all(v[64:96] == 0)
+
+
+def test_q6_k_single_scale_probes():
+    rng = np.random.default_rng(9)
+    for k in range(16):
+        b = np.zeros(210, np.uint8)
+        b[:192] = rng.integers(0, 256, 192, dtype=np.uint8)
+        b[192 + k] = np.uint8(np.int8(-3).view(np.uint8))
+        b[208:210] = np.frombuffer(np.float16(0.125).tobytes(), np.uint8)
+        v = oracle.load_rows(b.reshape(1, -1), "q6_k", 256)[0]
+        nz = np.nonzero(np.arange(256) // 16 == k)[0]
+        assert not np.delete(v, nz).any()
+        # brute force of value 16k + l: 6-bit code from ql/qh, centred at 32
+        for idx in nz:
+            n, j = divmod(idx, 128)
+            i, l = divmod(j, 32)
+            lowb = b[64 * n + l + 32 * (i & 1)]
+            q = (lowb & 15 if i < 2 else lowb >> 4) | (((b[128 + 32 * n + l] >> (2 * i)) & 3) << 4)
+            assert v[idx] == 0.125 * -3 * (int(q) - 32)
+    # q = 32 everywhere decodes to zero whatever the scales
+    b = np.zeros(210, np.uint8)
+    b[128:192] = 0xAA  # high bits 2 in every pair -> q = 32
+    b[192:208] = 7
+    b[208:210] = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+    assert not oracle.load_rows(b.reshape(1, -1), "q6_k", 256).any()
+
+
+@pytest.mark.parametrize("w_dtype", ["q4_k", "q4_k_q6_k"])
+def test_kquant_dense_special_case(w_dtype):
+    """E = 1, K = 1: the layer is the dense FFN on gguf-dequantised weights (numpy matmuls)."""
+    gguf = pytest.importorskip("gguf")
+    Q = gguf.constants.GGMLQuantizationType
+    T, H, I = 5, 512, 256
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    g = _kq_blocks("q4_k", I * H // 256, 1, 1e-3, 5e-3)
+    u = _kq_blocks("q4_k", I * H // 256, 2, 1e-3, 5e-3)
+    dfmt = "q6_k" if w_dtype == "q4_k_q6_k" else "q4_k"
+    dq = _kq_blocks(dfmt, H * I // 256, 3, 2e-4, 5e-3)
+    L = oracle.Layer(T=T, H=H, E=1, I=I, K=1, act="silu", renormalize=True, act_dtype="f32", w_dtype=w_dtype,
+                     router_dtype="f32", x=x, router=np.zeros((1, H), np.float32), gate=g.reshape(1, I, -1),
+                     up=u.reshape(1, I, -1), down=dq.reshape(1, H, -1))
+    out = oracle.layer(L)["out"]
+    G = gguf.quants.dequantize(g.reshape(-1), Q.Q4_K).reshape(I, H).astype(np.float64)
+    U = gguf.quants.dequantize(u.reshape(-1), Q.Q4_K).reshape(I, H).astype(np.float64)
+    D = gguf.quants.dequantize(dq.reshape(-1), Q.Q6_K if dfmt == "q6_k" else Q.Q4_K).reshape(H, I).astype(np.float64)
+    a = x.astype(np.float64) @ G.T
+    ref = ((a / (1 + np.exp(-a))) * (x.astype(np.float64) @ U.T)) @ D.T
+    assert np.allclose(out, ref, rtol=1e-9, atol=1e-9 * np.max(np.abs(ref)))

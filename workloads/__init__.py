@@ -20,7 +20,9 @@ q8_0_decode_t16        16     2048  128  768   8  silu       Q8_0   none
 Distributions: x ~ N(0,1); router W and the shared-gate vector w_s ~ N(0,0.02)
 (second parameter = standard deviation); expert and shared projections
 ~ N(0, 1/sqrt(fan_in)); Q8_0 blocks q ~ U{-127..127}, d ~ U[0.001,0.01] rounded
-to fp16; bf16 tensors are rounded to nearest-even from the f32 samples.  The
+to fp16; Q4_K / Q6_K blocks with every quant, scale and min byte uniform over
+0..255 and fp16 d ~ U[1e-4, 2e-4], dmin ~ U[7.5e-4, 1.5e-3] (Q4_K) or
+d ~ U[2e-5, 4e-5] (Q6_K, fp16 subnormals included); bf16 tensors are rounded to nearest-even from the f32 samples.  The
 skewed workload adds a per-expert router bias b_e = 2 ln p_r with Zipf(s=1.1)
 rank r = e + 1 over the 256 experts.
 """
@@ -39,6 +41,7 @@ _SO = os.path.join(_HERE, "libmoegen.so")
 _SRC = os.path.join(_HERE, "gen.c")
 
 F32, BF16, Q8_0 = "f32", "bf16", "q8_0"
+Q4_K, Q4_K_Q6_K = "q4_k", "q4_k_q6_k"   # all projections Q4_K; gate/up Q4_K with down Q6_K
 SILU, GELU_TANH = "silu", "gelu_tanh"
 
 
@@ -101,6 +104,36 @@ def q8_0_blocks(seed: int, stream: int, shape, q_lo=-127, q_hi=127, d_lo=0.001, 
     return out.reshape(*lead, rows, cols // 32, 34)
 
 
+def _bytes(seed, stream, n):
+    u = uniform(seed, stream, (n,), 0.0, 256.0)
+    return np.minimum(np.floor(u), 255).astype(np.uint8)
+
+
+def _fp16_bits(seed, stream, n, lo, hi):
+    return uniform(seed, stream, (n,), lo, hi).astype(np.float16).view(np.uint8).reshape(n, 2)
+
+
+def kquant_blocks(seed: int, stream: int, shape, fmt: str, d=(1e-4, 2e-4), dmin=(7.5e-4, 1.5e-3)) -> np.ndarray:
+    """GGML Q4_K (144-byte) or Q6_K (210-byte) blocks of 256 values for a weight of logical shape
+    (..., rows, cols): uint8 [..., rows, cols/256, nbytes].  Every quant, scale and min byte is uniform
+    over 0..255; the fp16 super-block scale d (and Q4_K's dmin) are uniform over the given ranges."""
+    *lead, rows, cols = shape
+    assert cols % 256 == 0
+    nblk = int(np.prod(lead, dtype=np.int64)) * rows * (cols // 256)
+    if fmt == Q4_K:
+        b = np.empty((nblk, 144), np.uint8)
+        b[:, 0:2] = _fp16_bits(seed, stream | 1 << 8, nblk, *d)
+        b[:, 2:4] = _fp16_bits(seed, stream | 2 << 8, nblk, *dmin)
+        b[:, 4:] = _bytes(seed, stream | 3 << 8, nblk * 140).reshape(nblk, 140)
+    elif fmt == "q6_k":
+        b = np.empty((nblk, 210), np.uint8)
+        b[:, :208] = _bytes(seed, stream | 3 << 8, nblk * 208).reshape(nblk, 208)
+        b[:, 208:210] = _fp16_bits(seed, stream | 1 << 8, nblk, *d)
+    else:
+        raise ValueError(fmt)
+    return b.reshape(*lead, rows, cols // 256, b.shape[1])
+
+
 def f32_to_bf16(a: np.ndarray) -> np.ndarray:
     a = np.ascontiguousarray(a, np.float32)
     out = np.empty(a.shape, np.uint16)
@@ -159,6 +192,9 @@ CONFIGS = {
     # routing variants on the prefill shapes: sigmoid gating, 8 groups of 8 experts, 4 groups kept
     "grouped_sigmoid_t512": Spec(T=512, H=2048, E=64, I=1024, K=8, gating="sigmoid", n_groups=8, topk_groups=4,
                                  name="grouped_sigmoid_t512"),
+    # Q8_0-decode shapes with the k-quant stacks of the Metal MoE providers: gate/up Q4_K, down Q6_K
+    "q4k_q6k_decode_t16": Spec(T=16, H=2048, E=128, I=768, K=8, act_dtype=F32, w_dtype=Q4_K_Q6_K, router_dtype=F32,
+                               name="q4k_q6k_decode_t16"),
 }
 CONFIG_ORDER = list(CONFIGS)
 BASE_SEED = 0xB2000000
@@ -189,9 +225,13 @@ class Workload:
 S_X, S_ROUTER, S_GATE, S_UP, S_DOWN, S_SH_GATE, S_SH_UP, S_SH_DOWN, S_SH_GATE_W = range(1, 10)
 
 
-def _weight(seed, stream, shape, fan_in, w_dtype):
+def _weight(seed, stream, shape, fan_in, w_dtype, down=False):
     if w_dtype == Q8_0:
         return q8_0_blocks(seed, stream, shape)
+    if w_dtype in (Q4_K, Q4_K_Q6_K):
+        if down and w_dtype == Q4_K_Q6_K:  # |d sc (q - 32)| ~ d * 74 * 18.5: about 1/sqrt(I) for I = 768
+            return kquant_blocks(seed, stream, shape, "q6_k", d=(2e-5, 4e-5))
+        return kquant_blocks(seed, stream, shape, Q4_K)
     return normal(seed, stream, shape, 1.0 / math.sqrt(fan_in), w_dtype)
 
 
@@ -209,12 +249,12 @@ def make(spec: Spec, seed: int | None = None, x_std: float = 1.0) -> Workload:
     bias = zipf_log_bias(E) if spec.router_bias == "zipf1.1" else None
     gate = _weight(seed, S_GATE, (E, I, H), H, spec.w_dtype)
     up = _weight(seed, S_UP, (E, I, H), H, spec.w_dtype)
-    down = _weight(seed, S_DOWN, (E, H, I), I, spec.w_dtype)
+    down = _weight(seed, S_DOWN, (E, H, I), I, spec.w_dtype, down=True)
     wl = Workload(spec, seed, x, router, bias, gate, up, down)
     if Is > 0:
         wl.sh_gate = _weight(seed, S_SH_GATE, (Is, H), H, spec.w_dtype)
         wl.sh_up = _weight(seed, S_SH_UP, (Is, H), H, spec.w_dtype)
-        wl.sh_down = _weight(seed, S_SH_DOWN, (H, Is), Is, spec.w_dtype)
+        wl.sh_down = _weight(seed, S_SH_DOWN, (H, Is), Is, spec.w_dtype, down=True)
         if spec.shared_gated:
             wl.sh_gate_w = normal(seed, S_SH_GATE_W, (H,), 0.02, spec.router_dtype)
     return wl
