@@ -57,7 +57,9 @@ def algorithmic(spec, counts):
     T, H, E, I, K, Is = spec.T, spec.H, spec.E, spec.I, spec.K, spec.shared_I
     P = T * K
     touched = int(np.count_nonzero(counts))
-    wb = {"f32": 4, "bf16": 2, "q8_0": 1 + 2.0 / 32}[spec.w_dtype]
+    # stored bytes per weight of the gate/up and of the down projections
+    wb = {"f32": 4, "bf16": 2, "q8_0": 1 + 2.0 / 32, "q4_k": 144 / 256, "q4_k_q6_k": 144 / 256}[spec.w_dtype]
+    wbd = 210 / 256 if spec.w_dtype == "q4_k_q6_k" else wb
     ab = 4 if spec.act_dtype == "f32" else 2
     rb = 4 if spec.router_dtype == "f32" else 2
     tc = spec.act_dtype == "bf16" and spec.w_dtype == "bf16" and T > 64
@@ -66,7 +68,7 @@ def algorithmic(spec, counts):
     k["expert_gate_up_gemm"] = k["stream_gate_up"] = dict(
         bytes=touched * 2 * I * H * wb + P * H * ab + P * I * hb, flops=2.0 * P * 2 * I * H)
     k["expert_down_gemm"] = k["stream_down"] = dict(
-        bytes=touched * H * I * wb + P * I * hb + P * H * 4 + P * 4, flops=2.0 * P * H * I)
+        bytes=touched * H * I * wbd + P * I * hb + P * H * 4 + P * 4, flops=2.0 * P * H * I)
     k["router_gemm"] = k["router_logits"] = dict(bytes=E * H * rb + T * H * ab + T * E * 4, flops=2.0 * T * E * H)
     k["router_topk"] = dict(bytes=T * E * 4 * (2 if spec.router_bias else 1) + P * 8, flops=0)
     k["permute"] = dict(bytes=P * 4 * 3 + (2 * E + 1) * 4, flops=0)
@@ -74,8 +76,9 @@ def algorithmic(spec, counts):
     k["combine"] = dict(bytes=P * H * 4 + (T * H * 4 if Is else 0) + T * H * ab, flops=0)
     if Is:
         k["shared_gate_up_gemm"] = dict(bytes=2 * Is * H * wb + T * H * ab + T * Is * hb, flops=2.0 * T * 2 * Is * H)
-        k["shared_down_gemm"] = dict(bytes=Is * H * wb + T * Is * hb + T * H * 4, flops=2.0 * T * H * Is)
-    layer = dict(bytes=touched * 3 * I * H * wb + E * H * rb + (3 * Is * H * wb if Is else 0) + 2 * T * H * ab,
+        k["shared_down_gemm"] = dict(bytes=Is * H * wbd + T * Is * hb + T * H * 4, flops=2.0 * T * H * Is)
+    layer = dict(bytes=touched * (2 * wb + wbd) * I * H + E * H * rb + ((2 * wb + wbd) * Is * H if Is else 0)
+                 + 2 * T * H * ab,
                  flops=2.0 * (T * E * H + P * 3 * H * I + T * 3 * H * Is))
     # fused launches: the sum of the steps they replace
     k["route_permute_gather"] = dict(bytes=sum(k[n]["bytes"] for n in ("router_topk", "permute", "gather_rows")),
@@ -355,7 +358,7 @@ def run_ours(args, spec):
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": spec.act_dtype if spec.w_dtype != "q8_0" else "q8_0xf32",
+            "vs_baseline": None, "dtype": spec.act_dtype if spec.w_dtype in ("f32", "bf16") else f"{spec.w_dtype}x{spec.act_dtype}",
             "data": "synthetic",
             "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
                        "act": spec.act, "shared_I": spec.shared_I, "parallelism": f"replicas{ws_n}",

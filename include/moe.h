@@ -51,7 +51,10 @@ typedef enum {
   MOE_ERR_DEVICE_INDEX = 6 /* device: an expert id outside [0, E) reached the permutation */
 } moe_status;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_Q8_0 = 2 } moe_dtype;
+/* Storage formats.  MOE_Q4_K and MOE_Q4_K_Q6_K are expert-weight formats only
+ * (the k-quant stacks of the Metal MoE providers, ferrum-kernels vnext MoE:
+ * "q4k" for all projections, "q4k_q6k" for Q4_K gate/up with Q6_K down). */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_Q8_0 = 2, MOE_Q4_K = 3, MOE_Q4_K_Q6_K = 4 } moe_dtype;
 
 /* SiLU(g) = g / (1 + e^-g)  (hf2q qwen35/gpu_ffn.rs, silu_mul_cpu);
  * GELU_TANH(g) = 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3)))
@@ -68,7 +71,8 @@ typedef struct moe_desc {
   int32_t act;             /* moe_act, used by routed and shared experts */
   int32_t renormalize;     /* 1: selected gate values divided by their sum; 0: the gate values themselves */
   int32_t act_dtype;       /* MOE_F32 | MOE_BF16: x and out */
-  int32_t w_dtype;         /* MOE_F32 | MOE_BF16 | MOE_Q8_0: expert and shared projections */
+  int32_t w_dtype;         /* MOE_F32 | MOE_BF16 | MOE_Q8_0 | MOE_Q4_K | MOE_Q4_K_Q6_K: expert and shared
+                              projections (the k-quant formats need H, I and shared_I multiples of 256) */
   int32_t router_dtype;    /* MOE_F32 | MOE_BF16: router W and the shared-gate vector w_s */
   int32_t has_router_bias; /* 1: logits += b_e before selection (ferrox-models decoder.rs, gpt_oss_ffn) */
   int32_t shared_I;        /* 0: no shared expert */
@@ -89,7 +93,16 @@ typedef struct moe_desc {
  * same shapes and the *_scale pointers hold one fp16 scale per 32 consecutive
  * inputs ([E,I,H/32], [E,H,I/32], [Is,H/32], [H,Is/32]); value = scale * q.
  * moe_q8_0_split() converts GGML Q8_0 blocks into this split form.
- * Unused pointers may be NULL.
+ * For MOE_Q4_K every projection holds GGML Q4_K blocks in place, row by row:
+ * a row of n inputs is n/256 blocks of 144 bytes {fp16 d; fp16 dmin;
+ * u8 scales[12]; u8 qs[128]}, so gate is [E,I,H/256,144] bytes; the *_scale
+ * pointers are unused.  For MOE_Q4_K_Q6_K gate/up (and sh_gate/sh_up) are Q4_K
+ * as above and down / sh_down hold GGML Q6_K blocks {u8 ql[128]; u8 qh[64];
+ * i8 scales[16]; fp16 d} in the split form of moe_q6_k_split(): down is
+ * [E*H, I/256, 192] bytes (ql then qh of each block) and down_scale
+ * [E*H, srow] bytes with srow = ceil(18 * I/256 / 16) * 16: the 16 scales of
+ * every block of the row, then the fp16 d of every block, then zeros.
+ * All weight pointers are 16-byte aligned.  Unused pointers may be NULL.
  */
 typedef struct moe_weights {
   const void* router;
@@ -288,6 +301,22 @@ moe_status moe_combine_backward(int64_t T, int64_t K, int64_t H, const float* y,
  */
 moe_status moe_act_up_backward(int64_t P, int64_t I, int32_t act, const float* gate_up, const float* d_h,
                                float* d_gate_up, moe_stream_t stream);
+
+/*
+ * Split GGML Q6_K blocks (210 bytes {u8 ql[128]; u8 qh[64]; i8 scales[16];
+ * fp16 d} per 256 inputs, along the input dimension) of a [rows, cols] matrix
+ * into the 16-byte aligned form moe_weights expects for the down projections
+ * of MOE_Q4_K_Q6_K: q [rows, cols/256, 192] bytes (ql, qh of each block) and
+ * scales [rows, srow] bytes, srow = ceil(18 * cols/256 / 16) * 16 (the int8
+ * scales of the row's blocks, then their fp16 d, then zero padding).  Every
+ * byte is moved unchanged: a one-time load step (ferrum-kernels vnext MoE,
+ * prepare_q6_expert_part, prepares the Q6_K expert planes at load).
+ * blocks: device, any alignment; q and scales: device, 16-byte aligned,
+ * caller-owned.  cols % 256 != 0, negative sizes, null pointers or unaligned
+ * outputs: MOE_ERR_INVALID_ARG.  rows * cols == 0 does nothing.
+ */
+moe_status moe_q6_k_split(const void* blocks, int64_t rows, int64_t cols, void* q, void* scales,
+                          moe_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word of

@@ -18,9 +18,9 @@ from dataclasses import dataclass, fields
 from . import _lib
 from ._lib import (MOE_ACT_GELU_TANH, MOE_ACT_SILU, MOE_BF16, MOE_ERR_CUDA, MOE_ERR_DEVICE_INDEX,  # noqa: F401
                    MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_F32, MOE_OK,
-                   MOE_Q8_0, MoeError, check, status_string)
+                   MOE_Q4_K, MOE_Q4_K_Q6_K, MOE_Q8_0, MoeError, check, status_string)
 
-DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "q8_0": MOE_Q8_0}
+DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "q8_0": MOE_Q8_0, "q4_k": MOE_Q4_K, "q4_k_q6_k": MOE_Q4_K_Q6_K}
 ACTS = {"silu": MOE_ACT_SILU, "gelu_tanh": MOE_ACT_GELU_TANH}
 GATINGS = {"softmax": 0, "sigmoid": 1}  # moe_gating
 
@@ -170,6 +170,17 @@ def act_up_backward(act, gate_up, d_h, d_gate_up, stream=None):
     P, I = d_h.shape
     check(_lib.lib().moe_act_up_backward(P, I, ACTS[act] if isinstance(act, str) else act, _ptr(gate_up), _ptr(d_h),
                                          _ptr(d_gate_up), _stream(stream)), "moe_act_up_backward")
+
+
+def q6_k_split(blocks, rows, cols, q, scales, stream=None):
+    """moe_q6_k_split: GGML Q6_K blocks -> 16-byte aligned quant and scale planes."""
+    check(_lib.lib().moe_q6_k_split(_ptr(blocks), rows, cols, _ptr(q), _ptr(scales), _stream(stream)),
+          "moe_q6_k_split")
+
+
+def q6_k_srow_bytes(cols: int) -> int:
+    """Bytes of one scale row of the Q6_K split form (include/moe.h)."""
+    return (cols // 256 * 18 + 15) // 16 * 16
 
 
 def last_device_status(stream=None) -> int:

@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(HERE, "libmoe.so")
 # enums (include/moe.h)
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
     MOE_ERR_DEVICE_INDEX = range(7)
-MOE_F32, MOE_BF16, MOE_Q8_0 = 0, 1, 2
+MOE_F32, MOE_BF16, MOE_Q8_0, MOE_Q4_K, MOE_Q4_K_Q6_K = 0, 1, 2, 3, 4
 MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 MOE_ACT_SILU, MOE_ACT_GELU_TANH = 0, 1
 
@@ -23,7 +23,8 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route
            "moe_combine", "moe_layer", "moe_layer_host", "moe_layer_noalloc", "moe_q8_0_split",
            "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
            "moe_debug_set_wait_limit", "moe_debug_set_skip_stage", "moe_set_fused_decode",
-           "moe_workspace_regions", "moe_set_fused_front", "moe_combine_backward", "moe_act_up_backward")
+           "moe_workspace_regions", "moe_set_fused_front", "moe_combine_backward", "moe_act_up_backward",
+           "moe_q6_k_split")
 
 
 class MoeDesc(ctypes.Structure):
@@ -73,12 +74,13 @@ def lib():
         L.moe_layer_host.argtypes = [DP, P, WP, P, P, P, P, S, P]
         L.moe_layer_noalloc.argtypes = [DP, P, WP, P, P]
         L.moe_q8_0_split.argtypes = [P, I64, I64, P, P, P]
+        L.moe_q6_k_split.argtypes = [P, I64, I64, P, P, P]
         L.moe_last_device_status.argtypes = [P]
         L.moe_combine_backward.argtypes = [I64, I64, I64, P, P, P, P, P, P]
         L.moe_act_up_backward.argtypes = [I64, I64, I32, P, P, P, P]
         for f in (L.moe_route, L.moe_permute, L.moe_expert_ffn, L.moe_combine, L.moe_layer, L.moe_layer_host,
                   L.moe_layer_noalloc, L.moe_q8_0_split, L.moe_last_device_status, L.moe_combine_backward,
-                  L.moe_act_up_backward):
+                  L.moe_act_up_backward, L.moe_q6_k_split):
             f.restype = I32
         L.moe_launch_count.restype = ctypes.c_uint64
         L.moe_trace_enable.argtypes = [I32]

@@ -140,7 +140,7 @@ __device__ __forceinline__ void router_stage_x(const DecodeArgs& a, float* xs, i
   }
 }
 
-template <typename XT, int WK>
+template <typename XT, int WKG, int WKD>
 __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_expert[kMaxGroups], s_first[kMaxGroups], s_count[kMaxGroups], s_poff[kMaxGroups + 1];
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     __syncthreads();
     int p0, p1;
     cta_pairs(tb, s_ph[0], p0, p1);
-    if (!s_abort) run_phase<XT, WK, true, kDecodeTok>(s_ph[0], tb, p0, p1, sm);
+    if (!s_abort) run_phase<XT, WKG, true, kDecodeTok>(s_ph[0], tb, p0, p1, sm);
   }
   cta_grid_sync(a, &s_abort, &s_flag);
 
@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     __syncthreads();
     int p0, p1;
     cta_pairs(tb, s_ph[1], p0, p1);
-    if (!s_abort) run_phase<float, WK, false, kDecodeTok>(s_ph[1], tb, p0, p1, sm);
+    if (!s_abort) run_phase<float, WKD, false, kDecodeTok>(s_ph[1], tb, p0, p1, sm);
   }
   const bool ok = cta_grid_sync(a, &s_abort, &s_flag);
 
@@ -384,24 +384,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
 }
 
 // Static shared memory of a kernel instance (queried once).
-template <typename XT, int WK>
+template <typename XT, int WKG, int WKD>
 int static_smem() {
   static std::atomic<int> bytes{-1};
   int b = bytes.load();
   if (b < 0) {
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, decode_layer_kernel<XT, WK>) != cudaSuccess) return -1;
+    if (cudaFuncGetAttributes(&fa, decode_layer_kernel<XT, WKG, WKD>) != cudaSuccess) return -1;
     b = static_cast<int>(fa.sharedSizeBytes);
     bytes.store(b);
   }
   return b;
 }
 
-template <typename XT, int WK>
+template <typename XT, int WKG, int WKD>
 cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
-  auto kern = decode_layer_kernel<XT, WK>;
+  auto kern = decode_layer_kernel<XT, WKG, WKD>;
   const int smem = a.stage_bytes + 16 * P;
-  const int st = static_smem<XT, WK>();
+  const int st = static_smem<XT, WKG, WKD>();
   if (st < 0 || smem + st > c.smem_optin) return cudaErrorInvalidValue;
   const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -419,6 +419,19 @@ cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+template <typename XT>
+cudaError_t launch_kinds(const Ctx& c, const DecodeArgs& a, int P, int wkg, int wkd) {
+  if (wkg == WK_F32) return launch_fused<XT, WK_F32, WK_F32>(c, a, P);
+  if (wkg == WK_BF16) return launch_fused<XT, WK_BF16, WK_BF16>(c, a, P);
+  if (wkg == WK_Q8) return launch_fused<XT, WK_Q8, WK_Q8>(c, a, P);
+  if (wkd == WK_Q6K) return launch_fused<XT, WK_Q4K, WK_Q6K>(c, a, P);
+  return launch_fused<XT, WK_Q4K, WK_Q4K>(c, a, P);
+}
+
+cudaError_t launch_by_kind(const Ctx& c, const DecodeArgs& a, int P, bool x_f32, int wkg, int wkd) {
+  return x_f32 ? launch_kinds<float>(c, a, P, wkg, wkd) : launch_kinds<__nv_bfloat16>(c, a, P, wkg, wkd);
+}
+
 }  // namespace
 
 size_t decode_router_parts_floats(int T, int H, int E, bool shared_gate) {
@@ -430,14 +443,14 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
   if (L.T <= 0) return cudaSuccess;
   const int P = L.T * L.K;
   if (L.T > kMaxDecodeT || P > kMaxDecodePairs || L.E > 256 || (L.H % 4)) return cudaErrorInvalidValue;
-  const int wk = wk_of(L.w_dtype);
+  const int wkg = wk_gate_up(L.w_dtype), wkd = wk_down(L.w_dtype);
   const int ab = L.x_dtype == MOE_F32 ? 4 : 2;
   DecodeArgs a{};
   // gate/up: routed experts read x rows through the pair list, the shared expert reads x row r
-  a.g.plan[0] = make_plan(wk, true, L.H, L.I, ab, L.T, kDecodeTok);
-  a.g.plan[1] = L.Is > 0 ? make_plan(wk, true, L.H, L.Is, ab, L.T, kDecodeTok) : a.g.plan[0];
-  a.d.plan[0] = make_plan(wk, false, L.I, L.H, 4, L.T, kDecodeTok);
-  a.d.plan[1] = L.Is > 0 ? make_plan(wk, false, L.Is, L.H, 4, L.T, kDecodeTok) : a.d.plan[0];
+  a.g.plan[0] = make_plan(wkg, true, L.H, L.I, ab, L.T, kDecodeTok);
+  a.g.plan[1] = L.Is > 0 ? make_plan(wkg, true, L.H, L.Is, ab, L.T, kDecodeTok) : a.g.plan[0];
+  a.d.plan[0] = make_plan(wkd, false, L.I, L.H, 4, L.T, kDecodeTok);
+  a.d.plan[1] = L.Is > 0 ? make_plan(wkd, false, L.Is, L.H, 4, L.T, kDecodeTok) : a.d.plan[0];
   // phases R and S use the stage area for an f32 x chunk of a token group and one logit row per warp
   int stage = std::max(kTokGroup * kRouterChunk * 4, kWarps * kMaxRouterRows * 4);
   for (const Plan* p : {&a.g.plan[0], &a.g.plan[1], &a.d.plan[0], &a.d.plan[1]}) {
@@ -502,14 +515,7 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
   a.out = L.out;
   a.status = c.status;
   a.wait_limit = c.wait_limit;
-  if (L.x_dtype == MOE_F32) {
-    if (wk == WK_F32) return launch_fused<float, WK_F32>(c, a, P);
-    if (wk == WK_BF16) return launch_fused<float, WK_BF16>(c, a, P);
-    return launch_fused<float, WK_Q8>(c, a, P);
-  }
-  if (wk == WK_F32) return launch_fused<__nv_bfloat16, WK_F32>(c, a, P);
-  if (wk == WK_BF16) return launch_fused<__nv_bfloat16, WK_BF16>(c, a, P);
-  return launch_fused<__nv_bfloat16, WK_Q8>(c, a, P);
+  return launch_by_kind(c, a, P, L.x_dtype == MOE_F32, wkg, wkd);
 }
 
 }  // namespace moe

@@ -99,6 +99,7 @@ cudaError_t launch_combine_backward(const Ctx& c, const float* y, const float* w
                                     int K, long long H, float* d_y, float* d_w);
 cudaError_t launch_act_up_backward(const Ctx& c, const float* gate_up, const float* d_h, long long P, long long I,
                                    int act, float* d_gate_up);
+cudaError_t launch_q6_k_split(const Ctx& c, const void* blocks, int64_t rows, int64_t cols, void* q, void* scales);
 cudaError_t launch_q8_0_split(const Ctx& c, const void* blocks, int64_t rows, int64_t cols, int8_t* q,
                               void* scales);
 

@@ -112,10 +112,13 @@ moe_status check_desc(const moe_desc* d) {
       (d->has_router_bias != 0 && d->has_router_bias != 1) || (d->has_shared_gate != 0 && d->has_shared_gate != 1))
     return MOE_ERR_INVALID_ARG;
   if ((d->act_dtype != MOE_F32 && d->act_dtype != MOE_BF16) ||
-      (d->w_dtype != MOE_F32 && d->w_dtype != MOE_BF16 && d->w_dtype != MOE_Q8_0) ||
+      (d->w_dtype != MOE_F32 && d->w_dtype != MOE_BF16 && d->w_dtype != MOE_Q8_0 && d->w_dtype != MOE_Q4_K &&
+       d->w_dtype != MOE_Q4_K_Q6_K) ||
       (d->router_dtype != MOE_F32 && d->router_dtype != MOE_BF16))
     return MOE_ERR_INVALID_ARG;
   if (d->H % 32 || d->I % 32 || d->shared_I % 32) return MOE_ERR_UNSUPPORTED;
+  if ((d->w_dtype == MOE_Q4_K || d->w_dtype == MOE_Q4_K_Q6_K) && (d->H % 256 || d->I % 256 || d->shared_I % 256))
+    return MOE_ERR_UNSUPPORTED;
   if (d->gating != MOE_GATING_SOFTMAX && d->gating != MOE_GATING_SIGMOID) return MOE_ERR_INVALID_ARG;
   if (d->n_groups < 0 || d->n_groups > 32) return MOE_ERR_INVALID_ARG;
   if (d->n_groups > 1) {
@@ -359,6 +362,7 @@ moe_status check_expert_weights(const moe_desc& d, const moe_weights* w) {
   if (!w || !w->gate || !w->up || !w->down) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w->gate) || !aligned16(w->up) || !aligned16(w->down)) return MOE_ERR_INVALID_ARG;
   if (d.w_dtype == MOE_Q8_0 && (!w->gate_scale || !w->up_scale || !w->down_scale)) return MOE_ERR_INVALID_ARG;
+  if (d.w_dtype == MOE_Q4_K_Q6_K && (!w->down_scale || !aligned16(w->down_scale))) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -369,6 +373,7 @@ moe_status check_shared_weights(const moe_desc& d, const moe_weights* w) {
   if (!aligned16(w->sh_gate) || !aligned16(w->sh_up) || !aligned16(w->sh_down)) return MOE_ERR_INVALID_ARG;
   if (d.w_dtype == MOE_Q8_0 && (!w->sh_gate_scale || !w->sh_up_scale || !w->sh_down_scale))
     return MOE_ERR_INVALID_ARG;
+  if (d.w_dtype == MOE_Q4_K_Q6_K && (!w->sh_down_scale || !aligned16(w->sh_down_scale))) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -694,6 +699,16 @@ moe_status moe_act_up_backward(int64_t P, int64_t I, int32_t act, const float* g
   moe::Ctx c;
   if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
   return from_cuda(moe::launch_act_up_backward(c, gate_up, d_h, P, I, act, d_gate_up));
+}
+
+moe_status moe_q6_k_split(const void* blocks, int64_t rows, int64_t cols, void* q, void* scales,
+                          moe_stream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 256 || cols > (1LL << 30)) return MOE_ERR_INVALID_ARG;
+  if (rows * cols == 0) return MOE_OK;
+  if (!blocks || !q || !scales || !aligned16(q) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
+  moe::Ctx c;
+  if (!make_ctx(reinterpret_cast<cudaStream_t>(stream), &c)) return MOE_ERR_CUDA;
+  return from_cuda(moe::launch_q6_k_split(c, blocks, rows, cols, q, scales));
 }
 
 moe_status moe_last_device_status(moe_stream_t stream) {

@@ -21,7 +21,10 @@
 // Q8_0 codes are widened exactly in registers (the exponent-bias trick: with
 // the sign bit flipped, byte b is u = b + 128 and the word 0x4B0000uu is the
 // float 2^23 + u) and the fp16 block scale is applied to each 8-value
-// partial sum.
+// partial sum.  The k-quant stacks (Q4_K read in place, Q6_K in the split form
+// of moe_q6_k_split) give each lane one 32-value chunk of a 256-value block per
+// step; their codes are widened the same way and each weight is formed with one
+// rounding (d s q - dmin m for Q4_K, d s (q - 32) for Q6_K) before the dots.
 //
 //  gate/up (DUAL): h[r, i] = act(W_gate[e,i] . a_r) * (W_up[e,i] . a_r)
 //  down          : y[dest_r, j] = scale_r * (W_down[e,j] . a_r)
@@ -34,7 +37,7 @@
 namespace moe {
 namespace stream {
 
-enum { WK_F32 = 0, WK_BF16 = 1, WK_Q8 = 2 };
+enum { WK_F32 = 0, WK_BF16 = 1, WK_Q8 = 2, WK_Q4K = 3, WK_Q6K = 4 };
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
@@ -108,7 +111,20 @@ struct Smem {
 };
 
 // ---------------------------------------------------------------- host planning
-inline int wk_of(int w_dtype) { return w_dtype == MOE_F32 ? WK_F32 : (w_dtype == MOE_BF16 ? WK_BF16 : WK_Q8); }
+// Weight kinds of the gate/up and of the down projections of a layer format.
+inline int wk_gate_up(int w_dtype) {
+  switch (w_dtype) {
+    case MOE_F32: return WK_F32;
+    case MOE_BF16: return WK_BF16;
+    case MOE_Q8_0: return WK_Q8;
+    default: return WK_Q4K;  // MOE_Q4_K, MOE_Q4_K_Q6_K
+  }
+}
+inline int wk_down(int w_dtype) { return w_dtype == MOE_Q4_K_Q6_K ? WK_Q6K : wk_gate_up(w_dtype); }
+
+// Bytes of the scale row of a Q6_K split matrix with Kdim inputs: 16 int8
+// scales per block, then one fp16 d per block, padded to 16 bytes.
+__host__ __device__ constexpr int q6k_srow_bytes(int Kdim) { return ((Kdim / 256) * 18 + 15) / 16 * 16; }
 
 inline Plan make_plan(int wk, bool dual, int Kdim, int Nout, int act_bytes_per_elem, int max_tokens,
                       int tok_cap = kMaxTok) {
@@ -116,8 +132,8 @@ inline Plan make_plan(int wk, bool dual, int Kdim, int Nout, int act_bytes_per_e
   p.Kdim = Kdim;
   p.Nout = Nout;
   const int eb = wk == WK_F32 ? 4 : (wk == WK_BF16 ? 2 : 1);
-  p.row_bytes = Kdim * eb;
-  p.srow_bytes = wk == WK_Q8 ? (Kdim / 32) * 2 : 0;
+  p.row_bytes = wk == WK_Q4K ? (Kdim / 256) * 144 : (wk == WK_Q6K ? (Kdim / 256) * 192 : Kdim * eb);
+  p.srow_bytes = wk == WK_Q8 ? (Kdim / 32) * 2 : (wk == WK_Q6K ? q6k_srow_bytes(Kdim) : 0);
   p.xrow_bytes = Kdim * act_bytes_per_elem;
   p.TS = std::max(1, std::min(std::min(kMaxTok, tok_cap), max_tokens));
   while (p.TS > 1 && p.TS * p.xrow_bytes > kXStageBytes) --p.TS;
@@ -125,7 +141,9 @@ inline Plan make_plan(int wk, bool dual, int Kdim, int Nout, int act_bytes_per_e
   // a pair streams 2 rows of weights; Q8_0 spends about 1 ALU op per weight
   // per token on top of the widening, f32 / bf16 far less than the bytes cost
   p.cost_base = 2 * (p.row_bytes + p.srow_bytes) / 64 + 1;
-  p.cost_tok = wk == WK_Q8 ? std::max(1, 2 * Kdim / 256) : std::max(1, 2 * Kdim / 2048);
+  const bool kq = wk == WK_Q4K || wk == WK_Q6K;
+  if (kq) p.cost_base += 2 * Kdim / 128;  // forming the weights costs ALU work of its own
+  p.cost_tok = (wk == WK_Q8 || kq) ? std::max(1, 2 * Kdim / 256) : std::max(1, 2 * Kdim / 2048);
   return p;
 }
 
@@ -463,6 +481,188 @@ __device__ __forceinline__ void pair_dot(const uint8_t* wa, const uint8_t* wb, c
   }
 }
 
+// ---- k-quant stacks ----
+// Four unsigned bytes (codes below 2^8) widened exactly and offset by `bias`
+// (-2^23 gives the code, -(2^23 + 32) the centred Q6_K code).
+__device__ __forceinline__ void u8x4(uint32_t v, float bias, float2& lo, float2& hi) {
+  const float2 b = f2(bias, bias);
+  lo = __fadd2_rn(f2(__uint_as_float(__byte_perm(v, 0x4B000000u, 0x7650)),
+                     __uint_as_float(__byte_perm(v, 0x4B000000u, 0x7651))), b);
+  hi = __fadd2_rn(f2(__uint_as_float(__byte_perm(v, 0x4B000000u, 0x7652)),
+                     __uint_as_float(__byte_perm(v, 0x4B000000u, 0x7653))), b);
+}
+
+// Token values [p, p + 4) of a staged row (p a multiple of 4).
+template <typename AT>
+__device__ __forceinline__ void x4(uint32_t row, int p, float2& a, float2& b) {
+  if constexpr (sizeof(AT) == 4) {
+    const uint4 v = lds16(row + 16 * swz(p >> 2));
+    a = f2(__uint_as_float(v.x), __uint_as_float(v.y));
+    b = f2(__uint_as_float(v.z), __uint_as_float(v.w));
+  } else {
+    const uint2 v = lds8(row + 2 * p);
+    a = bf16x2_f2(v.x);
+    b = bf16x2_f2(v.y);
+  }
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// Scale d s_j and offset dmin m_j of sub-block j (32 values) of a Q4_K block
+// whose 16-byte head is h = {d, dmin | scales[0..3] | scales[4..7] | scales[8..11]}.
+__device__ __forceinline__ void q4k_sub(const uint4& h, int j, float& dsc, float& dm) {
+  const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu)));
+  const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x >> 16)));
+  uint32_t sc, mn;
+  if (j < 4) {
+    sc = (h.y >> (8 * j)) & 63u;
+    mn = (h.z >> (8 * j)) & 63u;
+  } else {
+    const int sh = 8 * (j - 4);
+    const uint32_t lo = h.w >> sh;
+    sc = (lo & 15u) | (((h.y >> sh) >> 6 & 3u) << 4);
+    mn = (lo >> 4 & 15u) | (((h.z >> sh) >> 6 & 3u) << 4);
+  }
+  dsc = d * static_cast<float>(sc);  // exact: 11 x 6 bits
+  dm = dmin * static_cast<float>(mn);
+}
+
+// Q4_K dot of two rows (blocks of 144 bytes read in place).  Chunk q of a
+// block holds qs bytes [16q, 16q + 16): low nibbles are values
+// 64c + 16h + [0, 16) of sub-block 2c, high nibbles values 64c + 32 + 16h +
+// [0, 16) of sub-block 2c + 1 (c = q / 2, h = q % 2).
+template <int NT, typename AT>
+__device__ __forceinline__ void q4k_pair_dot(const uint8_t* wa, const uint8_t* wb, uint32_t xs, int xrow_bytes,
+                                             int kb, int ke, float2 (&acc_a)[NT], float2 (&acc_b)[NT]) {
+  const int lane = threadIdx.x & 31;
+  const float bias = -8388608.0f;  // -2^23
+  for (int k = kb + 32 * lane; k < ke; k += 32 * 32) {
+    const int blk = k >> 8, q = (k >> 5) & 7, c2 = q >> 1;
+    const uint8_t* ba = wa + blk * 144;
+    const uint8_t* bb = wb + blk * 144;
+    const uint4 ha = ld_stream16(ba), hb = ld_stream16(bb);
+    const uint4 qa = ld_stream16(ba + 16 + 16 * q), qb = ld_stream16(bb + 16 + 16 * q);
+    float sa0, ma0, sa1, ma1, sb0, mb0, sb1, mb1;
+    q4k_sub(ha, 2 * c2, sa0, ma0);
+    q4k_sub(ha, 2 * c2 + 1, sa1, ma1);
+    q4k_sub(hb, 2 * c2, sb0, mb0);
+    q4k_sub(hb, 2 * c2 + 1, sb1, mb1);
+    const int p0 = (blk << 8) + 64 * c2 + 16 * (q & 1);
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      float2 a[4], b[4];  // [low run: 2 pairs | high run: 2 pairs]
+      const uint32_t va = word_of(qa, wi), vb = word_of(qb, wi);
+      u8x4(va & 0x0F0F0F0Fu, bias, a[0], a[1]);
+      u8x4((va >> 4) & 0x0F0F0F0Fu, bias, a[2], a[3]);
+      u8x4(vb & 0x0F0F0F0Fu, bias, b[0], b[1]);
+      u8x4((vb >> 4) & 0x0F0F0F0Fu, bias, b[2], b[3]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        a[i] = __ffma2_rn(f2(sa0, sa0), a[i], f2(-ma0, -ma0));
+        a[2 + i] = __ffma2_rn(f2(sa1, sa1), a[2 + i], f2(-ma1, -ma1));
+        b[i] = __ffma2_rn(f2(sb0, sb0), b[i], f2(-mb0, -mb0));
+        b[2 + i] = __ffma2_rn(f2(sb1, sb1), b[2 + i], f2(-mb1, -mb1));
+      }
+#pragma unroll
+      for (int c = 0; c < NT; ++c) {
+        float2 x[4];
+        x4<AT>(xs + c * xrow_bytes, p0 + 4 * wi, x[0], x[1]);
+        x4<AT>(xs + c * xrow_bytes, p0 + 32 + 4 * wi, x[2], x[3]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc_a[c] = __ffma2_rn(a[i], x[i], acc_a[c]);
+          acc_b[c] = __ffma2_rn(b[i], x[i], acc_b[c]);
+        }
+      }
+    }
+  }
+}
+
+// Q6_K dot of two rows in the split form: quant rows of 192-byte blocks
+// (ql[128] | qh[64]) and scale rows (16 int8 scales per block, then the fp16
+// d of each block).  Chunk q of a block is half n = q / 4 and l-range
+// [8m, 8m + 8) (m = q % 4): values 128n + 32i + 8m + [0, 8), i = 0..3, with
+// low bits from ql[64n + 8m + 32 (i & 1)] (low nibbles for i < 2, high for
+// i >= 2), high bits (qh[32n + 8m] >> 2i) & 3, scale sc[8n + 2i + m / 2].
+template <int NT, typename AT>
+__device__ __forceinline__ void q6k_pair_dot(const uint8_t* wa, const uint8_t* wb, const uint8_t* sa,
+                                             const uint8_t* sb, int Kdim, uint32_t xs, int xrow_bytes, int kb, int ke,
+                                             float2 (&acc_a)[NT], float2 (&acc_b)[NT]) {
+  const int lane = threadIdx.x & 31;
+  const int nb = Kdim >> 8;
+  const float bias = -8388640.0f;  // -(2^23 + 32)
+  for (int k = kb + 32 * lane; k < ke; k += 32 * 32) {
+    const int blk = k >> 8, q = (k >> 5) & 7, n = q >> 2, m = q & 3;
+    const uint8_t* ba = wa + blk * 192 + 64 * n + 8 * m;
+    const uint8_t* bb = wb + blk * 192 + 64 * n + 8 * m;
+    const uint2 la = ld_stream8(ba), ha = ld_stream8(ba + 32), qa = ld_stream8(ba + 128 - 32 * n);
+    const uint2 lb = ld_stream8(bb), hb = ld_stream8(bb + 32), qb = ld_stream8(bb + 128 - 32 * n);
+    const uint2 sca = ld_stream8(sa + 16 * blk + 8 * n), scb = ld_stream8(sb + 16 * blk + 8 * n);
+    const float da = __half2float(__ushort_as_half(ld_stream2(sa + 16 * nb + 2 * blk)));
+    const float db = __half2float(__ushort_as_half(ld_stream2(sb + 16 * nb + 2 * blk)));
+    float dsa[4], dsb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int bi = 2 * i + (m >> 1);  // scale byte within sc[8n .. 8n + 8)
+      const uint32_t wsa = bi < 4 ? sca.x : sca.y, wsb = bi < 4 ? scb.x : scb.y;
+      dsa[i] = da * static_cast<float>(static_cast<int8_t>((wsa >> (8 * (bi & 3))) & 0xFFu));  // exact: 11 x 8 bits
+      dsb[i] = db * static_cast<float>(static_cast<int8_t>((wsb >> (8 * (bi & 3))) & 0xFFu));
+    }
+    const int p0 = (blk << 8) + 128 * n + 8 * m;
+#pragma unroll
+    for (int wi = 0; wi < 2; ++wi) {
+      const uint32_t L_a = wi ? la.y : la.x, H_a = wi ? ha.y : ha.x, Q_a = wi ? qa.y : qa.x;
+      const uint32_t L_b = wi ? lb.y : lb.x, H_b = wi ? hb.y : hb.x, Q_b = wi ? qb.y : qb.x;
+      const uint32_t ca[4] = {(L_a & 0x0F0F0F0Fu) | ((Q_a << 4) & 0x30303030u),
+                              (H_a & 0x0F0F0F0Fu) | ((Q_a << 2) & 0x30303030u),
+                              ((L_a >> 4) & 0x0F0F0F0Fu) | (Q_a & 0x30303030u),
+                              ((H_a >> 4) & 0x0F0F0F0Fu) | ((Q_a >> 2) & 0x30303030u)};
+      const uint32_t cb[4] = {(L_b & 0x0F0F0F0Fu) | ((Q_b << 4) & 0x30303030u),
+                              (H_b & 0x0F0F0F0Fu) | ((Q_b << 2) & 0x30303030u),
+                              ((L_b >> 4) & 0x0F0F0F0Fu) | (Q_b & 0x30303030u),
+                              ((H_b >> 4) & 0x0F0F0F0Fu) | ((Q_b >> 2) & 0x30303030u)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 a0, a1, b0, b1;
+        u8x4(ca[i], bias, a0, a1);
+        u8x4(cb[i], bias, b0, b1);
+        a0 = __fmul2_rn(f2(dsa[i], dsa[i]), a0);
+        a1 = __fmul2_rn(f2(dsa[i], dsa[i]), a1);
+        b0 = __fmul2_rn(f2(dsb[i], dsb[i]), b0);
+        b1 = __fmul2_rn(f2(dsb[i], dsb[i]), b1);
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+          float2 x0, x1;
+          x4<AT>(xs + c * xrow_bytes, p0 + 32 * i + 4 * wi, x0, x1);
+          acc_a[c] = __ffma2_rn(a0, x0, acc_a[c]);
+          acc_a[c] = __ffma2_rn(a1, x1, acc_a[c]);
+          acc_b[c] = __ffma2_rn(b0, x0, acc_b[c]);
+          acc_b[c] = __ffma2_rn(b1, x1, acc_b[c]);
+        }
+      }
+    }
+  }
+}
+
+// Warp sums of the lane accumulators: lane c < NT receives token c's values.
+template <int NT>
+__device__ __forceinline__ void pair_reduce(const float2 (&acc_a)[NT], const float2 (&acc_b)[NT], float& va,
+                                            float& vb) {
+  const int lane = threadIdx.x & 31;
+  va = vb = 0.f;
+#pragma unroll
+  for (int c = 0; c < NT; ++c) {
+    const float sa_ = warp_sum(acc_a[c].x + acc_a[c].y);
+    const float sb_ = warp_sum(acc_b[c].x + acc_b[c].y);
+    if (lane == c) {
+      va = sa_;
+      vb = sb_;
+    }
+  }
+}
+
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -478,7 +678,7 @@ __device__ __forceinline__ void prefetch_pair(const Phase& ph, int kind, int e, 
   const int nb = DUAL ? 1 : min(2, pl.Nout - ia);  // down: rows ia, ia+1 are contiguous
   prefetch_l2(src.w0 + (row0 + ia) * pl.row_bytes, nb * pl.row_bytes);
   if (DUAL) prefetch_l2(src.w1 + (row0 + ia) * pl.row_bytes, pl.row_bytes);
-  if (WK == WK_Q8 && (pl.srow_bytes % 16) == 0) {
+  if ((WK == WK_Q8 || WK == WK_Q6K) && (pl.srow_bytes % 16) == 0) {
     prefetch_l2(src.s0 + (row0 + ia) * pl.srow_bytes, nb * pl.srow_bytes);
     if (DUAL) prefetch_l2(src.s1 + (row0 + ia) * pl.srow_bytes, pl.srow_bytes);
   }
@@ -497,10 +697,22 @@ __device__ __forceinline__ void run_unit(const Phase& ph, int kind, int e, int p
   const int ib = DUAL ? pi : min(2 * pi + 1, pl.Nout - 1);
   const uint8_t* wa = src.w0 + (row0 + ia) * pl.row_bytes;
   const uint8_t* wb = (DUAL ? src.w1 : src.w0) + (row0 + ib) * pl.row_bytes;
-  const uint8_t* sa = WK == WK_Q8 ? src.s0 + (row0 + ia) * pl.srow_bytes : nullptr;
-  const uint8_t* sb = WK == WK_Q8 ? (DUAL ? src.s1 : src.s0) + (row0 + ib) * pl.srow_bytes : nullptr;
+  constexpr bool scaled = WK == WK_Q8 || WK == WK_Q6K;  // weights with a scale plane
+  const uint8_t* sa = scaled ? src.s0 + (row0 + ia) * pl.srow_bytes : nullptr;
+  const uint8_t* sb = scaled ? (DUAL ? src.s1 : src.s0) + (row0 + ib) * pl.srow_bytes : nullptr;
   float va, vb;
-  pair_dot<NT, WK, AT>(wa, wb, sa, sb, smem_addr(sm.xs), pl.xrow_bytes, kb, ke, va, vb);
+  if constexpr (WK == WK_Q4K || WK == WK_Q6K) {
+    float2 acc_a[NT], acc_b[NT];
+#pragma unroll
+    for (int c = 0; c < NT; ++c) acc_a[c] = acc_b[c] = f2(0.f, 0.f);
+    if constexpr (WK == WK_Q4K)
+      q4k_pair_dot<NT, AT>(wa, wb, smem_addr(sm.xs), pl.xrow_bytes, kb, ke, acc_a, acc_b);
+    else
+      q6k_pair_dot<NT, AT>(wa, wb, sa, sb, pl.Kdim, smem_addr(sm.xs), pl.xrow_bytes, kb, ke, acc_a, acc_b);
+    pair_reduce<NT>(acc_a, acc_b, va, vb);
+  } else {
+    pair_dot<NT, WK, AT>(wa, wb, sa, sb, smem_addr(sm.xs), pl.xrow_bytes, kb, ke, va, vb);
+  }
   if (lane < NT) {
     if (part) {
       part[2 * lane] = va;

@@ -1,6 +1,6 @@
 // The weighted combine of the slot rows (plus the shared expert) and the
-// one-time split of GGML Q8_0 blocks into quant and scale planes.
-#include "kernels.h"
+// one-time splits of GGML Q8_0 and Q6_K blocks into quant and scale planes.
+#include "stream_core.cuh"
 
 namespace moe {
 
@@ -63,6 +63,37 @@ __global__ void __launch_bounds__(256) q8_0_split_kernel(const uint8_t* __restri
   }
 }
 
+// One thread per Q6_K block: ql|qh (192 bytes) to the quant plane, the 16
+// scales and the fp16 d to the block's places in its row of the scale plane;
+// the last block of a row also zeroes the row's padding.
+__global__ void __launch_bounds__(256) q6_k_split_kernel(const uint8_t* __restrict__ blocks, long long nblocks,
+                                                         int nb, int srow, uint8_t* __restrict__ q,
+                                                         uint8_t* __restrict__ scales) {
+  pdl_trigger();
+  pdl_wait();
+  for (long long b = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; b < nblocks;
+       b += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint8_t* src = blocks + b * 210;
+    uint4* dq = reinterpret_cast<uint4*>(q + b * 192);
+    for (int i = 0; i < 12; ++i) {
+      uint32_t w[4];
+      for (int j = 0; j < 4; ++j) {
+        const uint8_t* p = src + 16 * i + 4 * j;
+        w[j] = p[0] | (p[1] << 8) | (p[2] << 16) | (static_cast<uint32_t>(p[3]) << 24);
+      }
+      dq[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    const long long r = b / nb;
+    const int j = static_cast<int>(b - r * nb);
+    uint8_t* row = scales + r * srow;
+    for (int i = 0; i < 16; ++i) row[16 * j + i] = src[192 + i];
+    row[16 * nb + 2 * j] = src[208];
+    row[16 * nb + 2 * j + 1] = src[209];
+    if (j == nb - 1)
+      for (int i = 18 * nb; i < srow; ++i) row[i] = 0;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const Ctx& c, const float* y_slots, const float* y_shared, int T, int K, int H, void* out,
@@ -89,6 +120,17 @@ cudaError_t launch_q8_0_split(const Ctx& c, const void* blocks, int64_t rows, in
   KernelScope ks(c, "q8_0_split");
   return launch_kernel(c, q8_0_split_kernel, dim3(grid), dim3(256), 0, static_cast<const uint8_t*>(blocks), nb, q,
                        static_cast<uint16_t*>(scales));
+}
+
+cudaError_t launch_q6_k_split(const Ctx& c, const void* blocks, int64_t rows, int64_t cols, void* q, void* scales) {
+  const int nb = static_cast<int>(cols / 256);
+  const long long nblk = static_cast<long long>(rows) * nb;
+  if (nblk == 0) return cudaSuccess;
+  const int srow = stream::q6k_srow_bytes(static_cast<int>(cols));
+  const int grid = static_cast<int>(std::max(1LL, std::min<long long>((nblk + 255) / 256, 16LL * c.num_sms)));
+  KernelScope ks(c, "q6_k_split");
+  return launch_kernel(c, q6_k_split_kernel, dim3(grid), dim3(256), 0, static_cast<const uint8_t*>(blocks), nblk, nb,
+                       srow, static_cast<uint8_t*>(q), static_cast<uint8_t*>(scales));
 }
 
 }  // namespace moe

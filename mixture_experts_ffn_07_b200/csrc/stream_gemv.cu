@@ -88,7 +88,7 @@ cudaError_t launch_stream_gate_up(const Ctx& c, const void* x, int x_dtype, int 
   ph.K = K;
   ph.act_fn = act;
   const Launch a{offsets, offsets ? E : 1, offsets ? 0 : rows_bound};
-  const int wk = wk_of(w_dtype);
+  const int wk = wk_gate_up(w_dtype);
   // an expert owns at most one row per token: at most P / K rows
   const int max_tok = offsets ? std::max(1, rows_bound / std::max(1, K)) : rows_bound;
   ph.plan[0] = ph.plan[1] = make_plan(wk, true, H, I, x_dtype == MOE_F32 ? 4 : 2, max_tok);
@@ -96,10 +96,12 @@ cudaError_t launch_stream_gate_up(const Ctx& c, const void* x, int x_dtype, int 
   if (x_dtype == MOE_F32) {
     if (wk == WK_F32) return launch_typed<float, WK_F32, true>(c, ph, a, n);
     if (wk == WK_BF16) return launch_typed<float, WK_BF16, true>(c, ph, a, n);
+    if (wk == WK_Q4K) return launch_typed<float, WK_Q4K, true>(c, ph, a, n);
     return launch_typed<float, WK_Q8, true>(c, ph, a, n);
   }
   if (wk == WK_F32) return launch_typed<__nv_bfloat16, WK_F32, true>(c, ph, a, n);
   if (wk == WK_BF16) return launch_typed<__nv_bfloat16, WK_BF16, true>(c, ph, a, n);
+  if (wk == WK_Q4K) return launch_typed<__nv_bfloat16, WK_Q4K, true>(c, ph, a, n);
   return launch_typed<__nv_bfloat16, WK_Q8, true>(c, ph, a, n);
 }
 
@@ -119,11 +121,13 @@ cudaError_t launch_stream_down(const Ctx& c, const float* h, int I, int H, const
   ph.pairs = pairs;
   ph.K = 1;
   const Launch a{offsets, offsets ? E : 1, offsets ? 0 : rows_bound};
-  const int wk = wk_of(w_dtype);
+  const int wk = wk_down(w_dtype);
   ph.plan[0] = ph.plan[1] = make_plan(wk, false, I, H, 4, kMaxTok);
   const char* n = "stream_down";
   if (wk == WK_F32) return launch_typed<float, WK_F32, false>(c, ph, a, n);
   if (wk == WK_BF16) return launch_typed<float, WK_BF16, false>(c, ph, a, n);
+  if (wk == WK_Q4K) return launch_typed<float, WK_Q4K, false>(c, ph, a, n);
+  if (wk == WK_Q6K) return launch_typed<float, WK_Q6K, false>(c, ph, a, n);
   return launch_typed<float, WK_Q8, false>(c, ph, a, n);
 }
 

@@ -5,14 +5,16 @@ layouts include/moe.h expects, and run one call.  Argument marshalling only.
 (``spec`` with T, H, E, I, K, act, renormalize, act_dtype, w_dtype,
 router_dtype, shared_I; arrays x, router, router_bias, gate, up, down,
 sh_gate, sh_up, sh_down, sh_gate_w).  bf16 arrays are uint16 bit patterns;
-Q8_0 weights are GGML blocks and are split on the device by moe_q8_0_split.
+Q8_0 weights are GGML blocks and are split on the device by moe_q8_0_split;
+Q4_K blocks are used in place and Q6_K blocks are split by moe_q6_k_split.
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
-from . import Desc, Weights, last_device_status, layer, q8_0_split, route, workspace_bytes, MOE_OK
+from . import (Desc, Weights, last_device_status, layer, q6_k_split, q6_k_srow_bytes, q8_0_split, route,
+               workspace_bytes, MOE_OK)
 
 
 def to_device(a: np.ndarray, dtype: str) -> torch.Tensor:
@@ -28,6 +30,14 @@ def split_q8_0(blocks: np.ndarray, rows: int, cols: int):
     q = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
     s = torch.empty((rows, cols // 32), dtype=torch.float16, device="cuda")
     q8_0_split(b, rows, cols, q, s)
+    return q, s
+
+
+def split_q6_k(blocks: np.ndarray, rows: int, cols: int):
+    b = torch.from_numpy(np.ascontiguousarray(blocks).reshape(-1)).cuda()
+    q = torch.empty((rows, cols // 256, 192), dtype=torch.uint8, device="cuda")
+    s = torch.empty((rows, q6_k_srow_bytes(cols)), dtype=torch.uint8, device="cuda")
+    q6_k_split(b, rows, cols, q, s)
     return q, s
 
 
@@ -52,6 +62,12 @@ def upload(src):
             q, sc = split_q8_0(a, rows, cols)
             setattr(w, name, q)
             setattr(w, name + "_scale", sc)
+        elif s.w_dtype == "q4_k_q6_k" and name in ("down", "sh_down"):
+            q, sc = split_q6_k(a, rows, cols)
+            setattr(w, name, q)
+            setattr(w, name + "_scale", sc)
+        elif s.w_dtype in ("q4_k", "q4_k_q6_k"):
+            setattr(w, name, torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda())
         else:
             setattr(w, name, to_device(a, s.w_dtype))
     x = to_device(src.x, s.act_dtype)

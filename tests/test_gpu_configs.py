@@ -1,4 +1,4 @@
-"""GPU parity at the five measured workloads' full sizes, in the launch
+"""GPU parity at the measured workloads' full sizes, in the launch
 configuration the benchmark times (one moe_layer call).
 
 The oracle cannot redo a whole 8192-token layer in f64 in seconds, so the
@@ -20,7 +20,7 @@ import workloads  # noqa: E402
 from tests import _gpu  # noqa: E402
 
 SAMPLE = {"decode_f32_t1": 1, "prefill_bf16_t512": 48, "routed_shared_t4096": 24, "skewed_zipf_t8192": 8,
-          "q8_0_decode_t16": 16, "grouped_sigmoid_t512": 32}
+          "q8_0_decode_t16": 16, "grouped_sigmoid_t512": 32, "q4k_q6k_decode_t16": 16}
 
 
 @pytest.mark.parametrize("name", workloads.CONFIG_ORDER)
