@@ -11,7 +11,9 @@
 // Design (sm_100a):
 //  * persistent grid, one CTA per SM; work items (group, n-tile, m-tile) with
 //    the m-tile fastest so CTAs running at the same time share weight tiles
-//    in L2;
+//    in L2; in single mode, for memory-bound groups of more than one row tile,
+//    an item covers two row tiles against one weight tile (two accumulators),
+//    so each weight tile is loaded once per group;
 //  * warp 0: TMA producer (one lane) into a shared-memory ring of 128x64 A
 //    tiles and BNx64 B tiles, 128-byte swizzle (6 stages at BN = 128, 4 at 256);
 //  * warp 1: allocates 2*BN TMEM columns and issues tcgen05.mma (M=128, N=BN,
@@ -41,14 +43,16 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int MAX_G = 256;
 constexpr int THREADS = 192;
 
-// Tile shape per instantiation: the MMA is M=128 x N=BN; the ring holds STAGES
-// (A 128x64, B BNx64) stage pairs, ~192 KB either way.
-template <int BN>
+// Tile shape per instantiation: the MMA is M=128 x N=BN; an item covers MT
+// (1 or 2) row tiles of one group against the same BN weight rows, so a stage
+// holds MT A tiles (128x64) and one B tile (BNx64); ~192 KB of stages either way.
+template <int BN, int MT>
 struct Tile {
-  static constexpr int STAGES = BN == 128 ? 6 : 4;
+  static_assert(MT == 1 || BN == 128, "two row tiles per item need 4*BN <= 512 TMEM columns");
+  static constexpr int STAGES = MT == 2 ? 4 : (BN == 128 ? 6 : 4);
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+  static constexpr int STAGE_BYTES = MT * A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * MT * BN;  // two accumulator sets of MT tiles
 };
 
 template <int STAGES>
@@ -65,9 +69,10 @@ struct Aux {
   int cnt[MAX_G];
 };
 
-template <int BN>
+template <int BN, int MT>
 constexpr size_t smem_bytes() {
-  return 1024 + static_cast<size_t>(Tile<BN>::STAGES) * Tile<BN>::STAGE_BYTES + sizeof(Aux<Tile<BN>::STAGES>);
+  return 1024 + static_cast<size_t>(Tile<BN, MT>::STAGES) * Tile<BN, MT>::STAGE_BYTES +
+         sizeof(Aux<Tile<BN, MT>::STAGES>);
 }
 
 struct KParams {
@@ -99,9 +104,11 @@ __device__ __forceinline__ bool wait_cycles(uint64_t* bar, uint32_t parity, long
   return true;
 }
 
-template <typename AuxT>
-__device__ __forceinline__ void decode_item(const AuxT& aux, int G, int ksplit, int w, int& g, int& mt, int& nt,
-                                            int& ks) {
+// Item w -> group g, first row tile mt and the number nm (1..MT) of row tiles
+// it covers, column tile nt, K range ks.
+template <int MT, typename AuxT>
+__device__ __forceinline__ void decode_item(const AuxT& aux, int G, int ksplit, int w, int& g, int& mt, int& nm,
+                                            int& nt, int& ks) {
   int lo = 0, hi = G - 1;  // largest g with item_off[g] <= w
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -112,11 +119,13 @@ __device__ __forceinline__ void decode_item(const AuxT& aux, int G, int ksplit, 
   }
   g = lo;
   const int tiles = (aux.cnt[g] + BM - 1) / BM;
+  const int mitems = (tiles + MT - 1) / MT;
   const int local = w - aux.item_off[g];
   ks = local % ksplit;
   const int rest = local / ksplit;
-  nt = rest / tiles;
-  mt = rest - nt * tiles;
+  nt = rest / mitems;
+  mt = (rest - nt * mitems) * MT;
+  nm = min(MT, tiles - mt);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -124,14 +133,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <bool DUAL, int BN>
+template <bool DUAL, int BN, int MT>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                         const __grid_constant__ CUtensorMap mapB1, const KParams p) {
-  constexpr int STAGES = Tile<BN>::STAGES;
-  constexpr int STAGE_BYTES = Tile<BN>::STAGE_BYTES;
-  constexpr int B_BYTES = Tile<BN>::B_BYTES;
-  constexpr uint32_t TMEM_COLS = Tile<BN>::TMEM_COLS;
+  constexpr int STAGES = Tile<BN, MT>::STAGES;
+  constexpr int STAGE_BYTES = Tile<BN, MT>::STAGE_BYTES;
+  constexpr int B_BYTES = Tile<BN, MT>::B_BYTES;
+  constexpr uint32_t TMEM_COLS = Tile<BN, MT>::TMEM_COLS;
   constexpr int BN_MMA = BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -175,7 +184,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int g = lane * 8 + i;
-      v[i] = g < p.G ? ((aux.cnt[g] + BM - 1) / BM) * p.n_tiles * p.ksplit : 0;
+      v[i] = g < p.G ? ((aux.cnt[g] + MT * BM - 1) / (MT * BM)) * p.n_tiles * p.ksplit : 0;
       local += v[i];
     }
     int incl = local;
@@ -210,10 +219,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint64_t pol_w = l2_policy_evict_first();  // weights of a group with one row tile: read once
       const uint64_t pol_a = l2_policy_evict_last();   // activation rows: read by every column tile
       for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
-        int g, mt, nt, ks;
-        decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
+        int g, mt, nm, nt, ks;
+        decode_item<MT>(aux, p.G, p.ksplit, w, g, mt, nm, nt, ks);
         const int a_row = aux.row_off[g] + mt * BM;
-        const bool one_mtile = aux.cnt[g] <= BM;
+        const bool one_mtile = aux.cnt[g] <= MT * BM;  // this item covers every row tile of the group
         const int b_row = g * p.N + nt * p.col_step;
         const int kb0 = ks * p.kb_per_split, kb1 = min(nkb, kb0 + p.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
@@ -226,9 +235,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             continue;
           }
           uint8_t* sa = smem + s * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(&aux.full[s], STAGE_BYTES);
-          tma_load_2d_hint(sa, &mapA, &aux.full[s], kb * BK, a_row, pol_a);
+          uint8_t* sb = sa + MT * A_BYTES;
+          mbar_arrive_expect_tx(&aux.full[s], nm * A_BYTES + B_BYTES);
+          for (int j = 0; j < nm; ++j)
+            tma_load_2d_hint(sa + j * A_BYTES, &mapA, &aux.full[s], kb * BK, a_row + j * BM, pol_a);
           if (one_mtile) {  // the weight tile is not needed again
             tma_load_2d_hint(sb, &mapB0, &aux.full[s], kb * BK, b_row, pol_w);
             if (DUAL) tma_load_2d_hint(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row, pol_w);
@@ -252,14 +262,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t kbg = 0;
       int it = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-        int g, mt, nt, ks;
-        decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
+        int g, mt, nm, nt, ks;
+        decode_item<MT>(aux, p.G, p.ksplit, w, g, mt, nm, nt, ks);
         const int kb0 = ks * p.kb_per_split, kb1 = min(nkb, kb0 + p.kb_per_split);
         const int acc = it & 1;
         const uint32_t acc_ph = (it >> 1) & 1u;
         if (!mbar_wait_bounded(&aux.tempty[acc], acc_ph ^ 1u, limit, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN_MMA;
+        const uint32_t d_tmem = tmem_base + acc * MT * BN_MMA;  // row tile j accumulates at + j * BN
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
           const int s = kbg % STAGES;
@@ -270,12 +280,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = smem_addr(smem + s * STAGE_BYTES);
-          const uint64_t adesc = sw128_kmajor_desc(a_addr);
-          const uint64_t bdesc = sw128_kmajor_desc(a_addr + A_BYTES);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + MT * A_BYTES);
+          for (int j = 0; j < nm; ++j) {
+            const uint64_t adesc = sw128_kmajor_desc(a_addr + j * A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                      (kb > kb0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_bf16(d_tmem + j * BN_MMA, adesc + static_cast<uint64_t>(kk * 2),
+                        bdesc + static_cast<uint64_t>(kk * 2), idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
           umma_commit(&aux.empty[s]);
         }
         if (!ok) break;
@@ -290,18 +302,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int r = q * 32 + lane;
     int it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-      int g, mt, nt, ks;
-      decode_item(aux, p.G, p.ksplit, w, g, mt, nt, ks);
+      int g, mt0, nm, nt, ks;
+      decode_item<MT>(aux, p.G, p.ksplit, w, g, mt0, nm, nt, ks);
       const int acc = it & 1;
       const uint32_t acc_ph = (it >> 1) & 1u;
       // every lane waits; the outcome is made warp-uniform because the TMEM loads below are .sync.aligned
       const bool ok = mbar_wait_bounded(&aux.tfull[acc], acc_ph, limit, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      for (int j = 0; j < nm; ++j) {
+      const int mt = mt0 + j;
       const int rows_valid = min(BM, aux.cnt[g] - mt * BM);
       const int a_row = aux.row_off[g] + mt * BM;
       const int col0 = nt * p.col_step;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN_MMA;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc * MT + j) * BN_MMA;
       if (DUAL) {
         for (int c = 0; c < BN_MMA / 2; c += 32) {
           uint32_t gr[32], ur[32];
@@ -311,20 +325,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (r < rows_valid && col0 + c < p.N) {
             uint32_t packed[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float h0 = act_fn(p.act, __uint_as_float(gr[2 * j])) * __uint_as_float(ur[2 * j]);
-              const float h1 = act_fn(p.act, __uint_as_float(gr[2 * j + 1])) * __uint_as_float(ur[2 * j + 1]);
-              packed[j] = pack_bf16x2(h0, h1);
+            for (int jj = 0; jj < 16; ++jj) {
+              const float h0 = act_fn(p.act, __uint_as_float(gr[2 * jj])) * __uint_as_float(ur[2 * jj]);
+              const float h1 = act_fn(p.act, __uint_as_float(gr[2 * jj + 1])) * __uint_as_float(ur[2 * jj + 1]);
+              packed[jj] = pack_bf16x2(h0, h1);
             }
             __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(a_row + r) * p.N + col0 + c;
             if (col0 + c + 32 <= p.N) {
               uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+              for (int jj = 0; jj < 4; ++jj)
+                d4[jj] = make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]);
             } else {
               const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(packed);
-              for (int j = 0; j < 32 && col0 + c + j < p.N; ++j) dst[j] = hv[j];
+              for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj) dst[jj] = hv[jj];
             }
           }
         }
@@ -345,15 +359,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (col0 + c + 32 <= p.N) {
               float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                d4[j] = make_float4(scale * __uint_as_float(v[4 * j]), scale * __uint_as_float(v[4 * j + 1]),
-                                    scale * __uint_as_float(v[4 * j + 2]), scale * __uint_as_float(v[4 * j + 3]));
+              for (int jj = 0; jj < 8; ++jj)
+                d4[jj] = make_float4(scale * __uint_as_float(v[4 * jj]), scale * __uint_as_float(v[4 * jj + 1]),
+                                     scale * __uint_as_float(v[4 * jj + 2]), scale * __uint_as_float(v[4 * jj + 3]));
             } else {
-              for (int j = 0; j < 32 && col0 + c + j < p.N; ++j) dst[j] = scale * __uint_as_float(v[j]);
+              for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj) dst[jj] = scale * __uint_as_float(v[jj]);
             }
           }
         }
       }
+      }  // row tiles of the item
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&aux.tempty[acc]);
@@ -399,7 +414,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool DUAL, int BN>
+template <bool DUAL, int BN, int MT>
 cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int max_items_per_sm_hint) {
   (void)max_items_per_sm_hint;
   CUtensorMap mA, mB0, mB1;
@@ -436,11 +451,12 @@ cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int max_items_per_sm_h
   const long long tiles_bound = static_cast<long long>(a.max_rows) / BM + std::min(a.G, a.max_rows);
   const long long items_bound = tiles_bound * p.n_tiles * p.ksplit;
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(c.num_sms, items_bound)));
-  auto kern = grouped_gemm_kernel<DUAL, BN>;
-  const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem_bytes<BN>()));
+  auto kern = grouped_gemm_kernel<DUAL, BN, MT>;
+  const cudaError_t e =
+      allow_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem_bytes<BN, MT>()));
   if (e != cudaSuccess) return e;
   KernelScope ks(c, a.name ? a.name : (DUAL ? "grouped_gemm_dual" : "grouped_gemm"));
-  return launch_kernel(c, kern, dim3(grid), dim3(THREADS), smem_bytes<BN>(), mA, mB0, mB1, p);
+  return launch_kernel(c, kern, dim3(grid), dim3(THREADS), smem_bytes<BN, MT>(), mA, mB0, mB1, p);
 }
 
 }  // namespace
@@ -467,10 +483,15 @@ cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   const double items_narrow = tiles * std::ceil(a.N / (cols_wide / 2));
   // weights are streamed once per group; rows per group sets flops per weight byte (ridge ~200)
   const bool memory_bound = rows_per_group < 200.0;
+  // single mode (the down projection: short K) with memory-bound groups that often span two row tiles: narrow
+  // tiles covering two row tiles per item, so each item is twice as long and each weight tile is loaded once per
+  // group.  The gate/up projection keeps one row tile per item: its long K rows already share weight tiles
+  // through L2 between the CTAs running a group's row tiles side by side, and it keeps 6 stages.
+  if (!a.dual && memory_bound && rows_per_group > 96.0) return launch_tiled<false, 128, 2>(c, a, 0);
   const bool narrow =
       memory_bound && wave_waste(items_wide, c.num_sms) - wave_waste(items_narrow, c.num_sms) > 0.03;
-  if (a.dual) return narrow ? launch_tiled<true, 128>(c, a, 0) : launch_tiled<true, 256>(c, a, 0);
-  return narrow ? launch_tiled<false, 128>(c, a, 0) : launch_tiled<false, 256>(c, a, 0);
+  if (a.dual) return narrow ? launch_tiled<true, 128, 1>(c, a, 0) : launch_tiled<true, 256, 1>(c, a, 0);
+  return narrow ? launch_tiled<false, 128, 1>(c, a, 0) : launch_tiled<false, 256, 1>(c, a, 0);
 }
 
 }  // namespace moe

@@ -11,7 +11,8 @@
 //      moe_route's bit for bit); the CTA counts its pairs per expert and
 //      publishes the counts in hist[c][*];                         -- barrier
 //   B  every CTA adds the published counts (totals, and the counts of the
-//      CTAs before it), scans them into expert offsets, places its own pairs
+//      CTAs before it; J = 512 / E threads per expert, register sums over a
+//      fixed subset of CTAs each, no atomics), scans them into expert offsets, places its own pairs
 //      in pair order (a stable counting sort, so the permutation is unique),
 //      writes sorted_pairs / pair_pos and copies each pair's x row into its
 //      place in x_perm.
@@ -55,6 +56,7 @@ struct FrontArgs {
 };
 
 __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
+  extern __shared__ __align__(16) uint8_t fsmem[];  // [16 warps][256] f32 logit rows, then [2][512] count partials
   __shared__ int s_hist[256], s_run[256], s_tot[256], s_off[257];
   __shared__ int s_abort, s_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -70,7 +72,8 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
   // ---- A: selection of this CTA's tokens, and its pair counts
   for (int t = t0 + warp; t < t1; t += kWarps)
     topk_token<__nv_bfloat16, __nv_bfloat16>(a.parts, a.nparts, a.part_stride, a.logits, a.bias, a.rc, a.ids, a.w,
-                                             a.x, a.w_s, a.H, a.shared_gate, t);
+                                             a.x, a.w_s, a.H, a.shared_gate, t,
+                                             reinterpret_cast<float*>(fsmem) + warp * 256);
   __syncthreads();
   for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&s_hist[a.ids[p]], 1);
   __syncthreads();
@@ -82,27 +85,39 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
   }
 
   // ---- B: offsets, this CTA's pair positions and rows
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_run[e] = 0;
-  __syncthreads();
-  {  // totals and the counts of the CTAs before this one: all G x E counts requested 8 at a time
-    const int n = G * E;
-#pragma unroll 1
-    for (int i0 = threadIdx.x; i0 < n; i0 += blockDim.x * 8) {
-      int v[8];
+  {  // totals and the counts of the CTAs before this one: J = 512 / E threads per expert, each summing the
+     // counts of CTAs j, j + J, ... in registers (16 loads in flight), then a fixed-order sum over j
+    int* red_tot = reinterpret_cast<int*>(fsmem + kWarps * 256 * 4);
+    int* red_run = red_tot + kThreads;
+    const int J = kThreads / E;
+    if (threadIdx.x < J * E) {
+      const int e = threadIdx.x % E, j = threadIdx.x / E;
+      int tot = 0, run = 0;
+      for (int c0 = j; c0 < G; c0 += 16 * J) {
+        int v[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = i0 + j * blockDim.x;
-        v[j] = i < n ? __ldcg(a.hist + i) : 0;
-      }
+        for (int q = 0; q < 16; ++q) {
+          const int cc = c0 + q * J;
+          v[q] = cc < G ? __ldcg(a.hist + static_cast<size_t>(cc) * E + e) : 0;
+        }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = i0 + j * blockDim.x;
-        if (i < n && v[j]) {
-          const int cc = i / E, e = i - cc * E;
-          atomicAdd(&s_tot[e], v[j]);
-          if (cc < c) atomicAdd(&s_run[e], v[j]);
+        for (int q = 0; q < 16; ++q) {
+          tot += v[q];
+          if (c0 + q * J < c) run += v[q];
         }
       }
+      red_tot[j * E + e] = tot;
+      red_run[j * E + e] = run;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int tot = 0, run = 0;
+      for (int j = 0; j < J; ++j) {
+        tot += red_tot[j * E + e];
+        run += red_run[j * E + e];
+      }
+      s_tot[e] = tot;
+      s_run[e] = run;
     }
   }
   __syncthreads();
@@ -205,8 +220,9 @@ cudaError_t launch_prefill_front(const Ctx& c, const PrefillFront& f) {
   a.hist = f.hist;
   a.status = c.status;
   a.wait_limit = c.wait_limit;
-  // more than half of an SM's shared memory: one CTA per SM, one such grid per device
-  const int smem = c.smem_optin / 2 + 1024;
+  // more than half of an SM's shared memory: one CTA per SM, one such grid per device (and room for the
+  // warps' logit rows and the count partials)
+  const int smem = std::max(c.smem_optin / 2 + 1024, kWarps * 256 * 4 + 2 * kThreads * 4);
   const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(front_kernel), smem);
   if (e != cudaSuccess) return e;
   KernelScope ks(c, "route_permute_gather");

@@ -48,34 +48,17 @@ __device__ __forceinline__ void raw_decode(const Raw8<__nv_bfloat16>& r, float (
   }
 }
 
-// Top-K (+ renormalisation) of one token, by one warp.  `row` holds the E raw
-// logits (global or shared memory); the biased logits go to logits_out.  With
-// n_groups > 1 the experts form n_groups contiguous groups, a group scores its
-// largest logit, and only the topk_groups best groups (lower index on ties)
-// are eligible.  Weights: softmax gate values over all E experts, or sigmoid
-// gate values; renormalised over the K selected when asked.
-__device__ __forceinline__ void warp_topk(const float* row, const float* __restrict__ bias, const RouteCfg& rc,
-                                          float* __restrict__ logits_out, int32_t* __restrict__ ids,
-                                          float* __restrict__ wout) {
+// Top-K (+ renormalisation) of one token, by one warp, from the lane's biased
+// logits v[i] of experts e = lane + 32 i (NaN already mapped to -inf; entries
+// beyond E are -inf) and m, their maximum over the warp.  With n_groups > 1 the
+// experts form n_groups contiguous groups, a group scores its largest logit,
+// and only the topk_groups best groups (lower index on ties) are eligible.
+// Weights: softmax gate values over all E experts, or sigmoid gate values;
+// renormalised over the K selected when asked.
+__device__ __forceinline__ void warp_select(const float (&v)[8], float m, const RouteCfg& rc,
+                                            int32_t* __restrict__ ids, float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
   const int E = rc.E, K = rc.K;
-  float v[8];
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = -INFINITY;
-    if (e < E) {
-      float l = row[e];
-      if (bias) l += bias[e];
-      logits_out[e] = l;
-      v[i] = l == l ? l : -INFINITY;  // a NaN logit ranks last, so K valid experts are always chosen
-      m = fmaxf(m, l);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-
   uint32_t taken = 0;  // bit i: v[i] chosen, or not eligible
   if (rc.n_groups > 1) {
     const int gs = E / rc.n_groups;
@@ -164,37 +147,88 @@ __device__ __forceinline__ void warp_topk(const float* row, const float* __restr
   }
 }
 
+// warp_select on the E raw logits of `row` (global or shared memory) plus the
+// bias; the biased logits go to logits_out (a different array than row).
+__device__ __forceinline__ void warp_topk(const float* __restrict__ row, const float* __restrict__ bias,
+                                          const RouteCfg& rc, float* __restrict__ logits_out,
+                                          int32_t* __restrict__ ids, float* __restrict__ wout) {
+  const int lane = threadIdx.x & 31;
+  float v[8];
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = -INFINITY;
+    if (e < rc.E) {
+      float l = row[e];
+      if (bias) l += bias[e];
+      logits_out[e] = l;
+      v[i] = l == l ? l : -INFINITY;  // a NaN logit ranks last, so K valid experts are always chosen
+      m = fmaxf(m, l);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  warp_select(v, m, rc, ids, wout);
+}
+
+// srow[e] = the sum of the `nparts` (<= 16 / EP) split-K partial logits of
+// expert e of token t (T*E floats each, `stride` apart), added in part order.
+// A lane takes EP of its experts per round, all their parts requested together.
+template <int EP>
+__device__ __forceinline__ void sum_parts(const float* __restrict__ parts, int nparts, size_t stride, int E, int t,
+                                          float* srow) {
+  constexpr int KP = 16 / EP;
+  const int lane = threadIdx.x & 31;
+  const float* src = parts + static_cast<size_t>(t) * E;
+  for (int e0 = lane; e0 < E; e0 += 32 * EP) {
+    float r[EP][KP];
+#pragma unroll
+    for (int q = 0; q < EP; ++q)
+#pragma unroll
+      for (int k = 0; k < KP; ++k)
+        r[q][k] = (e0 + 32 * q < E && k < nparts) ? src[e0 + 32 * q + k * stride] : 0.f;
+#pragma unroll
+    for (int q = 0; q < EP; ++q) {
+      if (e0 + 32 * q < E) {
+        float sum = r[q][0];
+#pragma unroll
+        for (int k = 1; k < KP; ++k)
+          if (k < nparts) sum += r[q][k];
+        srow[e0 + 32 * q] = sum;
+      }
+    }
+  }
+}
 
 // Selection for token t by one warp, from logits in global memory: `nparts`
-// (<= 16) partial logit arrays of T*E floats, part_stride apart starting at `parts`,
-// are first added in order into logits[t] (nparts == 0: logits[t] already
-// holds them); then warp_topk with the bias in place.  With w_s the warp also
-// writes shared_gate[t] = sigmoid(w_s . x[t]) (lane l accumulates elements
-// 8l + 256u + q in order; warp_sum).
+// (<= 16) partial logit arrays of T*E floats, part_stride apart starting at
+// `parts`, are added in order into `srow`, the warp's row of E floats in
+// shared memory (nparts == 0: logits[t] already holds the sums and is copied
+// there); warp_topk then writes the biased logits to logits[t].  With w_s the warp also writes shared_gate[t] = sigmoid(w_s . x[t])
+// (lane l accumulates elements 8l + 256u + q in order; warp_sum).
 template <typename XT, typename WT>
 __device__ __forceinline__ void topk_token(const float* parts, int nparts, size_t part_stride, float* logits,
                                            const float* bias, const RouteCfg& rc, int32_t* ids, float* wout,
-                                           const XT* x, const WT* w_s, int H, float* shared_gate, int t) {
-  constexpr int kUnroll = 8;
+                                           const XT* x, const WT* w_s, int H, float* shared_gate, int t,
+                                           float* srow) {
+  constexpr int kUnroll = 4;
   const int lane = threadIdx.x & 31;
   const int E = rc.E, K = rc.K;
   float* row = logits + static_cast<size_t>(t) * E;
-  if (nparts > 0) {  // all partials of an expert requested together, then added in range order
-    constexpr int kMaxParts = 16;
-    for (int e = lane; e < E; e += 32) {
-      const float* src = parts + static_cast<size_t>(t) * E + e;
-      float v[kMaxParts];
-#pragma unroll
-      for (int k = 0; k < kMaxParts; ++k) v[k] = k < nparts ? src[k * part_stride] : 0.f;
-      float sum = v[0];
-#pragma unroll
-      for (int k = 1; k < kMaxParts; ++k)
-        if (k < nparts) sum += v[k];
-      row[e] = sum;
-    }
-    __syncwarp();
+  if (nparts > 0) {
+    if (nparts <= 4)
+      sum_parts<4>(parts, nparts, part_stride, E, t, srow);
+    else if (nparts <= 8)
+      sum_parts<2>(parts, nparts, part_stride, E, t, srow);
+    else
+      sum_parts<1>(parts, nparts, part_stride, E, t, srow);
+  } else {
+    for (int e = lane; e < E; e += 32) srow[e] = row[e];
   }
-  warp_topk(row, bias, rc, row, ids + static_cast<size_t>(t) * K, wout + static_cast<size_t>(t) * K);
+  __syncwarp();
+  warp_topk(srow, bias, rc, row, ids + static_cast<size_t>(t) * K, wout + static_cast<size_t>(t) * K);
+  __syncwarp();
   if (w_s) {
     const XT* xr = x + static_cast<size_t>(t) * H;
     float acc = 0.f;

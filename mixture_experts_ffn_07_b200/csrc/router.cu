@@ -155,13 +155,13 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           float* __restrict__ wout, const XT* __restrict__ x,
                                                           const WT* __restrict__ w_s, int H,
                                                           float* __restrict__ shared_gate) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float s_row[8][256];  // one logit row per warp
+  const int warp = threadIdx.x >> 5;
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;
-  (void)lane;
-  topk_token(parts, nparts, part_stride, logits, bias, rc, ids, wout, x, w_s, H, shared_gate, t);
+  topk_token(parts, nparts, part_stride, logits, bias, rc, ids, wout, x, w_s, H, shared_gate, t, s_row[warp]);
 }
 
 template <typename XT, typename WT>

@@ -6,31 +6,41 @@ namespace moe {
 
 namespace {
 
-template <typename OT>
+// One thread per (token, float4 column) item, grid-stride; IT is the index
+// type (32-bit whenever the item count allows, which keeps the row division cheap).
+template <typename OT, typename IT>
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y_slots,
                                                       const float4* __restrict__ y_shared, int T, int K, int H4,
                                                       OT* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
-  const long long total = static_cast<long long>(T) * H4;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long t = idx / H4;
-    const int c = static_cast<int>(idx - t * H4);
-    float4 acc = __ldg(y_slots + (t * K) * H4 + c);
-    for (int k = 1; k < K; ++k) {
-      const float4 v = __ldg(y_slots + (t * K + k) * H4 + c);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+  const IT total = static_cast<IT>(T) * H4;
+  for (IT idx = static_cast<IT>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<IT>(gridDim.x) * blockDim.x) {
+    const IT t = idx / H4;
+    const IT c = idx - t * H4;
+    const float4* ys = y_slots + (t * K) * H4 + c;
+    float4 v[8];
+    float4 acc = __ldg(ys);
+    for (int k0 = 1; k0 < K; k0 += 8) {  // up to eight slot rows in flight, added in k order
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (k0 + j < K) v[j] = __ldg(ys + static_cast<IT>(k0 + j) * H4);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (k0 + j < K) {
+          acc.x += v[j].x;
+          acc.y += v[j].y;
+          acc.z += v[j].z;
+          acc.w += v[j].w;
+        }
     }
     if (y_shared) {
-      const float4 v = __ldg(y_shared + t * H4 + c);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+      const float4 w = __ldg(y_shared + t * H4 + c);
+      acc.x += w.x;
+      acc.y += w.y;
+      acc.z += w.z;
+      acc.w += w.w;
     }
     if constexpr (sizeof(OT) == 4) {
       reinterpret_cast<float4*>(out)[idx] = acc;
@@ -96,20 +106,29 @@ __global__ void __launch_bounds__(256) q6_k_split_kernel(const uint8_t* __restri
 
 }  // namespace
 
+template <typename OT, typename IT>
+cudaError_t combine_typed(const Ctx& c, const float* y_slots, const float* y_shared, int T, int K, int H4, void* out) {
+  auto kern = combine_kernel<OT, IT>;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+  const long long total = static_cast<long long>(T) * H4;
+  const int blocks = static_cast<int>(std::max(1LL, std::min<long long>((total + 255) / 256, 1LL * per_sm * c.num_sms)));
+  return launch_kernel(c, kern, dim3(blocks), dim3(256), 0, reinterpret_cast<const float4*>(y_slots),
+                       reinterpret_cast<const float4*>(y_shared), T, K, H4, static_cast<OT*>(out));
+}
+
 cudaError_t launch_combine(const Ctx& c, const float* y_slots, const float* y_shared, int T, int K, int H, void* out,
                            int out_dtype) {
   if (T == 0) return cudaSuccess;
   const int H4 = H / 4;
-  const long long total = static_cast<long long>(T) * H4;
-  const int blocks = static_cast<int>(std::max(1LL, std::min<long long>((total + 255) / 256, 16LL * c.num_sms)));
+  // 32-bit indices while every slot row offset fits
+  const bool narrow = static_cast<long long>(T) * K * H4 < (1LL << 31) - 256LL * 1024 * 148;
   KernelScope ks(c, "combine");
   if (out_dtype == MOE_F32)
-    return launch_kernel(c, combine_kernel<float>, dim3(blocks), dim3(256), 0,
-                         reinterpret_cast<const float4*>(y_slots), reinterpret_cast<const float4*>(y_shared), T, K,
-                         H4, static_cast<float*>(out));
-  return launch_kernel(c, combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0,
-                       reinterpret_cast<const float4*>(y_slots), reinterpret_cast<const float4*>(y_shared), T, K, H4,
-                       static_cast<__nv_bfloat16*>(out));
+    return narrow ? combine_typed<float, int>(c, y_slots, y_shared, T, K, H4, out)
+                  : combine_typed<float, long long>(c, y_slots, y_shared, T, K, H4, out);
+  return narrow ? combine_typed<__nv_bfloat16, int>(c, y_slots, y_shared, T, K, H4, out)
+                : combine_typed<__nv_bfloat16, long long>(c, y_slots, y_shared, T, K, H4, out);
 }
 
 cudaError_t launch_q8_0_split(const Ctx& c, const void* blocks, int64_t rows, int64_t cols, int8_t* q,

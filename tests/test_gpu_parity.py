@@ -124,6 +124,7 @@ def test_permute_reports_out_of_range_ids():
 FFN_CASES = {
     "tensor_ragged": spec(200, 256, 16, 160, 4),
     "tensor_multi_mtile": spec(300, 384, 8, 128, 2),
+    "tensor_two_row_tiles_per_item": spec(520, 384, 8, 128, 2),
     "stream_f32_gelu": spec(6, 256, 16, 96, 4, act="gelu_tanh", dt="f32"),
     "stream_bf16": spec(40, 256, 32, 128, 8),
     "stream_q8": spec(16, 256, 32, 128, 8, dt="f32", w_dt="q8_0", r_dt="f32"),
@@ -175,6 +176,11 @@ LAYER_CASES = {
     "no_renorm_gelu_tensor": (spec(150, 256, 32, 96, 4, act="gelu_tanh", renorm=False), {}),
     "K_equals_E_stream": (spec(3, 128, 4, 64, 4, dt="f32"), {}),
     "stream_f32_wide_H_token_batches": (spec(20, 4096, 4, 64, 2, dt="f32", shared=32), {}),
+    # more than 96 rows per expert: items of two row tiles against one weight tile
+    "tensor_bf16_two_row_tiles": (spec(700, 256, 8, 128, 2), {}),
+    "tensor_bf16_two_row_tiles_odd": (spec(390, 256, 4, 64, 2, act="gelu_tanh"), {}),
+    "tensor_bf16_two_row_tiles_skew": (spec(700, 256, 8, 96, 2), dict(skew=True)),
+    "tensor_bf16_shared_T150_two_row_tiles": (spec(150, 256, 16, 64, 4, shared=128, gated=True), {}),
 }
 
 
