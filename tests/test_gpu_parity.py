@@ -181,6 +181,7 @@ LAYER_CASES = {
     "tensor_bf16_two_row_tiles_odd": (spec(390, 256, 4, 64, 2, act="gelu_tanh"), {}),
     "tensor_bf16_two_row_tiles_skew": (spec(700, 256, 8, 96, 2), dict(skew=True)),
     "tensor_bf16_shared_T150_two_row_tiles": (spec(150, 256, 16, 64, 4, shared=128, gated=True), {}),
+    "tensor_bf16_wide_tiles": (spec(600, 256, 4, 64, 2), {}),   # 300 rows per expert: compute-bound, N = 256 tiles
 }
 
 
@@ -249,3 +250,4 @@ def test_token_order_invariance_on_gpu():
     perm = torch.randperm(s.T, generator=torch.Generator().manual_seed(0)).cuda()
     out_p = _gpu.run_layer(desc, w, x[perm].contiguous())
     assert torch.equal(out_p.view(torch.int16), out[perm].view(torch.int16))
+
