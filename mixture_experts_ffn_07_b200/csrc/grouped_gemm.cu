@@ -25,7 +25,10 @@
 //    [BN/2,BN) hold x W_up^T for the same outputs; the epilogue writes
 //    act(g) * u as bf16;
 //  * single mode (down, router): the epilogue scales row r by row_scale and
-//    stores it at row row_map[r] in f32 (the slot row of the pair).
+//    stores it at row row_map[r] in f32 (the slot row of the pair): each
+//    thread stages its row's 32-column segments in shared memory and the copy
+//    engine writes each as one 128-byte bulk store (full lines instead of
+//    16-byte pieces of 32 rows per warp store).
 //  * every mbarrier wait is bounded; on expiry the CTA records
 //    MOE_ERR_TIMEOUT, lets in-flight copies and MMAs land, frees TMEM and exits.
 #include <algorithm>
@@ -69,11 +72,30 @@ struct Aux {
   int cnt[MAX_G];
 };
 
+// Single-mode epilogue staging: each epilogue warp stages 32 rows x 32 f32
+// columns (a 144-byte pitch keeps the row writes free of bank conflicts) and
+// the copy engine stores each row's 128 bytes with one bulk copy.
+constexpr int kOutPitch = 144;
+constexpr int kOutStage = 4 * 32 * kOutPitch;
+
 template <int BN, int MT>
 constexpr size_t smem_bytes() {
   return 1024 + static_cast<size_t>(Tile<BN, MT>::STAGES) * Tile<BN, MT>::STAGE_BYTES +
-         sizeof(Aux<Tile<BN, MT>::STAGES>);
+         (sizeof(Aux<Tile<BN, MT>::STAGES>) + 127) / 128 * 128 + kOutStage;
 }
+
+// BYTES (a multiple of 16) of shared memory to global memory through the copy engine (one bulk group per call).
+template <int BYTES>
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "n"(BYTES)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The thread's bulk stores have finished reading shared memory / have completed.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Generic-proxy writes to shared memory become visible to the copy engine.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 struct KParams {
   const int32_t* offsets;
@@ -145,6 +167,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Aux<STAGES>& aux = *reinterpret_cast<Aux<STAGES>*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* out_stage = smem + STAGES * STAGE_BYTES + ((sizeof(Aux<STAGES>) + 127) / 128) * 128;
   volatile int* abort_flag = &aux.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -350,18 +373,40 @@ __global__ void __launch_bounds__(THREADS, 1)
           dest = p.row_map ? p.row_map[src] : src;
           scale = p.row_scale ? p.row_scale[dest] : 1.f;
         }
+        // this thread's row of the warp's staging area (32 rows x kOutPitch bytes)
+        uint8_t* srow = out_stage + (q * 32 + lane) * kOutPitch;
         for (int c = 0; c < BN_MMA; c += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tbase + c, v);
           tmem_ld_wait();
-          if (dest >= 0 && col0 + c < p.N) {
+          if (dest >= 0 && col0 + c < p.N && p.out_bf16) {  // bf16 rows (expert outputs of the tensor-core layer)
+            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(dest) * p.N + col0 + c;
+            if (col0 + c + 32 <= p.N) {  // a full 64-byte row segment: staged, then one bulk store
+              bulk_wait_read();
+              uint4* s4 = reinterpret_cast<uint4*>(srow);
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj)
+                s4[jj] = make_uint4(pack_bf16x2(scale * __uint_as_float(v[8 * jj]), scale * __uint_as_float(v[8 * jj + 1])),
+                                    pack_bf16x2(scale * __uint_as_float(v[8 * jj + 2]), scale * __uint_as_float(v[8 * jj + 3])),
+                                    pack_bf16x2(scale * __uint_as_float(v[8 * jj + 4]), scale * __uint_as_float(v[8 * jj + 5])),
+                                    pack_bf16x2(scale * __uint_as_float(v[8 * jj + 6]), scale * __uint_as_float(v[8 * jj + 7])));
+              fence_proxy_async_smem();
+              bulk_store<64>(dst, smem_addr(srow));
+            } else {
+              for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj)
+                dst[jj] = __float2bfloat16_rn(scale * __uint_as_float(v[jj]));
+            }
+          } else if (dest >= 0 && col0 + c < p.N) {
             float* dst = p.out_f32 + ks * p.part_stride + static_cast<size_t>(dest) * p.N + col0 + c;
-            if (col0 + c + 32 <= p.N) {
-              float4* d4 = reinterpret_cast<float4*>(dst);
+            if (col0 + c + 32 <= p.N) {  // a full 128-byte row segment: staged, then one bulk store
+              bulk_wait_read();          // the previous segment has left the staging row
+              float4* s4 = reinterpret_cast<float4*>(srow);
 #pragma unroll
               for (int jj = 0; jj < 8; ++jj)
-                d4[jj] = make_float4(scale * __uint_as_float(v[4 * jj]), scale * __uint_as_float(v[4 * jj + 1]),
+                s4[jj] = make_float4(scale * __uint_as_float(v[4 * jj]), scale * __uint_as_float(v[4 * jj + 1]),
                                      scale * __uint_as_float(v[4 * jj + 2]), scale * __uint_as_float(v[4 * jj + 3]));
+              fence_proxy_async_smem();
+              bulk_store<128>(dst, smem_addr(srow));
             } else {
               for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj) dst[jj] = scale * __uint_as_float(v[jj]);
             }
@@ -373,6 +418,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&aux.tempty[acc]);
     }
+    if (!DUAL) bulk_wait_all();  // every staged row segment is stored before the CTA ends
   }
 
   tc_fence_before();

@@ -90,6 +90,9 @@ cudaError_t launch_stream_down(const Ctx& c, const float* h, int I, int H, const
                                const float* row_scale, float* y);
 
 // out[t, :] = sum_k y_slots[t*K + k, :] (+ y_shared[t, :]) -> out_dtype.
+// out[t] = sum_k w[t,k] y_slots[t*K+k] in f32 (bf16 expert outputs), + y_shared[t] (f32), as bf16.
+cudaError_t launch_combine_weighted(const Ctx& c, const __nv_bfloat16* y_slots, const float* w, const float* y_shared,
+                                    int T, int K, int H, void* out);
 cudaError_t launch_combine(const Ctx& c, const float* y_slots, const float* y_shared, int T, int K, int H,
                            void* out, int out_dtype);
 

@@ -244,9 +244,12 @@ moe_status route_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const
   return MOE_OK;
 }
 
+// bf16_slots (tensor-core path of moe_layer): the slot rows hold the experts' unweighted outputs in bf16 and
+// the combine applies the routing weights (mlx-native moe_dispatch.rs, moe_weighted_sum_seq_bf16_input);
+// otherwise they hold topk_w-weighted f32 rows, as moe_expert_ffn documents.
 moe_status expert_impl(const moe::Ctx& c, const moe_desc& d, const void* x, const moe_weights& w,
                        const int32_t* offsets, const int32_t* sorted_pairs, const float* tw, float* y_slots, void* ws,
-                       const Layout& L, bool rows_gathered = false) {
+                       const Layout& L, bool rows_gathered = false, bool bf16_slots = false) {
   const int P = d.T * d.top_k;
   if (tensor_path(d)) {
     __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.x_perm);
@@ -279,9 +282,13 @@ moe_status expert_impl(const moe::Ctx& c, const moe_desc& d, const void* x, cons
     b.offsets = offsets;
     b.max_rows = P;
     b.dual = false;
-    b.out_f32 = y_slots;
+    if (bf16_slots) {
+      b.out_bf16 = reinterpret_cast<__nv_bfloat16*>(y_slots);
+    } else {
+      b.out_f32 = y_slots;
+      b.row_scale = tw;
+    }
     b.row_map = sorted_pairs;
-    b.row_scale = tw;
     b.name = "expert_down_gemm";
     MOE_TRY(moe::launch_grouped_gemm(c, b));
   } else {
@@ -295,7 +302,8 @@ moe_status expert_impl(const moe::Ctx& c, const moe_desc& d, const void* x, cons
 }
 
 moe_status combine_impl(const moe::Ctx& c, const moe_desc& d, const float* y_slots, const void* x,
-                        const moe_weights& w, const float* shared_gate, void* out, void* ws, const Layout& L) {
+                        const moe_weights& w, const float* shared_gate, void* out, void* ws, const Layout& L,
+                        const float* bf16_slot_weights = nullptr) {
   float* y_s = nullptr;
   if (d.shared_I > 0) {
     y_s = at<float>(ws, L.y_s);
@@ -338,7 +346,11 @@ moe_status combine_impl(const moe::Ctx& c, const moe_desc& d, const float* y_slo
                                       nullptr, d.T, gate, y_s));
     }
   }
-  MOE_TRY(moe::launch_combine(c, y_slots, y_s, d.T, d.top_k, d.H, out, d.act_dtype));
+  if (bf16_slot_weights)
+    MOE_TRY(moe::launch_combine_weighted(c, reinterpret_cast<const __nv_bfloat16*>(y_slots), bf16_slot_weights, y_s,
+                                         d.T, d.top_k, d.H, out));
+  else
+    MOE_TRY(moe::launch_combine(c, y_slots, y_s, d.T, d.top_k, d.H, out, d.act_dtype));
   return MOE_OK;
 }
 
@@ -626,14 +638,17 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
                                       d->act_dtype, w_s, d->router_dtype, d->H, sg));
       MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, f.counts, offsets, sorted_pairs, f.pair_pos));
     }
-    if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L, gathered)) != MOE_OK) return st;
-    return combine_impl(c, *d, y_slots, x, *w, sg, out, ws, L);
+    if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L, gathered, true)) != MOE_OK)
+      return st;
+    return combine_impl(c, *d, y_slots, x, *w, sg, out, ws, L, tw);
   }
   if ((st = route_impl(c, *d, x, *w, logits, parts, ids, tw, sg)) != MOE_OK) return st;
   MOE_TRY(moe::launch_permute(c, ids, d->T * d->top_k, d->E, at<int32_t>(ws, L.counts), offsets, sorted_pairs,
                               at<int32_t>(ws, L.pair_pos)));
-  if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L)) != MOE_OK) return st;
-  return combine_impl(c, *d, y_slots, x, *w, sg, out, ws, L);
+  const bool bf16_slots = tensor_path(*d);
+  if ((st = expert_impl(c, *d, x, *w, offsets, sorted_pairs, tw, y_slots, ws, L, false, bf16_slots)) != MOE_OK)
+    return st;
+  return combine_impl(c, *d, y_slots, x, *w, sg, out, ws, L, bf16_slots ? tw : nullptr);
 }
 
 moe_status moe_layer_host(const moe_desc* d, const void* x_host, const moe_weights* w, void* out_host, void* x_dev,

@@ -25,6 +25,11 @@ CASES = {
     "T1100_E256_shared_gated": (spec(1100, 1024, 256, 64, 8, shared=32, gated=True), {}),
     "T333_E64_shared_ungated": (spec(333, 512, 64, 256, 8, shared=96), {}),
     "skew_all_to_two": (spec(300, 256, 32, 64, 2), dict(skew=True)),
+    # E not dividing 512 (2, 3, 5 count threads per expert) and 16, 8, 4 split-K partial logits
+    # (one, two and four experts' parts requested together)
+    "T700_E224_16_parts": (spec(700, 1024, 224, 64, 8), {}),
+    "T2000_E160_8_parts": (spec(2000, 1024, 160, 64, 6), {}),
+    "T3000_E96_4_parts": (spec(3000, 512, 96, 64, 6), {}),
 }
 
 
