@@ -217,6 +217,10 @@ moe_status moe_combine(const moe_desc* d, const float* y_slots, const void* x, c
  * streaming path stages whole token rows in shared memory and returns
  * MOE_ERR_UNSUPPORTED (also from moe_expert_ffn / moe_combine) when
  * H * sizeof(act) > 65536 or I * 4 > 65536 or shared_I * 4 > 65536.
+ * On the tensor-core path each expert's output row is kept in bf16 and the
+ * combine adds w_k * y_k in f32 in slot order (mlx-native moe_dispatch.rs,
+ * moe_weighted_sum_seq_bf16_input), so the result may differ in the last bits
+ * from moe_expert_ffn + moe_combine, whose f32 slot rows are weighted first.
  *  x [T,H] act_dtype in, out [T,H] act_dtype out, ws >= moe_workspace_bytes(d).
  */
 moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, void* out, void* ws, size_t ws_bytes,
