@@ -351,6 +351,14 @@ int moe_trace_read(const char** names, float* ms, int max);
 void moe_debug_set_wait_limit(int64_t cycles);
 void moe_debug_set_skip_stage(int enable);
 
+/* Debug: CTA 0 of the cooperative kernels (the prefill front and the fused
+ * decode layer) spins `cycles` SM cycles before its first grid-barrier
+ * arrival (0: off).  With a wait limit below the delay the other CTAs give
+ * up on that barrier and report MOE_ERR_TIMEOUT; CTA 0 still arrives, so the
+ * barrier counter stays consistent for later launches.  Failure-detection
+ * tests only. */
+void moe_debug_set_barrier_delay(int64_t cycles);
+
 /* How moe_layer runs a batch of 1..64 tokens on the weight-streaming path:
  * enable = 1 (default) as one cooperative kernel ("decode_layer": router,
  * top-K, permutation, gate/up, down and combine as phases of one persistent

@@ -210,6 +210,11 @@ def debug_set_skip_stage(enable: bool) -> None:
     _lib.lib().moe_debug_set_skip_stage(int(enable))
 
 
+def debug_set_barrier_delay(cycles: int) -> None:
+    """moe_debug_set_barrier_delay: CTA 0 of the cooperative kernels arrives late at its first grid barrier."""
+    _lib.lib().moe_debug_set_barrier_delay(cycles)
+
+
 def set_fused_front(enable: bool) -> None:
     """moe_set_fused_front: selection + permutation + row gather of the tensor-core
     path as one cooperative kernel (True, default) or three launches (False)."""

@@ -24,7 +24,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route
            "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
            "moe_debug_set_wait_limit", "moe_debug_set_skip_stage", "moe_set_fused_decode",
            "moe_workspace_regions", "moe_set_fused_front", "moe_combine_backward", "moe_act_up_backward",
-           "moe_q6_k_split")
+           "moe_q6_k_split", "moe_debug_set_barrier_delay")
 
 
 class MoeDesc(ctypes.Structure):
@@ -91,6 +91,8 @@ def lib():
         L.moe_debug_set_wait_limit.restype = None
         L.moe_debug_set_skip_stage.argtypes = [I32]
         L.moe_debug_set_skip_stage.restype = None
+        L.moe_debug_set_barrier_delay.argtypes = [I64]
+        L.moe_debug_set_barrier_delay.restype = None
         L.moe_set_fused_decode.argtypes = [I32]
         L.moe_set_fused_decode.restype = None
         L.moe_set_fused_front.argtypes = [I32]

@@ -24,6 +24,8 @@ struct Ctx {
   int smem_optin;           // largest dynamic + static shared memory per block
   long long wait_limit;    // SM cycles a pipeline wait may spin before giving up
   int skip_stage;          // debug: grouped-GEMM producer skips one stage's loads
+  long long barrier_delay; // debug: CTA 0 of the cooperative kernels spins this many cycles before its first
+                           // grid-barrier arrival (it still arrives, so every barrier gets its full count)
   int pdl;                 // launch with programmatic stream serialization
 };
 
@@ -158,6 +160,15 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, long long limit, con
   }
   __threadfence();
   return true;
+}
+
+// Debug: thread 0 of CTA 0 spins `cycles` SM cycles (a fixed, finite delay).
+__device__ __forceinline__ void debug_delay_cta0(long long cycles) {
+  if (cycles > 0 && blockIdx.x == 0 && threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < cycles) {
+    }
+  }
 }
 
 // All threads of the CTA; false once this CTA has given up on a barrier.

@@ -69,6 +69,7 @@ struct DecodeArgs {
   void* out;
   int* status;
   long long wait_limit;
+  long long barrier_delay;
 };
 
 __device__ __forceinline__ bool cta_grid_sync(const DecodeArgs& a, int* s_abort, int* s_flag) {
@@ -197,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
         router_rows<float>(a, xs, rb * kWarps, ch, t0, nt, R);
     }
   }
+  debug_delay_cta0(a.barrier_delay);
   cta_grid_sync(a, &s_abort, &s_flag);
 
   // ---- S: logits, top-K and the pair permutation, in every CTA
@@ -515,6 +517,7 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
   a.out = L.out;
   a.status = c.status;
   a.wait_limit = c.wait_limit;
+  a.barrier_delay = c.barrier_delay;
   return launch_by_kind(c, a, P, L.x_dtype == MOE_F32, wkg, wkd);
 }
 

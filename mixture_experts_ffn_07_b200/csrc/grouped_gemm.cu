@@ -196,10 +196,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   pdl_trigger();
   pdl_wait();
   for (int g = threadIdx.x; g < p.G; g += THREADS) {
-    const int r0 = p.offsets ? p.offsets[g] : 0;
-    const int r1 = p.offsets ? p.offsets[g + 1] : p.rows_single;
+    const int o0 = p.offsets ? p.offsets[g] : 0;
+    const int o1 = p.offsets ? p.offsets[g + 1] : p.rows_single;
+    // a group's rows stay inside the A tensor (and so inside every output indexed by them), whatever the
+    // offsets hold; offsets outside it are reported
+    const int r0 = min(max(o0, 0), p.rows_single), r1 = min(max(o1, r0), p.rows_single);
+    if (r0 != o0 || r1 != o1) record_status(p.status, MOE_ERR_DEVICE_INDEX);
     aux.row_off[g] = r0;
-    aux.cnt[g] = max(0, r1 - r0);
+    aux.cnt[g] = r1 - r0;
   }
   __syncthreads();
   if (warp == 0) {  // exclusive scan of work items per group; lane owns groups [8*lane, 8*lane+8)
@@ -371,7 +375,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (r < rows_valid) {
           const int src = a_row + r;
           dest = p.row_map ? p.row_map[src] : src;
-          scale = p.row_scale ? p.row_scale[dest] : 1.f;
+          if (dest < 0 || dest >= p.rows_single) {  // output rows number the A rows: a bad map entry is skipped
+            record_status(p.status, MOE_ERR_DEVICE_INDEX);
+            dest = -1;
+          } else {
+            scale = p.row_scale ? p.row_scale[dest] : 1.f;
+          }
         }
         // this thread's row of the warp's staging area (32 rows x kOutPitch bytes)
         uint8_t* srow = out_stage + (q * 32 + lane) * kOutPitch;

@@ -33,6 +33,7 @@ std::mutex g_dev_mu;
 std::atomic<uint64_t> g_launches{0};
 std::atomic<long long> g_wait_limit{1LL << 31};
 std::atomic<int> g_skip_stage{0};
+std::atomic<long long> g_barrier_delay{0};
 std::atomic<int> g_fused_decode{1};
 std::atomic<int> g_fused_front{1};
 
@@ -69,6 +70,7 @@ bool make_ctx(cudaStream_t s, moe::Ctx* c) {
   c->stream = s;
   c->wait_limit = g_wait_limit.load();
   c->skip_stage = g_skip_stage.load();
+  c->barrier_delay = g_barrier_delay.load();
   c->pdl = 1;
   return true;
 }
@@ -789,6 +791,8 @@ moe_status moe_layer_noalloc(const moe_desc* d, const void* x, const moe_weights
 void moe_debug_set_wait_limit(int64_t cycles) { g_wait_limit.store(cycles > 0 ? cycles : (1LL << 31)); }
 
 void moe_debug_set_skip_stage(int enable) { g_skip_stage.store(enable ? 1 : 0); }
+
+void moe_debug_set_barrier_delay(int64_t cycles) { g_barrier_delay.store(cycles > 0 ? cycles : 0); }
 
 void moe_set_fused_decode(int enable) { g_fused_decode.store(enable ? 1 : 0); }
 

@@ -53,6 +53,7 @@ struct FrontArgs {
   int32_t* hist;  // [gridDim.x, E]
   int* status;
   long long wait_limit;
+  long long barrier_delay;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
@@ -78,9 +79,21 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
   for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&s_hist[a.ids[p]], 1);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) a.hist[static_cast<size_t>(c) * E + e] = s_hist[e];
+  debug_delay_cta0(a.barrier_delay);
   if (!grid_sync(&g_front_barrier, a.wait_limit, a.status, &s_abort, &s_flag)) {
-    // some CTA's counts may be missing: placing pairs could go out of range
+    // some CTA's counts may be missing: placing pairs could go out of range.  Leave tables the next kernels
+    // can follow without leaving their buffers: this CTA's pairs map to themselves, and CTA 0 (which writes
+    // the offsets when it gets through) gives every expert no rows.
     if (threadIdx.x == 0) record_status(a.status, MOE_ERR_TIMEOUT);
+    for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+      a.sorted_pairs[p] = p;
+      a.pair_pos[p] = p;
+    }
+    if (c == 0)
+      for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+        a.offsets[e] = 0;
+        if (e < E) a.counts[e] = 0;
+      }
     return;
   }
 
@@ -220,6 +233,7 @@ cudaError_t launch_prefill_front(const Ctx& c, const PrefillFront& f) {
   a.hist = f.hist;
   a.status = c.status;
   a.wait_limit = c.wait_limit;
+  a.barrier_delay = c.barrier_delay;
   // more than half of an SM's shared memory: one CTA per SM, one such grid per device (and room for the
   // warps' logit rows and the count partials)
   const int smem = std::max(c.smem_optin / 2 + 1024, kWarps * 256 * 4 + 2 * kThreads * 4);
