@@ -543,6 +543,8 @@ cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   // group.  The gate/up projection keeps one row tile per item: its long K rows already share weight tiles
   // through L2 between the CTAs running a group's row tiles side by side, and it keeps 6 stages.
   if (!a.dual && memory_bound && rows_per_group > 96.0) return launch_tiled<false, 128, 2>(c, a, 0);
+  // at most 128 output columns (the router: N = E): a 256-column tile would be three quarters zero fill
+  if (!a.dual && a.N <= 128) return launch_tiled<false, 128, 1>(c, a, 0);
   const bool narrow =
       memory_bound && wave_waste(items_wide, c.num_sms) - wave_waste(items_narrow, c.num_sms) > 0.03;
   if (a.dual) return narrow ? launch_tiled<true, 128, 1>(c, a, 0) : launch_tiled<true, 256, 1>(c, a, 0);
