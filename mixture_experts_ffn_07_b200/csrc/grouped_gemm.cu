@@ -549,8 +549,10 @@ cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   if (!a.dual && memory_bound && rows_per_group > 96.0) return launch_tiled<false, 128, 2>(c, a, 0);
   // at most 128 output columns (the router: N = E): a 256-column tile would be three quarters zero fill
   if (!a.dual && a.N <= 128) return launch_tiled<false, 128, 1>(c, a, 0);
-  const bool narrow =
-      memory_bound && wave_waste(items_wide, c.num_sms) - wave_waste(items_narrow, c.num_sms) > 0.03;
+  // narrow tiles waste less of the last wave, but every column tile re-reads the activation rows: with more than
+  // 96 rows per group (activations well beyond L2 on such launches) the dual launch keeps wide tiles
+  const bool narrow = memory_bound && !(a.dual && rows_per_group > 96.0) &&
+                      wave_waste(items_wide, c.num_sms) - wave_waste(items_narrow, c.num_sms) > 0.03;
   if (a.dual) return narrow ? launch_tiled<true, 128, 1>(c, a, 0) : launch_tiled<true, 256, 1>(c, a, 0);
   return narrow ? launch_tiled<false, 128, 1>(c, a, 0) : launch_tiled<false, 256, 1>(c, a, 0);
 }
