@@ -23,7 +23,7 @@
 //  * dual mode (gate/up): the BN-row B tile is BN/2 rows of W_gate followed
 //    by the same BN/2 rows of W_up, so TMEM columns [0,BN/2) hold x W_gate^T and
 //    [BN/2,BN) hold x W_up^T for the same outputs; the epilogue writes
-//    act(g) * u as bf16 (staged per row segment, one 64-byte bulk store each);
+//    act(g) * u as bf16;
 //  * single mode (down, router): the epilogue scales row r by row_scale and
 //    stores it at row row_map[r] in f32 (the slot row of the pair): each
 //    thread stages its row's 32-column segments in shared memory and the copy
@@ -344,7 +344,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int col0 = nt * p.col_step;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc * MT + j) * BN_MMA;
       if (DUAL) {
-        uint8_t* srow = out_stage + (q * 32 + lane) * kOutPitch;  // this thread's staging row
         for (int c = 0; c < BN_MMA / 2; c += 32) {
           uint32_t gr[32], ur[32];
           tmem_ld_32x32b_x32(tbase + c, gr);
@@ -359,14 +358,11 @@ __global__ void __launch_bounds__(THREADS, 1)
               packed[jj] = pack_bf16x2(h0, h1);
             }
             __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(a_row + r) * p.N + col0 + c;
-            if (col0 + c + 32 <= p.N) {  // a full 64-byte row segment: staged, then one bulk store
-              bulk_wait_read();
-              uint4* s4 = reinterpret_cast<uint4*>(srow);
+            if (col0 + c + 32 <= p.N) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
               for (int jj = 0; jj < 4; ++jj)
-                s4[jj] = make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]);
-              fence_proxy_async_smem();
-              bulk_store<64>(dst, smem_addr(srow));
+                d4[jj] = make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]);
             } else {
               const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(packed);
               for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj) dst[jj] = hv[jj];
@@ -431,7 +427,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&aux.tempty[acc]);
     }
-    bulk_wait_all();  // every staged row segment is stored before the CTA ends
+    if (!DUAL) bulk_wait_all();  // every staged row segment is stored before the CTA ends
   }
 
   tc_fence_before();
