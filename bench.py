@@ -208,6 +208,18 @@ def time_oracle(spec, wl, budget_s: float, max_tokens=None):
                         seconds=dt)
 
 
+def time_oracle_1thread(spec, wl, budget_s: float):
+    """The same oracle on one host thread, over a small token sample (about budget_s seconds)."""
+    import oracle
+    n_all = oracle.threads()
+    oracle.set_threads(1)
+    try:
+        v, info = time_oracle(spec, wl, budget_s=budget_s, max_tokens=max(1, min(spec.T, 64)))
+    finally:
+        oracle.set_threads(n_all)
+    return v, info
+
+
 def run_reference(args, spec):
     ws, rank, _ = _dist()
     if rank != 0:
@@ -354,7 +366,9 @@ def run_ours(args, spec):
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         v, info = time_oracle(spec, wl, budget_s=args.cpu_budget)
-        cpu = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle", "sample": info["sample"]}
+        v1, info1 = time_oracle_1thread(spec, wl, budget_s=min(3.0, args.cpu_budget))
+        cpu = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle", "sample": info["sample"],
+               "value_1thread": v1, "sample_1thread": info1["sample"]}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
