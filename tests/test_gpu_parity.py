@@ -251,3 +251,31 @@ def test_token_order_invariance_on_gpu():
     out_p = _gpu.run_layer(desc, w, x[perm].contiguous())
     assert torch.equal(out_p.view(torch.int16), out[perm].view(torch.int16))
 
+
+
+@pytest.mark.parametrize("case", ["tensor_bf16_shared_gated", "stream_q8_shared"])
+def test_two_streams_alternating_host_calls(case):
+    """moe_layer_host calls alternating over two streams, each with its own buffers and workspace (the pipelined
+    end-to-end benchmark), give the bits of one stream.  Both cooperative kernels (the prefill front and the fused
+    decode layer) keep their grid barriers consistent across the streams."""
+    s, _ = LAYER_CASES[case]
+    wl = make(s, seed=37)
+    desc, w, x = _gpu.upload(wl)
+    ref = _gpu.run_layer(desc, w, x)
+    xh = x.cpu().pin_memory()
+    sets = [dict(oh=torch.empty_like(xh).pin_memory(), xd=torch.empty_like(x), od=torch.empty_like(x),
+                 ws=torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda"),
+                 stream=torch.cuda.Stream()) for _ in range(2)]
+    outs = []
+    for i in range(8):
+        b = sets[i % 2]
+        if i >= 2:  # the pinned output of this stream's previous step is read before it is overwritten
+            b["stream"].synchronize()
+            outs.append(b["oh"].clone())
+        moe.layer_host(desc, xh, w, b["oh"], b["xd"], b["od"], b["ws"], stream=b["stream"])
+    torch.cuda.synchronize()
+    outs += [sets[0]["oh"].clone(), sets[1]["oh"].clone()]
+    assert moe.last_device_status() == moe.MOE_OK
+    bits = (lambda t: t.view(torch.int16)) if ref.dtype == torch.bfloat16 else (lambda t: t.view(torch.int32))
+    for o in outs:
+        assert torch.equal(bits(o), bits(ref.cpu()))
