@@ -141,7 +141,8 @@ __device__ __forceinline__ void router_stage_x(const DecodeArgs& a, float* xs, i
   }
 }
 
-template <typename XT, int WKG, int WKD>
+// MAXT: the most tokens of one expert batch (1 when T = 1: only single-token code, more loads in flight).
+template <typename XT, int WKG, int WKD, int MAXT>
 __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_expert[kMaxGroups], s_first[kMaxGroups], s_count[kMaxGroups], s_poff[kMaxGroups + 1];
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     __syncthreads();
     int p0, p1;
     cta_pairs(tb, s_ph[0], p0, p1);
-    if (!s_abort) run_phase<XT, WKG, true, kDecodeTok>(s_ph[0], tb, p0, p1, sm);
+    if (!s_abort) run_phase<XT, WKG, true, MAXT>(s_ph[0], tb, p0, p1, sm);
   }
   cta_grid_sync(a, &s_abort, &s_flag);
 
@@ -341,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     __syncthreads();
     int p0, p1;
     cta_pairs(tb, s_ph[1], p0, p1);
-    if (!s_abort) run_phase<float, WKD, false, kDecodeTok>(s_ph[1], tb, p0, p1, sm);
+    if (!s_abort) run_phase<float, WKD, false, MAXT>(s_ph[1], tb, p0, p1, sm);
   }
   const bool ok = cta_grid_sync(a, &s_abort, &s_flag);
 
@@ -386,24 +387,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
 }
 
 // Static shared memory of a kernel instance (queried once).
-template <typename XT, int WKG, int WKD>
+template <typename XT, int WKG, int WKD, int MAXT>
 int static_smem() {
   static std::atomic<int> bytes{-1};
   int b = bytes.load();
   if (b < 0) {
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, decode_layer_kernel<XT, WKG, WKD>) != cudaSuccess) return -1;
+    if (cudaFuncGetAttributes(&fa, decode_layer_kernel<XT, WKG, WKD, MAXT>) != cudaSuccess) return -1;
     b = static_cast<int>(fa.sharedSizeBytes);
     bytes.store(b);
   }
   return b;
 }
 
-template <typename XT, int WKG, int WKD>
-cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
-  auto kern = decode_layer_kernel<XT, WKG, WKD>;
+template <typename XT, int WKG, int WKD, int MAXT>
+cudaError_t launch_fused_t(const Ctx& c, const DecodeArgs& a, int P) {
+  auto kern = decode_layer_kernel<XT, WKG, WKD, MAXT>;
   const int smem = a.stage_bytes + 16 * P;
-  const int st = static_smem<XT, WKG, WKD>();
+  const int st = static_smem<XT, WKG, WKD, MAXT>();
   if (st < 0 || smem + st > c.smem_optin) return cudaErrorInvalidValue;
   const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -420,6 +421,13 @@ cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
+
+template <typename XT, int WKG, int WKD>
+cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
+  if (a.T == 1) return launch_fused_t<XT, WKG, WKD, 1>(c, a, P);
+  return launch_fused_t<XT, WKG, WKD, kDecodeTok>(c, a, P);
+}
+
 
 template <typename XT>
 cudaError_t launch_kinds(const Ctx& c, const DecodeArgs& a, int P, int wkg, int wkd) {

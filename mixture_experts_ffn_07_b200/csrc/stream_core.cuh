@@ -407,11 +407,13 @@ __device__ __forceinline__ void pair_out(const Phase& ph, int kind, int pi, int 
 // staged token rows (shared memory at `xs`, xrow_bytes apart); kb is a
 // multiple of kKSegAlign.  Lane partial sums are reduced over the warp; lane
 // c < NT returns token c's values in va, vb.
-template <int NT, int WK, typename AT>
+// U1: loads in flight per lane and row for one token (8 in code compiled for one token per batch, whose
+// registers allow it; 4 otherwise).
+template <int NT, int WK, typename AT, int U1 = 4>
 __device__ __forceinline__ void pair_dot(const uint8_t* wa, const uint8_t* wb, const uint8_t* sa, const uint8_t* sb,
                                          uint32_t xs, int xrow_bytes, int kb, int ke, float& va, float& vb) {
   constexpr int V = Chunk<WK, NT>::V;
-  constexpr int U = NT == 1 ? 4 : (NT == 2 ? 2 : 1);  // loads in flight per lane and row in each round
+  constexpr int U = NT == 1 ? U1 : (NT == 2 ? 2 : 1);  // loads in flight per lane and row in each round
   const int lane = threadIdx.x & 31;
   float2 acc_a[NT], acc_b[NT];
 #pragma unroll
@@ -686,7 +688,7 @@ __device__ __forceinline__ void prefetch_pair(const Phase& ph, int kind, int e, 
 
 // Elements [kb, ke) of row pair pi for NT tokens.  part == nullptr: the whole
 // row, outputs written; else the partial sums go to part[c][0..1].
-template <int NT, typename AT, int WK, bool DUAL>
+template <int NT, typename AT, int WK, bool DUAL, int MAXNT>
 __device__ __forceinline__ void run_unit(const Phase& ph, int kind, int e, int pi, int kb, int ke, float* part,
                                          const Smem& sm) {
   const GroupSrc& src = ph.src[kind];
@@ -711,7 +713,7 @@ __device__ __forceinline__ void run_unit(const Phase& ph, int kind, int e, int p
       q6k_pair_dot<NT, AT>(wa, wb, sa, sb, pl.Kdim, smem_addr(sm.xs), pl.xrow_bytes, kb, ke, acc_a, acc_b);
     pair_reduce<NT>(acc_a, acc_b, va, vb);
   } else {
-    pair_dot<NT, WK, AT>(wa, wb, sa, sb, smem_addr(sm.xs), pl.xrow_bytes, kb, ke, va, vb);
+    pair_dot<NT, WK, AT, MAXNT == 1 ? 8 : 4>(wa, wb, sa, sb, smem_addr(sm.xs), pl.xrow_bytes, kb, ke, va, vb);
   }
   if (lane < NT) {
     if (part) {
@@ -727,19 +729,24 @@ __device__ __forceinline__ void run_unit(const Phase& ph, int kind, int e, int p
 template <typename AT, int WK, bool DUAL, int MAXNT>
 __device__ __forceinline__ void unit_nt(int nr, const Phase& ph, int kind, int e, int pi, int kb, int ke, float* part,
                                         const Smem& sm) {
-  if (MAXNT <= 4 || nr <= 4) {
-    switch (nr) {
-      case 1: run_unit<1, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
-      case 2: run_unit<2, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
-      case 3: run_unit<3, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
-      default: run_unit<4, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
-    }
-  } else if constexpr (MAXNT > 4) {
-    switch (nr) {
-      case 5: run_unit<5, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
-      case 6: run_unit<6, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
-      case 7: run_unit<7, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
-      default: run_unit<8, AT, WK, DUAL>(ph, kind, e, pi, kb, ke, part, sm); break;
+  if constexpr (MAXNT == 1) {
+    (void)nr;
+    run_unit<1, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm);
+  } else {
+    if (MAXNT <= 4 || nr <= 4) {
+      switch (nr) {
+        case 1: run_unit<1, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+        case 2: run_unit<2, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+        case 3: run_unit<3, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+        default: run_unit<4, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+      }
+    } else if constexpr (MAXNT > 4) {
+      switch (nr) {
+        case 5: run_unit<5, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+        case 6: run_unit<6, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+        case 7: run_unit<7, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+        default: run_unit<8, AT, WK, DUAL, MAXNT>(ph, kind, e, pi, kb, ke, part, sm); break;
+      }
     }
   }
 }
