@@ -37,6 +37,7 @@ import workloads  # noqa: E402
 METRIC = "MoE layer tokens/s at 1 B200; % of BF16 tensor peak (prefill) / HBM BW (decode)"
 UNIT = "tokens/s"
 DEFAULT_CONFIG = "prefill_bf16_t512"
+NROT = 8  # token batches a layer bench rotates over
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -272,13 +273,20 @@ def run_ours(args, spec):
     wsb = torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    # routing once (outside timing) for the touched-expert count of the algorithmic bytes
-    _, ids, _, _ = host.run_route(desc, w, x)
-    counts = np.bincount(ids.cpu().numpy().reshape(-1), minlength=spec.E)
-    kern_alg, layer_alg, touched = algorithmic(spec, counts)
+    # Steps rotate over NROT seeded token batches, so consecutive steps route to different experts (a step
+    # that re-ran the same batch would find part of its experts' weights still in L2).
+    xs = [x] + [host.to_device(workloads.token_batch(spec, i), spec.act_dtype) for i in range(1, NROT)]
+    # routing once per batch (outside timing) for the touched-expert counts of the algorithmic bytes (mean)
+    algs = []
+    for xb in xs:
+        _, ids, _, _ = host.run_route(desc, w, xb)
+        algs.append(algorithmic(spec, np.bincount(ids.cpu().numpy().reshape(-1), minlength=spec.E)))
+    kern_alg = {n: {q: float(np.mean([a[0][n][q] for a in algs])) for q in ("bytes", "flops")} for n in algs[0][0]}
+    layer_alg = {q: float(np.mean([a[1][q] for a in algs])) for q in ("bytes", "flops")}
+    touched = float(np.mean([a[2] for a in algs]))
 
-    for _ in range(max(args.warmup, 3)):
-        moe.layer(desc, x, w, out, wsb)
+    for i in range(max(args.warmup, 3)):
+        moe.layer(desc, xs[i % NROT], w, out, wsb)
     torch.cuda.synchronize()
     assert moe.last_device_status() == moe.MOE_OK
 
@@ -290,8 +298,8 @@ def run_ours(args, spec):
     clocks.start()
     n_launch0 = moe.launch_count()
     ev0.record(stream)
-    for _ in range(args.steps):
-        moe.layer(desc, x, w, out, wsb)
+    for i in range(args.steps):
+        moe.layer(desc, xs[i % NROT], w, out, wsb)
     ev1.record(stream)
     torch.cuda.synchronize()
     n_launch = moe.launch_count() - n_launch0
@@ -304,8 +312,8 @@ def run_ours(args, spec):
     # per-kernel durations: the same steps again with an event pair around every launch
     # (events between kernels serialise them, so this pass is not the timed one)
     moe.trace_enable(True)
-    for _ in range(min(args.steps, 400)):
-        moe.layer(desc, x, w, out, wsb)
+    for i in range(min(args.steps, 400)):
+        moe.layer(desc, xs[i % NROT], w, out, wsb)
     torch.cuda.synchronize()
     moe.trace_enable(False)
     trace = moe.trace_read()
@@ -348,7 +356,8 @@ def run_ours(args, spec):
     # memory, runs the layer and copies its out back.  Two streams, each with its own device buffers, workspace
     # and pinned output, take alternate steps, so one step's copies overlap the other's compute -- how a server
     # keeps the GPU busy while it moves the next batch.
-    xh = x.cpu().pin_memory()
+    xhs = [xb.cpu().pin_memory() for xb in xs]
+    xh = xhs[0]
     e2e_sets = []
     for _ in range(2):
         e2e_sets.append(dict(oh=torch.empty_like(xh).pin_memory(), xd=torch.empty_like(x), od=torch.empty_like(x),
@@ -357,7 +366,7 @@ def run_ours(args, spec):
 
     def e2e_step(i):
         b = e2e_sets[i % 2]
-        moe.layer_host(desc, xh, w, b["oh"], b["xd"], b["od"], b["ws"], stream=b["stream"])
+        moe.layer_host(desc, xhs[i % NROT], w, b["oh"], b["xd"], b["od"], b["ws"], stream=b["stream"])
 
     for i in range(max(args.warmup, 3)):
         e2e_step(i)
@@ -393,7 +402,8 @@ def run_ours(args, spec):
             "data": "synthetic",
             "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
                        "act": spec.act, "shared_I": spec.shared_I, "parallelism": f"replicas{ws_n}",
-                       "l2": "no flush: inputs larger than L2 (expert weights streamed every step)"},
+                       "l2": f"no flush: inputs larger than L2; x rotates over {NROT} token batches, so consecutive "
+                             "steps route to different experts"},
             "e2e": {"value": job_throughput(ws_n, T, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
                     "d2h_bytes_per_step": io_bytes, "call": "moe_layer_host", "streams": 2},
             "roofline": roofline, "layer_roofline": layer_roof, "cpu_baseline": cpu, "gpu_launches": n_launch,

@@ -146,17 +146,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 // gave up still arrives at the later barriers (wait == false), so every
 // barrier of a launch sees all G arrivals and the counter stays consistent.
 // One thread per CTA; returns false when it did not wait to completion.
+// The poll is a relaxed load (one L2 round trip per turn; the fence after the
+// loop orders what follows), and the status word is read every 32nd turn only,
+// so the wake-up after the last arrival costs one round trip, not two.
 __device__ __forceinline__ bool grid_barrier(unsigned* bar, long long limit, const int* status, bool wait) {
   __threadfence();
   const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
   const unsigned old = atomicAdd(bar, add);
   if (!wait) return false;
   const long long t0 = clock64();
-  while (true) {
+  for (unsigned turn = 0;; ++turn) {
     unsigned cur;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
     if ((cur ^ old) & 0x80000000u) break;
-    if (*reinterpret_cast<const volatile int*>(status) != 0 || clock64() - t0 > limit) return false;
+    if ((turn & 31u) == 31u &&
+        (*reinterpret_cast<const volatile int*>(status) != 0 || clock64() - t0 > limit))
+      return false;
   }
   __threadfence();
   return true;

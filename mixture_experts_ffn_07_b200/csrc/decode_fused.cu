@@ -124,6 +124,17 @@ __device__ __forceinline__ void router_rows(const DecodeArgs& a, const float* xs
   }
 }
 
+// Asks L2 for router row r's chunk ch (lane 0; skipped unless 16-byte aligned).
+__device__ __forceinline__ void router_prefetch_row(const DecodeArgs& a, int r, int ch, int R) {
+  if ((threadIdx.x & 31) != 0 || r >= R) return;
+  const size_t es = a.router_bf16 ? 2 : 4;
+  const int h0 = ch * kRouterChunk, hc = min(kRouterChunk, a.H - h0);
+  const uint8_t* p = r < a.E ? static_cast<const uint8_t*>(a.router) + (static_cast<size_t>(r) * a.H + h0) * es
+                             : static_cast<const uint8_t*>(a.w_s) + h0 * es;
+  const uint32_t bytes = static_cast<uint32_t>(hc * es);
+  if (((reinterpret_cast<uintptr_t>(p) | bytes) & 15u) == 0) prefetch_l2(p, bytes);
+}
+
 // Stages x[t0 .. t0+nt) [h0 .. h0+hc) as f32 rows of kRouterChunk.  All threads.
 template <typename XT>
 __device__ __forceinline__ void router_stage_x(const DecodeArgs& a, float* xs, int ch, int t0, int nt) {
@@ -188,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
       const int ch = cg % nch, tg = cg / nch;
       const int t0 = tg * kTokGroup, nt = min(kTokGroup, T - t0);
       if (cg != staged) {
+        router_prefetch_row(a, rb * kWarps + warp, ch, R);  // the row chunk's fetch overlaps the x staging
         __syncthreads();
         router_stage_x<XT>(a, xs, ch, t0, nt);
         __syncthreads();
@@ -210,17 +222,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
       float l[9];  // experts lane + 32 i; chunk partials requested together, added in chunk order
 #pragma unroll
       for (int i = 0; i < 9; ++i) l[i] = 0.f;
-      for (int ch0 = 0; ch0 < nch; ch0 += 2) {
-        float v[2][9];
+      for (int ch0 = 0; ch0 < nch; ch0 += 4) {
+        float v[4][9];
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int i = 0; i < 9; ++i)
             v[j][i] = (ch0 + j < nch && lane + 32 * i < R)
                           ? __ldcg(a.parts + (static_cast<size_t>(ch0 + j) * T + t) * R + lane + 32 * i)
                           : 0.f;
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int i = 0; i < 9; ++i)
             if (ch0 + j < nch) l[i] += v[j][i];

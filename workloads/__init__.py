@@ -223,6 +223,7 @@ class Workload:
 
 # stream ids of the tensors of one workload
 S_X, S_ROUTER, S_GATE, S_UP, S_DOWN, S_SH_GATE, S_SH_UP, S_SH_DOWN, S_SH_GATE_W = range(1, 10)
+S_X_ALT = 64  # streams S_X_ALT + i: further token batches of a config
 
 
 def _weight(seed, stream, shape, fan_in, w_dtype, down=False):
@@ -235,6 +236,14 @@ def _weight(seed, stream, shape, fan_in, w_dtype, down=False):
     return normal(seed, stream, shape, 1.0 / math.sqrt(fan_in), w_dtype)
 
 
+def token_batch(spec: Spec, i: int, seed: int | None = None, x_std: float = 1.0) -> np.ndarray:
+    """Token batch i of a config: 0 is the workload's own x, i > 0 further batches of the same
+    distribution (benchmarks rotate over them so that consecutive steps route differently)."""
+    if seed is None:
+        seed = config_seed(spec.name)
+    return normal(seed, S_X if i == 0 else S_X_ALT + i, (spec.T, spec.H), x_std, spec.act_dtype)
+
+
 def make(spec: Spec, seed: int | None = None, x_std: float = 1.0) -> Workload:
     """Draw every input tensor of one layer invocation (host numpy arrays).
 
@@ -244,7 +253,7 @@ def make(spec: Spec, seed: int | None = None, x_std: float = 1.0) -> Workload:
     if seed is None:
         seed = config_seed(spec.name)
     T, H, E, I, Is = spec.T, spec.H, spec.E, spec.I, spec.shared_I
-    x = normal(seed, S_X, (T, H), x_std, spec.act_dtype)
+    x = token_batch(spec, 0, seed, x_std)
     router = normal(seed, S_ROUTER, (E, H), spec.router_std, spec.router_dtype)
     bias = zipf_log_bias(E) if spec.router_bias == "zipf1.1" else None
     gate = _weight(seed, S_GATE, (E, I, H), H, spec.w_dtype)
