@@ -170,6 +170,25 @@ def _dist():
     return ws, rank, local
 
 
+def per_call_ms(call, stream, n: int = 50, warmup: int = 10, flush=None) -> float:
+    """Median over n single calls of their CUDA-event time on `stream`; with `flush` (a device buffer
+    larger than L2) each call follows a write of the whole buffer, so it starts from a cold L2."""
+    import torch
+    for _ in range(warmup):
+        call()
+    ts = []
+    for i in range(n):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(statistics.median(ts))
+
+
 def max_over_ranks(dist, x: float, device) -> float:
     """The largest of every rank's x (a device time in ms): the job's time.  Every
     rank must call it at the same point."""
@@ -389,6 +408,17 @@ def run_ours(args, spec):
     e2e_ms = max_over_ranks(dist, e2e_ms, "cuda")
     io_bytes = T * H * x.element_size()
 
+    # single calls on one token batch: median of 50 after 10 warm-up calls, each after a 512 MB scratch write
+    # (cold L2), and back to back (warm: whatever of the step's data L2 still holds)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    one = lambda: moe.layer(desc, xs[0], w, out, wsb)  # noqa: E731
+    cold_ms = per_call_ms(one, stream, flush=flush)
+    warm_ms = per_call_ms(one, stream)
+    del flush
+    single = {"calls": 50, "warmup": 10, "flush_bytes": 512 << 20, "cold_median_ms": cold_ms,
+              "warm_median_ms": warm_ms, "cold_tokens_per_s": T / cold_ms * 1e3, "warm_tokens_per_s": T / warm_ms * 1e3,
+              "cold_hbm_frac": algs[0][1]["bytes"] / (cold_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         v, info = time_oracle(spec, wl, budget_s=args.cpu_budget)
@@ -407,7 +437,7 @@ def run_ours(args, spec):
             "e2e": {"value": job_throughput(ws_n, T, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
                     "d2h_bytes_per_step": io_bytes, "call": "moe_layer_host", "streams": 2},
             "roofline": roofline, "layer_roofline": layer_roof, "cpu_baseline": cpu, "gpu_launches": n_launch,
-            "clocks": clocks.summary(), "device_status": moe.status_string(status),
+            "single_call": single, "clocks": clocks.summary(), "device_status": moe.status_string(status),
             "kernels": {n: {"launches": k["launches"], "avg_us": 1e3 * k["avg_ms"], "share": round(k["share"], 4)}
                         for n, k in sorted(kernels.items(), key=lambda kv: -kv[1]["total_ms"])}}
     if rank == 0:
