@@ -54,3 +54,16 @@ def test_configs_shapes():
     assert wl.x.shape == (3, 64) and wl.x.dtype == np.uint16
     assert wl.gate.shape == (4, 32, 64) and wl.down.shape == (4, 64, 32)
     assert wl.sh_gate.shape == (32, 64) and wl.sh_down.shape == (64, 32) and wl.sh_gate_w.shape == (64,)
+
+
+def test_token_batches():
+    spec = workloads.Spec(T=3, H=64, E=4, I=32, K=2)
+    wl = workloads.make(spec, seed=5)
+    assert np.array_equal(workloads.token_batch(spec, 0, seed=5), wl.x)  # batch 0 is the workload's own x
+    b1, b2 = workloads.token_batch(spec, 1, seed=5), workloads.token_batch(spec, 2, seed=5)
+    assert b1.shape == wl.x.shape and b1.dtype == wl.x.dtype
+    assert not np.array_equal(b1, wl.x) and not np.array_equal(b1, b2)
+    assert np.array_equal(b1, workloads.token_batch(spec, 1, seed=5))
+    # no further batch shares a stream with the weights
+    assert not np.array_equal(workloads.token_batch(spec, 1, seed=5).reshape(-1)[:16],
+                              wl.gate.reshape(-1)[:16])
