@@ -29,6 +29,9 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+// dynamic shared memory: [kWarps][256] f32 logit rows (A), [2][kThreads] count partials (B), then the
+// positions of this CTA's pairs (B)
+constexpr int kPosOff = kWarps * 256 * 4 + 2 * kThreads * 4;
 
 __device__ unsigned g_front_barrier;
 
@@ -51,13 +54,14 @@ struct FrontArgs {
   int32_t* pair_pos;
   __nv_bfloat16* x_perm;
   int32_t* hist;  // [gridDim.x, E]
+  int pos_cap;    // pair positions the shared-memory area after the count partials holds (0: none)
   int* status;
   long long wait_limit;
   long long barrier_delay;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
-  extern __shared__ __align__(16) uint8_t fsmem[];  // [16 warps][256] f32 logit rows, then [2][512] count partials
+  extern __shared__ __align__(16) uint8_t fsmem[];  // layout: kPosOff
   __shared__ int s_hist[256], s_run[256], s_tot[256], s_off[257];
   __shared__ int s_abort, s_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -167,6 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
   }
   if (c == 0 && threadIdx.x == 0) a.offsets[E] = s_off[E];
   __syncthreads();
+  int* s_pos = reinterpret_cast<int*>(fsmem + kPosOff);
+  const bool pos_in_smem = p1 - p0 <= a.pos_cap;
   if (warp == 0) {  // in pair order, 32 at a time; equal experts ranked by lane
     for (int base = p0; base < p1; base += 32) {
       const int p = base + lane;
@@ -179,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
         const int pos = before + rank;
         a.sorted_pairs[pos] = p;
         a.pair_pos[p] = pos;
+        if (pos_in_smem) s_pos[p - p0] = pos;
         if (rank == 0) s_run[e] = before + __popc(m);
       }
       __syncwarp();
@@ -190,14 +197,14 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
   uint4* dst = reinterpret_cast<uint4*>(a.x_perm);
   for (int p = p0 + warp; p < p1; p += kWarps) {
     const uint4* s = src + static_cast<size_t>(p / K) * n16;
-    uint4* d = dst + static_cast<size_t>(a.pair_pos[p]) * n16;
-    for (int o = lane; o < n16; o += 32 * 4) {
-      uint4 v[4];
+    uint4* d = dst + static_cast<size_t>(pos_in_smem ? s_pos[p - p0] : a.pair_pos[p]) * n16;
+    for (int o = lane; o < n16; o += 32 * 8) {  // a 4 KB row (H = 2048) in one round of loads
+      uint4 v[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 8; ++j)
         if (o + 32 * j < n16) v[j] = __ldg(s + o + 32 * j);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 8; ++j)
         if (o + 32 * j < n16) d[o + 32 * j] = v[j];
     }
   }
@@ -235,13 +242,16 @@ cudaError_t launch_prefill_front(const Ctx& c, const PrefillFront& f) {
   a.wait_limit = c.wait_limit;
   a.barrier_delay = c.barrier_delay;
   // more than half of an SM's shared memory: one CTA per SM, one such grid per device (and room for the
-  // warps' logit rows and the count partials)
-  const int smem = std::max(c.smem_optin / 2 + 1024, kWarps * 256 * 4 + 2 * kThreads * 4);
+  // warps' logit rows, the count partials and, when they fit, the positions of a CTA's pairs)
+  const int grid = std::min(c.num_sms, kMaxFrontCtas);
+  const long long max_pairs = (static_cast<long long>(f.T) + grid - 1) / grid * f.K;
+  a.pos_cap = kPosOff + max_pairs * 4 <= c.smem_optin ? static_cast<int>(max_pairs) : 0;
+  const int smem = std::max(c.smem_optin / 2 + 1024, kPosOff + a.pos_cap * 4);
   const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(front_kernel), smem);
   if (e != cudaSuccess) return e;
   KernelScope ks(c, "route_permute_gather");
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(std::min(c.num_sms, kMaxFrontCtas));
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = c.stream;
