@@ -440,7 +440,6 @@ cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
   return launch_fused_t<XT, WKG, WKD, kDecodeTok>(c, a, P);
 }
 
-
 template <typename XT>
 cudaError_t launch_kinds(const Ctx& c, const DecodeArgs& a, int P, int wkg, int wkd) {
   if (wkg == WK_F32) return launch_fused<XT, WK_F32, WK_F32>(c, a, P);

@@ -61,7 +61,7 @@ struct FrontArgs {
 };
 
 __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
-  extern __shared__ __align__(16) uint8_t fsmem[];  // layout: kPosOff
+  extern __shared__ __align__(16) uint8_t fsmem[];  // logit rows, count partials, pair positions (kPosOff)
   __shared__ int s_hist[256], s_run[256], s_tot[256], s_off[257];
   __shared__ int s_abort, s_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
