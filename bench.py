@@ -4,10 +4,13 @@
 
 A step is one moe_layer call (router, top-K, permutation, expert GEMMs, shared
 expert, combine) over one batch of the workload, inputs resident in HBM.  The
-default workload is the batched prefill layer (T=512, H=2048, E=64, K=8,
-I=1024, SiLU, bf16).  Under torchrun (N > 1) every rank runs an independent
-replica of the layer on its own GPU (the layer does not shard); the time is
-the max over ranks and `value` counts the tokens of all ranks.
+default workload is the largest one that fits one GPU: the skewed layer
+(T=8192, H=7168, E=256, K=8, I=2048, SiLU, bf16, one ungated shared expert of
+intermediate 2048, Zipf(1.1) router bias; 22.5 GB of expert weights).  Under
+torchrun (N > 1) every rank runs an independent replica of the layer on its own
+GPU (the layer does not shard); the time is the max over ranks and `value`
+counts the tokens of all ranks.  `--gpus N` with N > 1 outside torchrun starts
+the N ranks itself (torch.distributed.run on 127.0.0.1).
 
 --impl reference times the f64 CPU oracle on the host cores instead (rank 0
 only), on bounded token samples of the same workload.
@@ -36,9 +39,10 @@ import workloads  # noqa: E402
 
 METRIC = "MoE layer tokens/s at 1 B200; % of BF16 tensor peak (prefill) / HBM BW (decode)"
 UNIT = "tokens/s"
-DEFAULT_CONFIG = "prefill_bf16_t512"
+DEFAULT_CONFIG = "skewed_zipf_t8192"
 NROT = 8  # token batches a layer bench rotates over
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}  # B200 data-sheet HBM3e bandwidth and dense bf16 rate
 
 
 def _peaks():
@@ -86,6 +90,50 @@ def algorithmic(spec, counts):
                                      flops=0)
     k["decode_layer"] = dict(layer)  # the whole layer in one launch
     return k, layer, touched
+
+
+def kernel_roofline(alg, avg_ms, peaks, peak_src):
+    """One kernel's achieved rate against its roofline: TFLOP/s when its arithmetic intensity is above the
+    ridge of the measured peaks, else GB/s.  `frac` divides by the sustained bf16 rate (a kernel timed inside a
+    long loop of steps) or the measured copy bandwidth; `frac_burst` by the burst bf16 rate; `frac_nominal` by
+    the data-sheet figure (2.25 PFLOP/s dense bf16, 8 TB/s)."""
+    avg_s = avg_ms / 1e3
+    tensor_bound = alg["flops"] / max(alg["bytes"], 1) > 1e3 * peaks["bf16_tflops"] / peaks["hbm_gbs"]
+    if tensor_bound:
+        achieved, peak, unit = alg["flops"] / avg_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        extra = {"frac_burst": achieved / peaks["bf16_tflops"], "peak_burst": peaks["bf16_tflops"],
+                 "frac_nominal": achieved / NOMINAL["bf16_tflops"]}
+    else:
+        achieved, peak, unit = alg["bytes"] / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        extra = {"frac_nominal": achieved / NOMINAL["hbm_gbs"]}
+    return dict({"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
+                 "frac": achieved / peak}, **extra, avg_us=1e3 * avg_ms,
+                algorithmic_bytes_per_launch=alg["bytes"], algorithmic_flops_per_launch=alg["flops"],
+                peak_source=f"{peak_src} ({'bf16_tflops_sustained' if tensor_bound else 'hbm_gbs'})")
+
+
+def expert_load(counts_list):
+    """Rows per expert over the step's token batches: touched experts, the largest and the smallest
+    nonzero load (mean over batches), and batch 0's sorted loads in full."""
+    touched = [int(np.count_nonzero(c)) for c in counts_list]
+    mx = [int(c.max()) for c in counts_list]
+    mn = [int(c[c > 0].min()) if np.any(c > 0) else 0 for c in counts_list]
+    c0 = np.sort(counts_list[0])[::-1]
+    return {"touched_mean": float(np.mean(touched)), "max_rows_mean": float(np.mean(mx)),
+            "min_nonzero_rows_mean": float(np.mean(mn)), "max_rows": max(mx), "min_nonzero_rows": min(mn),
+            "batch0_rows_desc": [int(v) for v in c0[c0 > 0]]}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 # ------------------------------------------------------------------ clocks during the timed region
@@ -262,7 +310,7 @@ def run_reference(args, spec):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
                        "shared_I": spec.shared_I, "step_sample_tokens": per_step},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
                              "sample": f"{per_step} random tokens of {spec.T} per step, full layer in f64"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -296,10 +344,11 @@ def run_ours(args, spec):
     # that re-ran the same batch would find part of its experts' weights still in L2).
     xs = [x] + [host.to_device(workloads.token_batch(spec, i), spec.act_dtype) for i in range(1, NROT)]
     # routing once per batch (outside timing) for the touched-expert counts of the algorithmic bytes (mean)
-    algs = []
+    algs, loads = [], []
     for xb in xs:
         _, ids, _, _ = host.run_route(desc, w, xb)
-        algs.append(algorithmic(spec, np.bincount(ids.cpu().numpy().reshape(-1), minlength=spec.E)))
+        loads.append(np.bincount(ids.cpu().numpy().reshape(-1), minlength=spec.E))
+        algs.append(algorithmic(spec, loads[-1]))
     kern_alg = {n: {q: float(np.mean([a[0][n][q] for a in algs])) for q in ("bytes", "flops")} for n in algs[0][0]}
     layer_alg = {q: float(np.mean([a[1][q] for a in algs])) for q in ("bytes", "flops")}
     touched = float(np.mean([a[2] for a in algs]))
@@ -353,23 +402,18 @@ def run_ours(args, spec):
     peaks, peak_src = _peaks()
     roofline = None
     if dom:
-        alg = kern_alg.get(dom, {"bytes": 0, "flops": 0})
-        avg_s = kernels[dom]["avg_ms"] / 1e3
-        tensor_bound = alg["flops"] / max(alg["bytes"], 1) > 1e3 * peaks["bf16_tflops"] / peaks["hbm_gbs"]
-        if tensor_bound:
-            achieved, peak, unit = alg["flops"] / avg_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
-        else:
-            achieved, peak, unit = alg["bytes"] / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
-        roofline = {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
-                    "frac": achieved / peak, "traffic": _traffic(dom, spec.name), "kernel": dom,
-                    "algorithmic_bytes_per_launch": alg["bytes"], "algorithmic_flops_per_launch": alg["flops"],
-                    "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if tensor_bound else 'hbm_gbs'})"}
+        roofline = kernel_roofline(kern_alg.get(dom, {"bytes": 0, "flops": 0}), kernels[dom]["avg_ms"], peaks,
+                                   peak_src)
+        roofline.update(traffic=_traffic(dom, spec.name), kernel=dom)
+        # every GEMM of the step against the same peaks (the expert GEMMs carry the layer's arithmetic)
+        roofline["gemms"] = {n: kernel_roofline(kern_alg[n], kernels[n]["avg_ms"], peaks, peak_src)
+                             for n in kernels if n.endswith("_gemm") and n in kern_alg}
     layer_s = ms_step / 1e3
     layer_roof = {"bytes": layer_alg["bytes"], "flops": layer_alg["flops"],
                   "GB/s": layer_alg["bytes"] / layer_s / 1e9, "TFLOP/s": layer_alg["flops"] / layer_s / 1e12,
                   "hbm_frac": layer_alg["bytes"] / layer_s / 1e9 / peaks["hbm_gbs"],
                   "tensor_frac": layer_alg["flops"] / layer_s / 1e12 / peaks["bf16_tflops_sustained"],
-                  "touched_experts": touched}
+                  "touched_experts": touched, "expert_load": expert_load(loads)}
 
     # end to end through the public host-buffer call (moe_layer_host): every step copies its x from pinned host
     # memory, runs the layer and copies its out back.  Two streams, each with its own device buffers, workspace
@@ -423,8 +467,10 @@ def run_ours(args, spec):
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         v, info = time_oracle(spec, wl, budget_s=args.cpu_budget)
         v1, info1 = time_oracle_1thread(spec, wl, budget_s=min(3.0, args.cpu_budget))
-        cpu = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle", "sample": info["sample"],
-               "value_1thread": v1, "sample_1thread": info1["sample"]}
+        cpu = {"value": v, "unit": UNIT, "cores": info["cores"], "cpu_model": cpu_model(), "kind": "oracle",
+               "sample": info["sample"], "value_1thread": v1, "sample_1thread": info1["sample"]}
+        if info["tokens"] < spec.T:  # tokens/s of the sample; the full layer's time is extrapolated from it
+            cpu["extrapolation"] = {"full_layer_s": spec.T / v, "from_tokens": info["tokens"], "of_tokens": spec.T}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -608,6 +654,37 @@ def run_backward(args, spec):
     return 0
 
 
+def spawn_ranks(n: int) -> int:
+    """Runs this command again as n ranks on this node (torch.distributed.run, rendezvous on 127.0.0.1)
+    and returns its exit status."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def dist_selftest(args) -> int:
+    """The multi-rank plumbing without a GPU: each rank reports a time that depends on its rank, the job
+    takes the largest, and rank 0 prints the line the GPU bench would print for it."""
+    import datetime
+
+    import torch.distributed as dist
+    ws, rank, _ = _dist()
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = max_over_ranks(dist, 10.0 + rank, "cpu")
+        if rank == 0:
+            print(json.dumps({"selftest": True, "n_gpus": ws, "ms": ms,
+                              "value": job_throughput(ws, 1, args.steps, ms)}), flush=True)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -619,7 +696,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default="layer", choices=["layer", "backward"],
                     help="backward: the combine and act*up backward kernels on the workload's slots")
+    ap.add_argument("--dist-selftest", action="store_true",
+                    help="ranks only: gloo process group, max over ranks of a rank-dependent time, no GPU work")
     args = ap.parse_args()
+    ws = int(os.environ.get("WORLD_SIZE", "0"))
+    if args.gpus > 1 and ws == 0:
+        return spawn_ranks(args.gpus)
+    if ws and ws != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={ws}", file=sys.stderr)
+        return 2
+    if args.dist_selftest:
+        return dist_selftest(args)
     spec = workloads.CONFIGS[args.config]
     if args.op == "backward":
         return run_backward(args, spec)

@@ -58,3 +58,25 @@ def test_kquant_bytes_per_weight():
     _, b, _ = bench.algorithmic(s, _counts(s.E, 11))
     # Q4_K: 144 bytes per 256 weights (gate, up); Q6_K: 210 bytes per 256 (down)
     assert b["bytes"] - a["bytes"] == pytest.approx((2 * 144 + 210) / 256 * s.I * s.H)
+
+
+def test_kernel_roofline_fractions():
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    # 1 TFLOP over 1 GB in 1 ms: 1000 TFLOP/s, far above the ridge -> tensor bound
+    r = bench.kernel_roofline({"flops": 1e12, "bytes": 1e9}, 1.0, peaks, "measured")
+    assert r["bound"] == "tensor" and r["achieved"] == pytest.approx(1000.0)
+    assert r["frac"] == pytest.approx(1000 / 1400) and r["frac_burst"] == pytest.approx(1000 / 1600)
+    assert r["frac_nominal"] == pytest.approx(1000 / 2250)
+    # 1 GB and 1 GFLOP in 0.5 ms: 2000 GB/s -> HBM bound
+    r = bench.kernel_roofline({"flops": 1e9, "bytes": 1e9}, 0.5, peaks, "measured")
+    assert r["bound"] == "hbm" and r["achieved"] == pytest.approx(2000.0)
+    assert r["frac"] == pytest.approx(2000 / 6500) and r["frac_nominal"] == pytest.approx(0.25)
+
+
+def test_expert_load_summary():
+    a = np.array([0, 5, 1, 0, 9])
+    b = np.array([2, 2, 2, 2, 0])
+    d = bench.expert_load([a, b])
+    assert d["touched_mean"] == 3.5 and d["max_rows"] == 9 and d["min_nonzero_rows"] == 1
+    assert d["max_rows_mean"] == 5.5 and d["min_nonzero_rows_mean"] == 1.5
+    assert d["batch0_rows_desc"] == [9, 5, 1]

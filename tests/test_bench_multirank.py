@@ -61,3 +61,27 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(None, 2.5, "cpu") == 2.5
     assert bench.job_throughput(1, 512, 4, 2.0) == pytest.approx(512 * 4 / 2e-3)
+
+
+def test_gpus_flag_starts_the_ranks_itself():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself; rank 0 alone prints one line whose time is
+    the slower rank's (the rank-1 time 11 ms)."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "4",
+                        "--dist-selftest"], capture_output=True, text=True, timeout=240, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["ms"] == 11.0
+    assert d["value"] == pytest.approx(2 * 4 / 11e-3)
+
+
+def test_gpus_flag_disagreeing_with_world_size_fails():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="3")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dist-selftest"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0

@@ -20,7 +20,8 @@ import workloads  # noqa: E402
 from tests import _gpu  # noqa: E402
 
 SAMPLE = {"decode_f32_t1": 1, "prefill_bf16_t512": 48, "routed_shared_t4096": 24, "skewed_zipf_t8192": 8,
-          "q8_0_decode_t16": 16, "grouped_sigmoid_t512": 32, "q4k_q6k_decode_t16": 16}
+          "q8_0_decode_t16": 16, "grouped_sigmoid_t512": 32, "q4k_q6k_decode_t16": 16,
+          "gemm_h7168_i2048_e8_t2048": 16}
 
 
 @pytest.mark.parametrize("name", workloads.CONFIG_ORDER)

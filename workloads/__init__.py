@@ -195,6 +195,9 @@ CONFIGS = {
     # Q8_0-decode shapes with the k-quant stacks of the Metal MoE providers: gate/up Q4_K, down Q6_K
     "q4k_q6k_decode_t16": Spec(T=16, H=2048, E=128, I=768, K=8, act_dtype=F32, w_dtype=Q4_K_Q6_K, router_dtype=F32,
                                name="q4k_q6k_decode_t16"),
+    # the skewed layer's expert shapes (H=7168, I=2048) with every token on all 8 experts: 2048 rows per expert,
+    # a few GB on the device, for profiling the expert GEMMs where they are tensor bound
+    "gemm_h7168_i2048_e8_t2048": Spec(T=2048, H=7168, E=8, I=2048, K=8, name="gemm_h7168_i2048_e8_t2048"),
 }
 CONFIG_ORDER = list(CONFIGS)
 BASE_SEED = 0xB2000000
