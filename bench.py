@@ -93,7 +93,8 @@ def algorithmic(spec, counts):
 
 
 def kernel_roofline(alg, avg_ms, peaks, peak_src):
-    """One kernel's achieved rate against its roofline: TFLOP/s when its arithmetic intensity is above the
+    """One kernel's achieved rate (its algorithmic work per step over its time per step, `avg_ms`) against its
+    roofline: TFLOP/s when its arithmetic intensity is above the
     ridge of the measured peaks, else GB/s.  `frac` divides by the sustained bf16 rate (a kernel timed inside a
     long loop of steps) or the measured copy bandwidth; `frac_burst` by the burst bf16 rate; `frac_nominal` by
     the data-sheet figure (2.25 PFLOP/s dense bf16, 8 TB/s)."""
@@ -333,6 +334,7 @@ def run_ours(args, spec):
     import mixture_experts_ffn_07_b200 as moe
     from mixture_experts_ffn_07_b200 import host
 
+    moe.set_pair_gemm(bool(args.pair_gemm))
     wl = workloads.make(spec)
     desc, w, x = host.upload(wl)
     T, H = spec.T, spec.H
@@ -397,17 +399,25 @@ def run_ours(args, spec):
     tot = sum(k["total_ms"] for k in kernels.values()) or 1.0
     for k in kernels.values():
         k["share"] = k["total_ms"] / tot
-    dom = max(kernels, key=lambda n: kernels[n]["total_ms"]) if kernels else None
+    # a step's time per kernel: a compute-bound expert GEMM runs as two launches (full 256-row tiles on CTA pairs,
+    # then each group's remaining rows, traced as "<name>_tail"), which together do that GEMM's work
+    traced_steps = min(args.steps, 400)
+    step_ms = {}
+    for n, k in kernels.items():
+        base = n[: -len("_tail")] if n.endswith("_tail") else n
+        step_ms[base] = step_ms.get(base, 0.0) + k["total_ms"] / traced_steps
+    dom = max(step_ms, key=step_ms.get) if step_ms else None
 
     peaks, peak_src = _peaks()
     roofline = None
     if dom:
-        roofline = kernel_roofline(kern_alg.get(dom, {"bytes": 0, "flops": 0}), kernels[dom]["avg_ms"], peaks,
-                                   peak_src)
-        roofline.update(traffic=_traffic(dom, spec.name), kernel=dom)
+        roofline = kernel_roofline(kern_alg.get(dom, {"bytes": 0, "flops": 0}), step_ms[dom], peaks, peak_src)
+        roofline.update(traffic=_traffic(dom, spec.name), kernel=dom,
+                        launches_per_step=sum(k["launches"] for n, k in kernels.items()
+                                              if n in (dom, dom + "_tail")) / traced_steps)
         # every GEMM of the step against the same peaks (the expert GEMMs carry the layer's arithmetic)
-        roofline["gemms"] = {n: kernel_roofline(kern_alg[n], kernels[n]["avg_ms"], peaks, peak_src)
-                             for n in kernels if n.endswith("_gemm") and n in kern_alg}
+        roofline["gemms"] = {n: kernel_roofline(kern_alg[n], step_ms[n], peaks, peak_src)
+                             for n in step_ms if n.endswith("_gemm") and n in kern_alg}
     layer_s = ms_step / 1e3
     layer_roof = {"bytes": layer_alg["bytes"], "flops": layer_alg["flops"],
                   "GB/s": layer_alg["bytes"] / layer_s / 1e9, "TFLOP/s": layer_alg["flops"] / layer_s / 1e12,
@@ -478,6 +488,7 @@ def run_ours(args, spec):
             "data": "synthetic",
             "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
                        "act": spec.act, "shared_I": spec.shared_I, "parallelism": f"replicas{ws_n}",
+                       "pair_gemm": bool(args.pair_gemm),
                        "l2": f"no flush: inputs larger than L2; x rotates over {NROT} token batches, so consecutive "
                              "steps route to different experts"},
             "e2e": {"value": job_throughput(ws_n, T, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
@@ -654,6 +665,70 @@ def run_backward(args, spec):
     return 0
 
 
+# ------------------------------------------------------------------ where the two paths cross
+CROSS_T = (8, 16, 32, 48, 64, 96, 128, 192, 256)
+CROSS_SHAPES = {  # bf16 layers: the prefill and routed+shared shapes, and the Q8_0-decode shape with bf16 weights
+    "prefill_bf16": workloads.Spec(T=max(CROSS_T), H=2048, E=64, I=1024, K=8, name="cross_prefill_bf16"),
+    "routed_shared_bf16": workloads.Spec(T=max(CROSS_T), H=2048, E=256, I=512, K=8, shared_I=512, shared_gated=True,
+                                         name="cross_routed_shared_bf16"),
+    "decode_shape_bf16": workloads.Spec(T=max(CROSS_T), H=2048, E=128, I=768, K=8, name="cross_decode_shape_bf16"),
+}
+
+
+def run_crossover(args):
+    """--op crossover: one bf16 layer call per step on the weight-streaming path (the fused decode kernel up to
+    64 tokens, the step-by-step streaming launches beyond) and on the tensor-core path, for each batch size in
+    CROSS_T, over 8 rotating token batches (weights of every shape exceed L2).  Prints the table as one JSON line;
+    the fastest path per size is where moe_layer's default threshold should sit."""
+    import dataclasses
+
+    import torch
+    import mixture_experts_ffn_07_b200 as moe
+    from mixture_experts_ffn_07_b200 import host
+    ws_n, rank, local = _dist()
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    stream = torch.cuda.current_stream()
+    table = {}
+    for shape, spec in CROSS_SHAPES.items():
+        wl = workloads.make(spec)
+        desc0, w, x0 = host.upload(wl)
+        xs = [x0] + [host.to_device(workloads.token_batch(spec, i), "bf16") for i in range(1, NROT)]
+        rows = {}
+        for T in CROSS_T:
+            desc = dataclasses.replace(desc0, T=T)
+            res = {}
+            for path, thr in (("streaming", 10 ** 9), ("tensor", 1)):
+                moe.set_tensor_min_tokens(thr)
+                try:
+                    out = torch.empty((T, spec.H), dtype=torch.bfloat16, device="cuda")
+                    wsb = torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+                    xb = [xx[:T] for xx in xs]
+                    for i in range(max(args.warmup, 3)):
+                        moe.layer(desc, xb[i % NROT], w, out, wsb)
+                    n = max(10, min(args.steps, 200))
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    torch.cuda.synchronize()
+                    a.record(stream)
+                    for i in range(n):
+                        moe.layer(desc, xb[i % NROT], w, out, wsb)
+                    b.record(stream)
+                    torch.cuda.synchronize()
+                    res[path] = 1e3 * a.elapsed_time(b) / n
+                finally:
+                    moe.set_tensor_min_tokens(65)
+            assert moe.last_device_status() == moe.MOE_OK
+            res["faster"] = min(("streaming", "tensor"), key=lambda k: res[k])
+            rows[T] = res
+        table[shape] = rows
+        del w, xs
+        torch.cuda.empty_cache()
+    print(json.dumps({"op": "crossover", "unit": "us per layer call", "tokens": list(CROSS_T), "table": table}),
+          flush=True)
+    return 0
+
+
 def spawn_ranks(n: int) -> int:
     """Runs this command again as n ranks on this node (torch.distributed.run, rendezvous on 127.0.0.1)
     and returns its exit status."""
@@ -694,8 +769,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="layer", choices=["layer", "backward"],
-                    help="backward: the combine and act*up backward kernels on the workload's slots")
+    ap.add_argument("--op", default="layer", choices=["layer", "backward", "crossover"],
+                    help="backward: the combine and act*up backward kernels on the workload's slots; "
+                         "crossover: both paths of bf16 layers over batch sizes 8..256")
+    ap.add_argument("--pair-gemm", type=int, default=1, choices=[0, 1],
+                    help="0: compute-bound expert GEMMs on single CTAs only (moe_set_pair_gemm), for comparison")
     ap.add_argument("--dist-selftest", action="store_true",
                     help="ranks only: gloo process group, max over ranks of a rank-dependent time, no GPU work")
     args = ap.parse_args()
@@ -708,6 +786,8 @@ def main():
     if args.dist_selftest:
         return dist_selftest(args)
     spec = workloads.CONFIGS[args.config]
+    if args.op == "crossover":
+        return run_crossover(args)
     if args.op == "backward":
         return run_backward(args, spec)
     if args.impl == "reference":

@@ -376,6 +376,24 @@ void moe_set_fused_decode(int enable);
  * moe_layer takes the three launches by itself.  Process-wide. */
 void moe_set_fused_front(int enable);
 
+/* How the tensor-core expert GEMMs run compute-bound launches (groups that
+ * average at least 200 rows): enable = 1 (default) puts every group's full
+ * 256-row tiles on pairs of CTAs (clusters of two SMs sharing one
+ * tcgen05.mma.cta_group::2 of M = 256, N = 256) and the rows left in each group
+ * on the single-CTA kernel; 0 runs all rows on the single-CTA kernel
+ * (M = 128).  Same arithmetic per output element either way (one f32
+ * accumulator per element, K in the same order), so the same bits.
+ * Process-wide; takes effect at the next call. */
+void moe_set_pair_gemm(int enable);
+
+/* The fewest tokens for which a bf16 layer (bf16 activations and expert
+ * weights) takes the tensor-core path (router GEMM, grouped tcgen05 GEMMs)
+ * instead of the weight-streaming path; default 65 (the streaming path for
+ * 1..64 tokens).  Values below 1 count as 1.  moe_workspace_bytes follows the
+ * current setting, so size workspaces after changing it.  Process-wide; for
+ * measuring where the two paths cross. */
+void moe_set_tensor_min_tokens(int tokens);
+
 #ifdef __cplusplus
 }
 #endif

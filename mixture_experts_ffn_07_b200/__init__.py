@@ -221,6 +221,18 @@ def set_fused_front(enable: bool) -> None:
     _lib.lib().moe_set_fused_front(int(enable))
 
 
+def set_pair_gemm(enable: bool) -> None:
+    """moe_set_pair_gemm: full 256-row tiles of compute-bound expert GEMMs on CTA pairs
+    (tcgen05.mma.cta_group::2, True, default) or every row on single CTAs (False)."""
+    _lib.lib().moe_set_pair_gemm(int(enable))
+
+
+def set_tensor_min_tokens(tokens: int) -> None:
+    """moe_set_tensor_min_tokens: bf16 layers of at least `tokens` tokens take the tensor-core path
+    (default 65); size workspaces after changing it."""
+    _lib.lib().moe_set_tensor_min_tokens(int(tokens))
+
+
 def set_fused_decode(enable: bool) -> None:
     """moe_set_fused_decode: one cooperative kernel (True, default) or step-by-step
     launches (False) for 1..64 tokens on the weight-streaming path."""

@@ -23,7 +23,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route
            "moe_combine", "moe_layer", "moe_layer_host", "moe_layer_noalloc", "moe_q8_0_split",
            "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
            "moe_debug_set_wait_limit", "moe_debug_set_skip_stage", "moe_set_fused_decode",
-           "moe_workspace_regions", "moe_set_fused_front", "moe_combine_backward", "moe_act_up_backward",
+           "moe_workspace_regions", "moe_set_fused_front", "moe_set_pair_gemm", "moe_set_tensor_min_tokens", "moe_combine_backward", "moe_act_up_backward",
            "moe_q6_k_split", "moe_debug_set_barrier_delay")
 
 
@@ -97,6 +97,10 @@ def lib():
         L.moe_set_fused_decode.restype = None
         L.moe_set_fused_front.argtypes = [I32]
         L.moe_set_fused_front.restype = None
+        L.moe_set_pair_gemm.argtypes = [I32]
+        L.moe_set_pair_gemm.restype = None
+        L.moe_set_tensor_min_tokens.argtypes = [I32]
+        L.moe_set_tensor_min_tokens.restype = None
         L.moe_workspace_regions.argtypes = [DP, ctypes.POINTER(MoeWsRegions)]
         L.moe_workspace_regions.restype = I32
         _lib = L

@@ -138,27 +138,34 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 
 // ---- grid barrier (cooperative launches only) ----
 // A barrier over every CTA of a grid that is resident as a whole (a
-// cooperative launch), on a counter in device memory: CTA 0 adds
-// 2^31 - (G-1) and the others add 1, so each complete barrier moves the
-// counter by exactly 2^31 (its top bit flips, its low bits come back); a CTA
-// waits for the top bit to differ from the value it saw on arrival.  The wait
-// is bounded and abandoned when the status word reports an error; a CTA that
-// gave up still arrives at the later barriers (wait == false), so every
-// barrier of a launch sees all G arrivals and the counter stays consistent.
-// One thread per CTA; returns false when it did not wait to completion.
-// The poll is a relaxed load (one L2 round trip per turn; the fence after the
-// loop orders what follows), and the status word is read every 32nd turn only,
-// so the wake-up after the last arrival costs one round trip, not two.
-__device__ __forceinline__ bool grid_barrier(unsigned* bar, long long limit, const int* status, bool wait) {
+// cooperative launch), on a 64-bit counter in device memory that only grows:
+// CTA 0 adds 2^32 - (G-1) and the others add 1, so each complete barrier adds
+// exactly 2^32 and the counter rests at a multiple of 2^32 between barriers
+// (while a barrier fills, the high word stays where it was).  A CTA waits
+// until the high word differs from the one it saw on arrival: the completion
+// of its own barrier, which a later barrier on the same counter can only move
+// further, so a CTA that polls late never misses it.  Arrivals of two grids
+// never mix on one barrier: each launch is checked on the host to fit one CTA
+// per SM, so a CTA of a later grid starts only on an SM that a CTA of the
+// earlier grid has left, after that grid's last barrier completed.
+// The wait is bounded and abandoned when the status word reports an error; a
+// CTA that gave up still arrives at the later barriers (wait == false), so
+// every barrier of a launch sees all G arrivals and the counter stays at a
+// multiple of 2^32.  One thread per CTA; returns false when it did not wait
+// to completion.  The poll is a relaxed load (one L2 round trip per turn; the
+// fence after the loop orders what follows), and the status word is read every
+// 32nd turn only, so the wake-up after the last arrival costs one round trip.
+__device__ __forceinline__ bool grid_barrier(unsigned long long* bar, long long limit, const int* status, bool wait) {
   __threadfence();
-  const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
-  const unsigned old = atomicAdd(bar, add);
+  const unsigned long long add = blockIdx.x == 0 ? (1ull << 32) - (gridDim.x - 1) : 1ull;
+  const unsigned long long old = atomicAdd(bar, add);
   if (!wait) return false;
+  const unsigned hi = static_cast<unsigned>(old >> 32);
   const long long t0 = clock64();
   for (unsigned turn = 0;; ++turn) {
-    unsigned cur;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
-    if ((cur ^ old) & 0x80000000u) break;
+    unsigned long long cur;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(cur) : "l"(bar) : "memory");
+    if (static_cast<unsigned>(cur >> 32) != hi) break;
     if ((turn & 31u) == 31u &&
         (*reinterpret_cast<const volatile int*>(status) != 0 || clock64() - t0 > limit))
       return false;
@@ -177,7 +184,7 @@ __device__ __forceinline__ void debug_delay_cta0(long long cycles) {
 }
 
 // All threads of the CTA; false once this CTA has given up on a barrier.
-__device__ __forceinline__ bool grid_sync(unsigned* bar, long long limit, const int* status, int* s_abort,
+__device__ __forceinline__ bool grid_sync(unsigned long long* bar, long long limit, const int* status, int* s_abort,
                                           int* s_flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -270,6 +277,75 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---- CTA pairs (clusters of two CTAs sharing one tcgen05.mma.cta_group::2) ----
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address in the cluster's shared window of the same variable in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_addr(p)), "r"(rank));
+  return a;
+}
+// Every thread of both CTAs; orders the shared-memory work before it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster (cluster address).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+// 2D tiled TMA load into this CTA's shared memory whose completion is counted
+// on an mbarrier of either CTA of the pair (cluster address); no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t cluster_bar, int c0,
+                                                 int r0, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_addr(smem_dst)),
+      "l"(map), "r"(cluster_bar), "r"(c0), "r"(r0), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(smem_slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem of both CTAs] (+)= A[smem of both CTAs] * B[smem of both CTAs]^T:
+// M = 256 (each CTA's 128 rows of A land in its own TMEM lanes), N = 256 (each
+// CTA holds N/2 rows of B at the same shared-memory offset).  Issued by one
+// thread of the even CTA.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at this offset in every CTA of `mask` when the
+// pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(mask)
+      : "memory");
+}
 
 // Shared-memory matrix descriptor: K-major tile whose rows are 128 bytes (64 bf16),
 // 8-row groups 1024 bytes apart, 128-byte swizzle (the layout TMA writes with

@@ -19,14 +19,13 @@
 //      its gate).                                                  -- barrier
 //   C  combine: out[t] = sum_k y_slot[t, k] (+ y_shared[t]) in that order.
 //
-// The grid barrier is a counter in device memory: CTA 0 adds 2^31 - (G-1) and
-// the others add 1, so every complete barrier moves the counter by exactly
-// 2^31 (its top bit flips, its low bits come back to 0); a CTA waits for the
-// top bit to differ from the value it saw on arrival.  Waits are bounded; a
-// CTA that gives up still arrives at the later barriers, so every barrier of a
-// launch sees all G arrivals and the counter is consistent for the next launch.
-// Only one such grid can be resident on a device at a time (each takes every
-// SM), so one counter per device serves all launches.
+// The grid barrier is the bounded counter barrier of common.cuh (a 64-bit
+// counter per device that grows by 2^32 per completed barrier).  Waits are
+// bounded; a CTA that gives up still arrives at the later barriers, so every
+// barrier of a launch sees all G arrivals and the counter is consistent for
+// the next launch.  The launch asks for more than half of an SM's shared
+// memory and checks on the host that one CTA per SM is the most that fits, so
+// only one such grid runs on a device at a time and one counter serves all.
 #include <atomic>
 
 #include "route_util.cuh"
@@ -43,7 +42,7 @@ constexpr int kDecodeTok = 4;  // token rows per expert batch in the GEMV phases
 constexpr int kMaxRouterRows = 257;
 constexpr int kRouterSteps = kRouterChunk / 256;  // 8-element steps of a lane per chunk
 
-__device__ unsigned g_decode_barrier;
+__device__ unsigned long long g_decode_barrier;
 
 struct DecodeArgs {
   const void* x;
@@ -415,11 +414,17 @@ int static_smem() {
 template <typename XT, int WKG, int WKD, int MAXT>
 cudaError_t launch_fused_t(const Ctx& c, const DecodeArgs& a, int P) {
   auto kern = decode_layer_kernel<XT, WKG, WKD, MAXT>;
-  const int smem = a.stage_bytes + 16 * P;
+  // more than half of an SM's shared memory, so one CTA per SM whatever the register count: a CTA of a later
+  // grid then starts only after this grid's last barrier (the barrier counter is shared by all launches)
+  const int smem = std::max(a.stage_bytes + 16 * P, c.smem_optin / 2 + 1024);
   const int st = static_smem<XT, WKG, WKD, MAXT>();
   if (st < 0 || smem + st > c.smem_optin) return cudaErrorInvalidValue;
-  const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
+  cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm != 1) return cudaErrorInvalidValue;  // the step-by-step launches run instead
   KernelScope ks(c, "decode_layer");
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(c.num_sms);

@@ -25,13 +25,15 @@
 //    [BN/2,BN) hold x W_up^T for the same outputs; the epilogue writes
 //    act(g) * u as bf16;
 //  * single mode (down, router): the epilogue scales row r by row_scale and
-//    stores it at row row_map[r] in f32 (the slot row of the pair): each
-//    thread stages its row's 32-column segments in shared memory and the copy
-//    engine writes each as one 128-byte bulk store (full lines instead of
-//    16-byte pieces of 32 rows per warp store).
+//    stores it at row row_map[r] (the slot row of the pair), f32 or bf16;
+//  * both epilogues pass each row's output through the warp's staging rows in
+//    shared memory, 128 bytes per row at a time, and the warp writes them out
+//    as whole 128-byte row segments (four rows per store instruction) instead
+//    of 16-byte pieces of 32 rows, or one small bulk copy per row segment;
 //  * every mbarrier wait is bounded; on expiry the CTA records
 //    MOE_ERR_TIMEOUT, lets in-flight copies and MMAs land, frees TMEM and exits.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 
 #include "kernels.h"
@@ -45,6 +47,7 @@ constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int MAX_G = 256;
 constexpr int THREADS = 192;
+constexpr int kMaxPairDevices = 64;
 
 // Tile shape per instantiation: the MMA is M=128 x N=BN; an item covers MT
 // (1 or 2) row tiles of one group against the same BN weight rows, so a stage
@@ -72,9 +75,9 @@ struct Aux {
   int cnt[MAX_G];
 };
 
-// Single-mode epilogue staging: each epilogue warp stages 32 rows x 32 f32
-// columns (a 144-byte pitch keeps the row writes free of bank conflicts) and
-// the copy engine stores each row's 128 bytes with one bulk copy.
+// Epilogue staging: each epilogue warp owns 32 rows x 128 bytes of shared
+// memory (a 144-byte pitch keeps both the row writes and the row-segment
+// reads free of bank conflicts).
 constexpr int kOutPitch = 144;
 constexpr int kOutStage = 4 * 32 * kOutPitch;
 
@@ -83,19 +86,6 @@ constexpr size_t smem_bytes() {
   return 1024 + static_cast<size_t>(Tile<BN, MT>::STAGES) * Tile<BN, MT>::STAGE_BYTES +
          (sizeof(Aux<Tile<BN, MT>::STAGES>) + 127) / 128 * 128 + kOutStage;
 }
-
-// BYTES (a multiple of 16) of shared memory to global memory through the copy engine (one bulk group per call).
-template <int BYTES>
-__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "n"(BYTES)
-               : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// The thread's bulk stores have finished reading shared memory / have completed.
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Generic-proxy writes to shared memory become visible to the copy engine.
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 struct KParams {
   const int32_t* offsets;
@@ -116,6 +106,8 @@ struct KParams {
   int* status;
   long long wait_limit;
   int skip_stage;
+  int head_mult;       // single-CTA kernel: skip each group's first floor(rows / head_mult) * head_mult rows
+                       // (the CTA-pair kernel's full 256-row tiles); 0: all rows
 };
 
 // Wait ignoring the abort flag (used to drain in-flight work before exit).
@@ -153,6 +145,97 @@ __device__ __forceinline__ void decode_item(const AuxT& aux, int G, int ksplit, 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+// Epilogue of one accumulator tile: TMEM lane q*32 + lane (this thread's row)
+// holds BN f32 columns from `tbase`.  The output goes out in slabs of 128 bytes
+// per row: each thread writes its row's slab into the warp's staging rows, then
+// the warp copies the 32 staged rows out with 16-byte stores, 8 lanes per row,
+// so each store instruction writes four whole 128-byte row segments wherever
+// the rows go (rows are scattered through row_map in the down projection).
+//  DUAL: h[dest, col0 + c] = act(g_c) * u_c as bf16, c < BN/2 (g: columns
+//        [0, BN/2), u: [BN/2, BN));
+//  else: out[dest, col0 + c] = scale * acc_c, bf16 (out_bf16) or f32.
+// dest < 0: the row is not written.  Column chunks at or beyond p.N are not
+// written (N is a multiple of 32, so a 16-byte chunk is all in or all out).
+// All lanes of the warp; the TMEM loads are .sync.aligned.
+template <bool DUAL, int BN>
+__device__ __forceinline__ void epilogue_tile(const KParams& p, uint32_t tbase, uint8_t* wstage, int dest, float scale,
+                                              int col0, int ks) {
+  const int lane = threadIdx.x & 31;
+  uint8_t* srow = wstage + lane * kOutPitch;
+  const uint32_t stage_s = smem_addr(wstage);
+  const bool f32_out = !DUAL && p.out_bf16 == nullptr;
+  const int ocols = DUAL ? BN / 2 : BN;      // output columns of the tile
+  const int slab = f32_out ? 32 : 64;        // output columns per 128-byte slab
+  for (int s0 = 0; s0 < ocols; s0 += slab) {
+    if (col0 + s0 >= p.N) break;  // warp-uniform
+    if (f32_out) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tbase + s0, v);
+      tmem_ld_wait();
+      uint4* s4 = reinterpret_cast<uint4*>(srow);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+        s4[jj] = make_uint4(__float_as_uint(scale * __uint_as_float(v[4 * jj])),
+                            __float_as_uint(scale * __uint_as_float(v[4 * jj + 1])),
+                            __float_as_uint(scale * __uint_as_float(v[4 * jj + 2])),
+                            __float_as_uint(scale * __uint_as_float(v[4 * jj + 3])));
+    } else {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // 32 output columns = 64 bytes of the slab each
+        const int c = s0 + 32 * half;
+        uint32_t packed[16];
+        if (DUAL) {
+          uint32_t gr[32], ur[32];
+          tmem_ld_32x32b_x32(tbase + c, gr);
+          tmem_ld_32x32b_x32(tbase + BN / 2 + c, ur);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const float h0 = act_fn(p.act, __uint_as_float(gr[2 * jj])) * __uint_as_float(ur[2 * jj]);
+            const float h1 = act_fn(p.act, __uint_as_float(gr[2 * jj + 1])) * __uint_as_float(ur[2 * jj + 1]);
+            packed[jj] = pack_bf16x2(h0, h1);
+          }
+        } else {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            packed[jj] = pack_bf16x2(scale * __uint_as_float(v[2 * jj]), scale * __uint_as_float(v[2 * jj + 1]));
+        }
+        uint4* s4 = reinterpret_cast<uint4*>(srow + 64 * half);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          s4[jj] = make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]);
+      }
+    }
+    __syncwarp();
+    // copy out: lane -> staged row 4 i + lane / 8, 16-byte chunk lane % 8
+    const int ch = lane & 7;
+    const int cpe = f32_out ? 4 : 8;  // output columns per 16-byte chunk
+    const int col = col0 + s0 + ch * cpe;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = 4 * i + (lane >> 3);
+      const int d = __shfl_sync(0xffffffffu, dest, rr);
+      const uint4 v = lds128(stage_s + rr * kOutPitch + ch * 16);
+      if (d >= 0 && col < p.N) {
+        if (f32_out)
+          *reinterpret_cast<uint4*>(p.out_f32 + ks * p.part_stride + static_cast<size_t>(d) * p.N + col) = v;
+        else
+          *reinterpret_cast<uint4*>(p.out_bf16 + static_cast<size_t>(d) * p.N + col) = v;
+      }
+    }
+    __syncwarp();  // the staged rows are read before the next slab overwrites them
+  }
 }
 
 template <bool DUAL, int BN, int MT>
@@ -194,7 +277,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_relinquish();
   }
   pdl_trigger();
-  pdl_wait();
+  // The tail launch after the CTA-pair kernel (head_mult > 0) reads only what the kernels before the pair
+  // kernel wrote, which the pair kernel's CTAs waited for before they let this launch start, and writes rows
+  // the pair kernel does not: it starts at once (filling the pair kernel's last wave) and waits for the pair
+  // kernel only before it exits, so that the launches after it see both kernels' output.
+  if (p.head_mult == 0) pdl_wait();
   for (int g = threadIdx.x; g < p.G; g += THREADS) {
     const int o0 = p.offsets ? p.offsets[g] : 0;
     const int o1 = p.offsets ? p.offsets[g + 1] : p.rows_single;
@@ -202,8 +289,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // offsets hold; offsets outside it are reported
     const int r0 = min(max(o0, 0), p.rows_single), r1 = min(max(o1, r0), p.rows_single);
     if (r0 != o0 || r1 != o1) record_status(p.status, MOE_ERR_DEVICE_INDEX);
-    aux.row_off[g] = r0;
-    aux.cnt[g] = r1 - r0;
+    const int head = p.head_mult > 0 ? (r1 - r0) / p.head_mult * p.head_mult : 0;
+    aux.row_off[g] = r0 + head;
+    aux.cnt[g] = r1 - r0 - head;
   }
   __syncthreads();
   if (warp == 0) {  // exclusive scan of work items per group; lane owns groups [8*lane, 8*lane+8)
@@ -343,37 +431,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int a_row = aux.row_off[g] + mt * BM;
       const int col0 = nt * p.col_step;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc * MT + j) * BN_MMA;
-      if (DUAL) {
-        for (int c = 0; c < BN_MMA / 2; c += 32) {
-          uint32_t gr[32], ur[32];
-          tmem_ld_32x32b_x32(tbase + c, gr);
-          tmem_ld_32x32b_x32(tbase + BN_MMA / 2 + c, ur);
-          tmem_ld_wait();
-          if (r < rows_valid && col0 + c < p.N) {
-            uint32_t packed[16];
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              const float h0 = act_fn(p.act, __uint_as_float(gr[2 * jj])) * __uint_as_float(ur[2 * jj]);
-              const float h1 = act_fn(p.act, __uint_as_float(gr[2 * jj + 1])) * __uint_as_float(ur[2 * jj + 1]);
-              packed[jj] = pack_bf16x2(h0, h1);
-            }
-            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(a_row + r) * p.N + col0 + c;
-            if (col0 + c + 32 <= p.N) {
-              uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-              for (int jj = 0; jj < 4; ++jj)
-                d4[jj] = make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]);
-            } else {
-              const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(packed);
-              for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj) dst[jj] = hv[jj];
-            }
-          }
-        }
-      } else {
-        int dest = -1;
-        float scale = 1.f;
-        if (r < rows_valid) {
-          const int src = a_row + r;
+      int dest = -1;
+      float scale = 1.f;
+      if (r < rows_valid) {
+        const int src = a_row + r;
+        if (DUAL) {
+          dest = src;
+        } else {
           dest = p.row_map ? p.row_map[src] : src;
           if (dest < 0 || dest >= p.rows_single) {  // output rows number the A rows: a bad map entry is skipped
             record_status(p.status, MOE_ERR_DEVICE_INDEX);
@@ -382,52 +446,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             scale = p.row_scale ? p.row_scale[dest] : 1.f;
           }
         }
-        // this thread's row of the warp's staging area (32 rows x kOutPitch bytes)
-        uint8_t* srow = out_stage + (q * 32 + lane) * kOutPitch;
-        for (int c = 0; c < BN_MMA; c += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tbase + c, v);
-          tmem_ld_wait();
-          if (dest >= 0 && col0 + c < p.N && p.out_bf16) {  // bf16 rows (expert outputs of the tensor-core layer)
-            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(dest) * p.N + col0 + c;
-            if (col0 + c + 32 <= p.N) {  // a full 64-byte row segment: staged, then one bulk store
-              bulk_wait_read();
-              uint4* s4 = reinterpret_cast<uint4*>(srow);
-#pragma unroll
-              for (int jj = 0; jj < 4; ++jj)
-                s4[jj] = make_uint4(pack_bf16x2(scale * __uint_as_float(v[8 * jj]), scale * __uint_as_float(v[8 * jj + 1])),
-                                    pack_bf16x2(scale * __uint_as_float(v[8 * jj + 2]), scale * __uint_as_float(v[8 * jj + 3])),
-                                    pack_bf16x2(scale * __uint_as_float(v[8 * jj + 4]), scale * __uint_as_float(v[8 * jj + 5])),
-                                    pack_bf16x2(scale * __uint_as_float(v[8 * jj + 6]), scale * __uint_as_float(v[8 * jj + 7])));
-              fence_proxy_async_smem();
-              bulk_store<64>(dst, smem_addr(srow));
-            } else {
-              for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj)
-                dst[jj] = __float2bfloat16_rn(scale * __uint_as_float(v[jj]));
-            }
-          } else if (dest >= 0 && col0 + c < p.N) {
-            float* dst = p.out_f32 + ks * p.part_stride + static_cast<size_t>(dest) * p.N + col0 + c;
-            if (col0 + c + 32 <= p.N) {  // a full 128-byte row segment: staged, then one bulk store
-              bulk_wait_read();          // the previous segment has left the staging row
-              float4* s4 = reinterpret_cast<float4*>(srow);
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj)
-                s4[jj] = make_float4(scale * __uint_as_float(v[4 * jj]), scale * __uint_as_float(v[4 * jj + 1]),
-                                     scale * __uint_as_float(v[4 * jj + 2]), scale * __uint_as_float(v[4 * jj + 3]));
-              fence_proxy_async_smem();
-              bulk_store<128>(dst, smem_addr(srow));
-            } else {
-              for (int jj = 0; jj < 32 && col0 + c + jj < p.N; ++jj) dst[jj] = scale * __uint_as_float(v[jj]);
-            }
-          }
-        }
       }
+      epilogue_tile<DUAL, BN_MMA>(p, tbase, out_stage + q * 32 * kOutPitch, dest, scale, col0, ks);
       }  // row tiles of the item
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&aux.tempty[acc]);
     }
-    if (!DUAL) bulk_wait_all();  // every staged row segment is stored before the CTA ends
   }
 
   tc_fence_before();
@@ -435,6 +460,237 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && aux.abort) record_status(p.status, MOE_ERR_TIMEOUT);
+  if (p.head_mult > 0) pdl_wait();  // complete only after the pair kernel (see above)
+}
+
+// ------------------------------------------------------------------ CTA-pair kernel
+// For compute-bound launches: the full 256-row tiles of each group run on
+// pairs of CTAs (clusters of two) that share one tcgen05.mma.cta_group::2 of
+// M = 256, N = 256.  CTA r of a pair loads rows [128 r, 128 r + 128) of the
+// tile's A rows and 128 rows of B: in dual mode CTA 0 the W_gate rows and CTA 1
+// the same W_up rows (TMEM columns [0,128) are then gate, [128,256) up); in
+// single mode rows [128 r, 128 r + 128) of the 256 output columns.  Per MMA
+// flop each CTA stages half the B bytes of the single-CTA 128 x 256 tile.  Both
+// CTAs' loads complete on CTA 0's stage barrier (CTA 0 expects both CTAs'
+// bytes); CTA 0's MMA thread issues the MMAs and its commits arrive on the
+// stage-empty and accumulator-full barriers of both CTAs; each CTA's epilogue
+// drains its own 128 TMEM lanes (epilogue_tile) and arrives on CTA 0's
+// accumulator-empty barrier.  No load is multicast.  The rows of a group past
+// its last full 256-row tile are left to the single-CTA kernel (head_mult).
+constexpr int PAIR_M = 256;
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_B_BYTES = 128 * BK * 2;
+constexpr int PAIR_STAGE_BYTES = A_BYTES + PAIR_B_BYTES;
+constexpr uint32_t PAIR_TMEM_COLS = 512;  // two accumulators of 256 columns
+
+constexpr size_t pair_smem_bytes() {
+  return 1024 + static_cast<size_t>(PAIR_STAGES) * PAIR_STAGE_BYTES + (sizeof(Aux<PAIR_STAGES>) + 127) / 128 * 128 +
+         kOutStage;
+}
+
+// Item w of the pair kernel -> group g, 256-row tile mt, column tile nt.
+template <typename AuxT>
+__device__ __forceinline__ void decode_pair_item(const AuxT& aux, int G, int w, int& g, int& mt, int& nt) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (aux.item_off[mid] <= w)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  g = lo;
+  const int tiles = aux.cnt[g] / PAIR_M;
+  const int local = w - aux.item_off[g];
+  nt = local / tiles;
+  mt = local - nt * tiles;
+}
+
+template <bool DUAL>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
+                             const __grid_constant__ CUtensorMap mapB1, const KParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Aux<PAIR_STAGES>& aux = *reinterpret_cast<Aux<PAIR_STAGES>*>(smem + PAIR_STAGES * PAIR_STAGE_BYTES);
+  uint8_t* out_stage = smem + PAIR_STAGES * PAIR_STAGE_BYTES + ((sizeof(Aux<PAIR_STAGES>) + 127) / 128) * 128;
+  volatile int* abort_flag = &aux.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: the CTA that issues the MMAs
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(&aux.full[s], 1);
+      mbar_init(&aux.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&aux.tfull[b], 1);
+      mbar_init(&aux.tempty[b], 8);  // the four epilogue warps of both CTAs
+    }
+    mbar_init(&aux.done, 1);
+    aux.abort = 0;
+    fence_mbar_init();
+  } else if (threadIdx.x == 32) {
+    prefetch_tensormap(&mapA);
+    prefetch_tensormap(&mapB0);
+    if (DUAL) prefetch_tensormap(&mapB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&aux.tmem_base, PAIR_TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  pdl_wait();
+  pdl_trigger();  // after the wait: the tail launch relies on this grid having waited for its predecessors
+  for (int g = threadIdx.x; g < p.G; g += THREADS) {
+    const int o0 = p.offsets ? p.offsets[g] : 0;
+    const int o1 = p.offsets ? p.offsets[g + 1] : p.rows_single;
+    const int r0 = min(max(o0, 0), p.rows_single), r1 = min(max(o1, r0), p.rows_single);
+    if (r0 != o0 || r1 != o1) record_status(p.status, MOE_ERR_DEVICE_INDEX);
+    aux.row_off[g] = r0;
+    aux.cnt[g] = (r1 - r0) / PAIR_M * PAIR_M;
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of work items per group; lane owns groups [8*lane, 8*lane+8)
+    int v[8], local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int g = lane * 8 + i;
+      v[i] = g < p.G ? (aux.cnt[g] / PAIR_M) * p.n_tiles : 0;
+      local += v[i];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    int run = incl - local;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int g = lane * 8 + i;
+      if (g < p.G) aux.item_off[g] = run;
+      run += v[i];
+    }
+    if (lane == 31) aux.item_off[p.G] = incl;
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers and TMEM are ready before any load, MMA or remote arrive
+  tc_fence_after();
+
+  const uint32_t tmem_base = aux.tmem_base;
+  const int total = aux.item_off[p.G];
+  const int nkb = (p.Kdim + BK - 1) / BK;
+  const long long limit = p.wait_limit;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer (both CTAs)
+      uint32_t kbg = 0, outstanding = 0, out_phase = 0;
+      const uint64_t pol_a = l2_policy_evict_last();    // activation rows: read by every column tile
+      const uint64_t pol_b = l2_policy_evict_normal();  // weight tiles: read by each row tile of the group
+      const CUtensorMap* mb = (DUAL && rank == 1) ? &mapB1 : &mapB0;
+      for (int w = pair; w < total && !*abort_flag; w += npairs) {
+        int g, mt, nt;
+        decode_pair_item(aux, p.G, w, g, mt, nt);
+        const int a_row = aux.row_off[g] + mt * PAIR_M + static_cast<int>(rank) * BM;
+        const int b_row = g * p.N + nt * p.col_step + (DUAL ? 0 : static_cast<int>(rank) * 128);
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = kbg % PAIR_STAGES;
+          const uint32_t ph = (kbg / PAIR_STAGES) & 1u;
+          if (!mbar_wait_bounded(&aux.empty[s], ph ^ 1u, limit, abort_flag)) break;
+          outstanding &= ~(1u << s);
+          uint8_t* sa = smem + s * PAIR_STAGE_BYTES;
+          const uint32_t full_s = cluster_addr(&aux.full[s], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&aux.full[s], 2 * PAIR_STAGE_BYTES);
+          tma_load_2d_pair(sa, &mapA, full_s, kb * BK, a_row, pol_a);
+          tma_load_2d_pair(sa + A_BYTES, mb, full_s, kb * BK, b_row, pol_b);
+          outstanding |= 1u << s;
+          out_phase = (out_phase & ~(1u << s)) | (ph << s);
+        }
+      }
+      if (*abort_flag && rank == 0) {  // let issued copies land before the pair exits
+        for (int s = 0; s < PAIR_STAGES; ++s)
+          if (outstanding & (1u << s)) wait_cycles(&aux.full[s], (out_phase >> s) & 1u, limit);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (CTA 0 of the pair)
+      const uint32_t idesc = idesc_bf16_f32(PAIR_M, 256);
+      uint32_t kbg = 0;
+      int it = 0;
+      for (int w = pair; w < total; w += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_ph = (it >> 1) & 1u;
+        if (!mbar_wait_bounded(&aux.tempty[acc], acc_ph ^ 1u, limit, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * 256;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = kbg % PAIR_STAGES;
+          const uint32_t ph = (kbg / PAIR_STAGES) & 1u;
+          if (!mbar_wait_bounded(&aux.full[s], ph, limit, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(smem + s * PAIR_STAGE_BYTES);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair(&aux.empty[s], 0x3);
+        }
+        if (!ok) break;
+        umma_commit_pair(&aux.tfull[acc], 0x3);
+      }
+      umma_commit_pair(&aux.done, 0x3);  // every MMA issued above completes before TMEM is released
+      wait_cycles(&aux.done, 0, limit);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int it = 0;
+    for (int w = pair; w < total; w += npairs, ++it) {
+      int g, mt, nt;
+      decode_pair_item(aux, p.G, w, g, mt, nt);
+      const int acc = it & 1;
+      const uint32_t acc_ph = (it >> 1) & 1u;
+      const bool ok = mbar_wait_bounded(&aux.tfull[acc], acc_ph, limit, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int src = aux.row_off[g] + mt * PAIR_M + static_cast<int>(rank) * BM + r;  // full tiles: every row valid
+      int dest = src;
+      float scale = 1.f;
+      if (!DUAL) {
+        dest = p.row_map ? p.row_map[src] : src;
+        if (dest < 0 || dest >= p.rows_single) {
+          record_status(p.status, MOE_ERR_DEVICE_INDEX);
+          dest = -1;
+        } else {
+          scale = p.row_scale ? p.row_scale[dest] : 1.f;
+        }
+      }
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256;
+      epilogue_tile<DUAL, 256>(p, tbase, out_stage + q * 32 * kOutPitch, dest, scale, nt * p.col_step, 0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_addr(&aux.tempty[acc], 0));
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();  // both CTAs are done with each other's barriers, shared memory and TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, PAIR_TMEM_COLS);
   }
   if (threadIdx.x == 0 && aux.abort) record_status(p.status, MOE_ERR_TIMEOUT);
 }
@@ -469,9 +725,33 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+KParams make_params(const Ctx& c, const GemmArgs& a, int col_step, int head_mult) {
+  KParams p;
+  p.offsets = a.offsets;
+  p.G = a.G;
+  const int nkb = (a.Kdim + BK - 1) / BK;
+  p.ksplit = effective_ksplit(a.ksplit, a.Kdim);
+  p.kb_per_split = (nkb + p.ksplit - 1) / p.ksplit;
+  p.part_stride = a.part_stride;
+  p.rows_single = static_cast<int>(a.rows_A);
+  p.N = a.N;
+  p.Kdim = a.Kdim;
+  p.col_step = col_step;
+  p.n_tiles = (a.N + p.col_step - 1) / p.col_step;
+  p.act = a.act;
+  p.out_bf16 = a.out_bf16;
+  p.out_f32 = a.out_f32;
+  p.row_map = a.row_map;
+  p.row_scale = a.row_scale;
+  p.status = c.status;
+  p.wait_limit = c.wait_limit;
+  p.skip_stage = c.skip_stage;
+  p.head_mult = head_mult;
+  return p;
+}
+
 template <bool DUAL, int BN, int MT>
-cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int max_items_per_sm_hint) {
-  (void)max_items_per_sm_hint;
+cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int head_mult = 0) {
   CUtensorMap mA, mB0, mB1;
   const uint32_t brows = DUAL ? BN / 2 : BN;
   if (!make_map(&mA, a.A, static_cast<uint64_t>(a.rows_A), static_cast<uint64_t>(a.Kdim), BM) ||
@@ -483,27 +763,11 @@ cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int max_items_per_sm_h
   } else {
     mB1 = mB0;
   }
-  KParams p;
-  p.offsets = a.offsets;
-  p.G = a.G;
-  const int nkb = (a.Kdim + BK - 1) / BK;
-  p.ksplit = effective_ksplit(a.ksplit, a.Kdim);
-  p.kb_per_split = (nkb + p.ksplit - 1) / p.ksplit;
-  p.part_stride = a.part_stride;
-  p.rows_single = static_cast<int>(a.rows_A);
-  p.N = a.N;
-  p.Kdim = a.Kdim;
-  p.col_step = DUAL ? BN / 2 : BN;
-  p.n_tiles = (a.N + p.col_step - 1) / p.col_step;
-  p.act = a.act;
-  p.out_bf16 = a.out_bf16;
-  p.out_f32 = a.out_f32;
-  p.row_map = a.row_map;
-  p.row_scale = a.row_scale;
-  p.status = c.status;
-  p.wait_limit = c.wait_limit;
-  p.skip_stage = c.skip_stage;
-  const long long tiles_bound = static_cast<long long>(a.max_rows) / BM + std::min(a.G, a.max_rows);
+  const KParams p = make_params(c, a, DUAL ? BN / 2 : BN, head_mult);
+  // rows left after the pair kernel's full tiles: fewer than head_mult per group
+  const long long rows = head_mult > 0 ? std::min<long long>(a.max_rows, static_cast<long long>(a.G) * (head_mult - 1))
+                                       : a.max_rows;
+  const long long tiles_bound = rows / BM + std::min<long long>(a.G, rows);
   const long long items_bound = tiles_bound * p.n_tiles * p.ksplit;
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(c.num_sms, items_bound)));
   auto kern = grouped_gemm_kernel<DUAL, BN, MT>;
@@ -512,6 +776,57 @@ cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int max_items_per_sm_h
   if (e != cudaSuccess) return e;
   KernelScope ks(c, a.name ? a.name : (DUAL ? "grouped_gemm_dual" : "grouped_gemm"));
   return launch_kernel(c, kern, dim3(grid), dim3(THREADS), smem_bytes<BN, MT>(), mA, mB0, mB1, p);
+}
+
+// Clusters of two that fit on the device at once (0 if none), once per device and kernel.
+template <bool DUAL>
+int pair_clusters(const Ctx& c) {
+  static std::atomic<int> cached[kMaxPairDevices];
+  static std::atomic<bool> init[kMaxPairDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxPairDevices) return 0;
+  if (init[dev].load()) return cached[dev].load();
+  auto kern = grouped_gemm_pair_kernel<DUAL>;
+  int n = 0;
+  if (allow_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(pair_smem_bytes())) == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * (c.num_sms / 2));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = pair_smem_bytes();
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cached[dev].store(n);
+  init[dev].store(true);
+  return n;
+}
+
+// The full 256-row tiles of every group on CTA pairs (M = 256, N = 256 per
+// MMA), then the rows left in each group on the single-CTA kernel.
+template <bool DUAL>
+cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, int clusters) {
+  CUtensorMap mA, mB0, mB1;
+  if (!make_map(&mA, a.A, static_cast<uint64_t>(a.rows_A), static_cast<uint64_t>(a.Kdim), BM) ||
+      !make_map(&mB0, a.B0, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), 128))
+    return cudaErrorInvalidValue;
+  if (DUAL) {
+    if (!make_map(&mB1, a.B1, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), 128))
+      return cudaErrorInvalidValue;
+  } else {
+    mB1 = mB0;
+  }
+  const KParams p = make_params(c, a, DUAL ? 128 : 256, 0);
+  const long long items_bound = static_cast<long long>(a.max_rows / PAIR_M) * p.n_tiles;
+  const int pairs = static_cast<int>(std::max(1LL, std::min<long long>(clusters, items_bound)));
+  auto kern = grouped_gemm_pair_kernel<DUAL>;
+  {
+    KernelScope ks(c, a.name ? a.name : (DUAL ? "grouped_gemm_dual" : "grouped_gemm"));
+    const cudaError_t e = launch_kernel(c, kern, dim3(2 * pairs), dim3(THREADS), pair_smem_bytes(), mA, mB0, mB1, p);
+    if (e != cudaSuccess) return e;
+  }
+  GemmArgs tail = a;
+  if (a.name) tail.name = DUAL ? "expert_gate_up_gemm_tail" : "expert_down_gemm_tail";
+  return launch_tiled<DUAL, 256, 1>(c, tail, PAIR_M);
 }
 
 }  // namespace
@@ -528,7 +843,7 @@ double wave_waste(double items, int sms) {
 // compute-bound shapes, where they halve the A-tile traffic per flop.
 cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   if (a.G <= 0 || a.max_rows <= 0 || a.N <= 0 || a.rows_A <= 0) return cudaSuccess;
-  if (a.G > MAX_G) return cudaErrorInvalidValue;
+  if (a.G > MAX_G || a.N % 32) return cudaErrorInvalidValue;  // the epilogue writes whole 16-byte column chunks
   const int groups = std::min(a.G, a.max_rows);
   const double rows_per_group = static_cast<double>(a.max_rows) / groups;
   // about half an M tile of padding per group
@@ -542,15 +857,20 @@ cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   // tiles covering two row tiles per item, so each item is twice as long and each weight tile is loaded once per
   // group.  The gate/up projection keeps one row tile per item: its long K rows already share weight tiles
   // through L2 between the CTAs running a group's row tiles side by side, and it keeps 6 stages.
-  if (!a.dual && memory_bound && rows_per_group > 96.0) return launch_tiled<false, 128, 2>(c, a, 0);
+  if (!a.dual && memory_bound && rows_per_group > 96.0) return launch_tiled<false, 128, 2>(c, a);
   // at most 128 output columns (the router: N = E): a 256-column tile would be three quarters zero fill
-  if (!a.dual && a.N <= 128) return launch_tiled<false, 128, 1>(c, a, 0);
+  if (!a.dual && a.N <= 128) return launch_tiled<false, 128, 1>(c, a);
+  // compute-bound launches with at least one full 256-row tile: CTA pairs for the full tiles
+  if (!memory_bound && a.ksplit <= 1 && a.max_rows >= PAIR_M && pair_gemm_enabled()) {
+    const int clusters = a.dual ? pair_clusters<true>(c) : pair_clusters<false>(c);
+    if (clusters > 0) return a.dual ? launch_pair<true>(c, a, clusters) : launch_pair<false>(c, a, clusters);
+  }
   // narrow tiles waste less of the last wave, but every column tile re-reads the activation rows: with more than
   // 96 rows per group (activations well beyond L2 on such launches) the dual launch keeps wide tiles
   const bool narrow = memory_bound && !(a.dual && rows_per_group > 96.0) &&
                       wave_waste(items_wide, c.num_sms) - wave_waste(items_narrow, c.num_sms) > 0.03;
-  if (a.dual) return narrow ? launch_tiled<true, 128, 1>(c, a, 0) : launch_tiled<true, 256, 1>(c, a, 0);
-  return narrow ? launch_tiled<false, 128, 1>(c, a, 0) : launch_tiled<false, 256, 1>(c, a, 0);
+  if (a.dual) return narrow ? launch_tiled<true, 128, 1>(c, a) : launch_tiled<true, 256, 1>(c, a);
+  return narrow ? launch_tiled<false, 128, 1>(c, a) : launch_tiled<false, 256, 1>(c, a);
 }
 
 }  // namespace moe

@@ -66,6 +66,7 @@ struct GemmArgs {
   size_t part_stride = 0;  // f32 results go to out_f32 + range * part_stride (summed by the caller)
 };
 cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a);
+bool pair_gemm_enabled();  // moe_set_pair_gemm
 
 // The number of K ranges a split request really produces for a reduction of
 // Kdim: at most one per 64-wide k-block, and no empty range.  The caller sums

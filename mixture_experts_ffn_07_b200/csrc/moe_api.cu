@@ -2,7 +2,7 @@
 // workspace layout, the order of kernel launches for each entry point, the
 // device status word, and the host-side launch counter and event trace.
 //
-// Path choice: bf16 activations with bf16 expert weights and T > 64 take the
+// Path choice: bf16 activations with bf16 expert weights and T >= 65 (moe_set_tensor_min_tokens) take the
 // tensor-core path (row gather + tcgen05 grouped GEMMs); everything else takes
 // the weight-streaming path (expert-major GEMV kernels), which reads each
 // touched expert's weights once and is the bandwidth-optimal form for small T.
@@ -38,6 +38,7 @@ std::atomic<int> g_skip_stage{0};
 std::atomic<long long> g_barrier_delay{0};
 std::atomic<int> g_fused_decode{1};
 std::atomic<int> g_fused_front{1};
+std::atomic<int> g_pair_gemm{1};
 
 struct TraceRec {
   const char* name;
@@ -81,10 +82,15 @@ inline size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255);
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool tensor_path(const moe_desc& d) { return d.act_dtype == MOE_BF16 && d.w_dtype == MOE_BF16 && d.T > 64; }
+// Fewest tokens for which a bf16 layer takes the tensor-core path (moe_set_tensor_min_tokens).
+std::atomic<int> g_tensor_min_tokens{65};
+
+bool tensor_path(const moe_desc& d) {
+  return d.act_dtype == MOE_BF16 && d.w_dtype == MOE_BF16 && d.T >= g_tensor_min_tokens.load();
+}
 
 bool tensor_router(const moe_desc& d) {
-  return d.act_dtype == MOE_BF16 && d.router_dtype == MOE_BF16 && d.T > 64 && d.E % 32 == 0;
+  return d.act_dtype == MOE_BF16 && d.router_dtype == MOE_BF16 && d.T >= g_tensor_min_tokens.load() && d.E % 32 == 0;
 }
 
 // Selection, permutation and row gather as one cooperative kernel after the
@@ -414,6 +420,8 @@ cudaError_t allow_dynamic_smem(const void* kernel, int bytes) {
 // Every launch also opens an NVTX range named after its kernel, so a profiler's
 // timeline groups the launches by step; without a profiler attached the NVTX
 // calls return at once.
+bool pair_gemm_enabled() { return g_pair_gemm.load() != 0; }
+
 KernelScope::KernelScope(const Ctx& c, const char* name) : ctx(c), slot(-1) {
   g_launches.fetch_add(1);
   nvtxRangePushA(name);
@@ -804,5 +812,9 @@ void moe_debug_set_barrier_delay(int64_t cycles) { g_barrier_delay.store(cycles 
 void moe_set_fused_decode(int enable) { g_fused_decode.store(enable ? 1 : 0); }
 
 void moe_set_fused_front(int enable) { g_fused_front.store(enable ? 1 : 0); }
+
+void moe_set_pair_gemm(int enable) { g_pair_gemm.store(enable ? 1 : 0); }
+
+void moe_set_tensor_min_tokens(int tokens) { g_tensor_min_tokens.store(std::max(1, tokens)); }
 
 }  // extern "C"

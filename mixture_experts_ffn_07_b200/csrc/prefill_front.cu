@@ -33,7 +33,7 @@ constexpr int kWarps = kThreads / 32;
 // positions of this CTA's pairs (B)
 constexpr int kPosOff = kWarps * 256 * 4 + 2 * kThreads * 4;
 
-__device__ unsigned g_front_barrier;
+__device__ unsigned long long g_front_barrier;
 
 struct FrontArgs {
   const float* parts;  // split-K partial logits (nparts > 0) or nullptr
@@ -247,8 +247,12 @@ cudaError_t launch_prefill_front(const Ctx& c, const PrefillFront& f) {
   const long long max_pairs = (static_cast<long long>(f.T) + grid - 1) / grid * f.K;
   a.pos_cap = kPosOff + max_pairs * 4 <= c.smem_optin ? static_cast<int>(max_pairs) : 0;
   const int smem = std::max(c.smem_optin / 2 + 1024, kPosOff + a.pos_cap * 4);
-  const cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(front_kernel), smem);
+  cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(front_kernel), smem);
   if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, front_kernel, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm != 1) return cudaErrorInvalidValue;  // the separate launches run instead
   KernelScope ks(c, "route_permute_gather");
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);

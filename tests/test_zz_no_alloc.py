@@ -28,6 +28,9 @@ def _noalloc(desc, x, w, out):
 
 @pytest.mark.parametrize("spec", [
     workloads.Spec(T=200, H=256, E=16, I=128, K=4, shared_I=64, shared_gated=True, name="noalloc_tensor"),
+    # E % 32 == 0 and T > 64: the tensor-core router with split-K partials and the fused selection / permutation
+    # / gather kernel, whose partial-logit and count regions of the static scratch then hold the first call's data
+    workloads.Spec(T=200, H=256, E=32, I=128, K=4, shared_I=64, shared_gated=True, name="noalloc_tensor_front"),
     workloads.Spec(T=16, H=2048, E=128, I=768, K=8, act_dtype="f32", w_dtype="q8_0", router_dtype="f32",
                    name="noalloc_q8_decode"),
 ], ids=lambda s: s.name)
