@@ -386,12 +386,38 @@ void moe_set_fused_front(int enable);
  * Process-wide; takes effect at the next call. */
 void moe_set_pair_gemm(int enable);
 
+/* How the cooperative decode kernel (moe_set_fused_decode) runs gate/up and
+ * down: mode = 1 (default) runs them for f32 and bf16 weights as one stream of
+ * work items (32 weight rows each, fed through the copy engine into a ring of
+ * 32 KB stages per CTA, taken from a device-wide queue that hands out all
+ * gate/up items, expert by expert, before the down items; a down item waits
+ * only for its own expert's gate/up items), and for the other formats as two
+ * phases separated by a grid barrier, each CTA streaming a contiguous slice of
+ * the rows; mode = 2 also streams Q8_0 (measured slower than its two phases);
+ * mode = 0 runs every format as two phases.  Same routing and the same values
+ * up to the order of f32 additions.  Shapes whose weight rows cannot be mapped
+ * for the copy engine (Q8_0 with K % 256 != 0, misaligned pointers) take the
+ * two phases by themselves.  Process-wide; takes effect at the next call. */
+void moe_set_decode_stream(int mode);
+
+/* How the tensor-core path feeds the routed gate/up GEMM its x rows in expert
+ * order: enable = 0 (default) first copies them into a workspace array of
+ * P x H bf16 rows (in the fused selection kernel, or a gather kernel), which
+ * the GEMM reads with 128-row box loads; 1 gathers them inside the GEMM, each
+ * pair's row straight from x by the copy engine (tile::gather4 loads of four
+ * rows, 32 per 128-row tile and k-block), which saves the copy's traffic and
+ * workspace but measured slower on B200 (the skewed layer's gate/up GEMM
+ * 3.0 -> 7.4 ms: the copy engine's cost per small load bounds it).  Same values.
+ * moe_workspace_bytes follows the current setting (the copy needs
+ * P * H * 2 more bytes), so size workspaces after changing it.  Process-wide. */
+void moe_set_tma_gather(int enable);
+
 /* The fewest tokens for which a bf16 layer (bf16 activations and expert
  * weights) takes the tensor-core path (router GEMM, grouped tcgen05 GEMMs)
- * instead of the weight-streaming path; default 65 (the streaming path for
- * 1..64 tokens).  Values below 1 count as 1.  moe_workspace_bytes follows the
- * current setting, so size workspaces after changing it.  Process-wide; for
- * measuring where the two paths cross. */
+ * instead of the weight-streaming path; default 8 (the streaming path for 1..7
+ * tokens), where the two paths cross on B200 (between 2 and 8 tokens on the
+ * measured shapes).  Values below 1 count as 1.  moe_workspace_bytes follows
+ * the current setting, so size workspaces after changing it.  Process-wide. */
 void moe_set_tensor_min_tokens(int tokens);
 
 #ifdef __cplusplus

@@ -227,9 +227,22 @@ def set_pair_gemm(enable: bool) -> None:
     _lib.lib().moe_set_pair_gemm(int(enable))
 
 
+def set_decode_stream(mode) -> None:
+    """moe_set_decode_stream: gate/up and down of the cooperative decode kernel as one TMA-fed stream of
+    work items for f32 / bf16 weights (1 or True, default), for Q8_0 too (2), or two phases with a grid
+    barrier for every format (0 or False)."""
+    _lib.lib().moe_set_decode_stream(int(mode))
+
+
+def set_tma_gather(enable: bool) -> None:
+    """moe_set_tma_gather: the routed gate/up GEMM gathers its x rows with the copy engine (True) or
+    reads a copy of them in expert order (False, default); size workspaces after changing it."""
+    _lib.lib().moe_set_tma_gather(int(enable))
+
+
 def set_tensor_min_tokens(tokens: int) -> None:
     """moe_set_tensor_min_tokens: bf16 layers of at least `tokens` tokens take the tensor-core path
-    (default 65); size workspaces after changing it."""
+    (default 8); size workspaces after changing it."""
     _lib.lib().moe_set_tensor_min_tokens(int(tokens))
 
 

@@ -23,7 +23,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_workspace_bytes", "moe_route
            "moe_combine", "moe_layer", "moe_layer_host", "moe_layer_noalloc", "moe_q8_0_split",
            "moe_last_device_status", "moe_launch_count", "moe_trace_enable", "moe_trace_read",
            "moe_debug_set_wait_limit", "moe_debug_set_skip_stage", "moe_set_fused_decode",
-           "moe_workspace_regions", "moe_set_fused_front", "moe_set_pair_gemm", "moe_set_tensor_min_tokens", "moe_combine_backward", "moe_act_up_backward",
+           "moe_workspace_regions", "moe_set_fused_front", "moe_set_pair_gemm", "moe_set_decode_stream", "moe_set_tma_gather", "moe_set_tensor_min_tokens", "moe_combine_backward", "moe_act_up_backward",
            "moe_q6_k_split", "moe_debug_set_barrier_delay")
 
 
@@ -99,6 +99,10 @@ def lib():
         L.moe_set_fused_front.restype = None
         L.moe_set_pair_gemm.argtypes = [I32]
         L.moe_set_pair_gemm.restype = None
+        L.moe_set_decode_stream.argtypes = [I32]
+        L.moe_set_decode_stream.restype = None
+        L.moe_set_tma_gather.argtypes = [I32]
+        L.moe_set_tma_gather.restype = None
         L.moe_set_tensor_min_tokens.argtypes = [I32]
         L.moe_set_tensor_min_tokens.restype = None
         L.moe_workspace_regions.argtypes = [DP, ctypes.POINTER(MoeWsRegions)]

@@ -28,6 +28,9 @@
 // only one such grid runs on a device at a time and one counter serves all.
 #include <atomic>
 
+#include <mutex>
+
+#include "decode_stream.cuh"
 #include "route_util.cuh"
 #include "stream_core.cuh"
 
@@ -69,7 +72,15 @@ struct DecodeArgs {
   int* status;
   long long wait_limit;
   long long barrier_delay;
+  int tma;                 // gate/up and down as one TMA-fed stream (decode_stream.cuh), else the two phases
+  dstream::Sync* sync;     // queue and per-group counters of the stream (workspace)
 };
+
+// The stream instance of a weight format: one format for gate/up and down, f32, bf16 or Q8_0.
+template <int WKG, int WKD>
+__host__ __device__ constexpr bool stream_format() {
+  return WKG == WKD && (WKG == WK_F32 || WKG == WK_BF16 || WKG == WK_Q8);
+}
 
 __device__ __forceinline__ bool cta_grid_sync(const DecodeArgs& a, int* s_abort, int* s_flag) {
   return grid_sync(&g_decode_barrier, a.wait_limit, a.status, s_abort, s_flag);
@@ -153,7 +164,8 @@ __device__ __forceinline__ void router_stage_x(const DecodeArgs& a, float* xs, i
 
 // MAXT: the most tokens of one expert batch (1 when T = 1: only single-token code, more loads in flight).
 template <typename XT, int WKG, int WKD, int MAXT>
-__global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_layer_kernel(const DecodeArgs a, const __grid_constant__ dstream::Maps maps) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_expert[kMaxGroups], s_first[kMaxGroups], s_count[kMaxGroups], s_poff[kMaxGroups + 1];
   __shared__ long long s_coff[kMaxGroups + 1];
@@ -165,6 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
   __shared__ float s_part[kMaxUnits * kMaxTok * 2];
   __shared__ int s_warp[8];
   __shared__ int s_n, s_flag, s_abort;
+  __shared__ int s_gi[kMaxGroups + 1], s_di[kMaxGroups + 1];
+  __shared__ dstream::Ring s_ring;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = a.T, E = a.E, K = a.K, P = T * K;
   const int R = E + (a.w_s ? 1 : 0);
@@ -184,6 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     s_ph[1].src[0].row_scale = s_w;
     s_ph[1].src[1].row_scale = a.w_s ? s_sgate : nullptr;
   }
+
+  if (blockIdx.x == 0 && a.tma)  // the stream's queue and counters start at zero (visible after the barrier)
+    for (int i = threadIdx.x; i < 1 + dstream::kMaxGroups; i += blockDim.x) reinterpret_cast<unsigned*>(a.sync)[i] = 0;
 
   // ---- R: partial router logits; a CTA item is (hidden chunk, token group, block of kWarps rows)
   {
@@ -335,27 +352,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     __syncthreads();
   }
 
-  // ---- G: gate/up
-  {
-    const Tables tb{s_expert, s_first, s_count, s_poff, s_coff, s_n};
-    if (warp == 0) build_prefix(tb, s_ph[0]);
-    __syncthreads();
-    int p0, p1;
-    cta_pairs(tb, s_ph[0], p0, p1);
-    if (!s_abort) run_phase<XT, WKG, true, MAXT>(s_ph[0], tb, p0, p1, sm);
+  bool ok;
+  bool streamed = false;
+  if constexpr (stream_format<WKG, WKD>()) {
+    if (a.tma) {
+      // ---- G + D as one stream of items (decode_stream.cuh); then one barrier before the combine
+      constexpr int NT = MAXT == 1 ? 1 : 4;
+      dstream::Params dp;
+      dp.H = a.H;
+      dp.K = a.K;
+      dp.I = a.g.plan[0].Nout;
+      dp.Is = a.has_shared ? a.g.plan[1].Nout : 0;
+      dp.act = a.g.act_fn;
+      dp.x = a.x;
+      dp.h = a.g.src[0].out;
+      dp.h_s = a.g.src[1].out;
+      dp.y_slots = a.d.src[0].out;
+      dp.y_s = a.d.src[1].out;
+      dp.sync = a.sync;
+      dp.wait_limit = a.wait_limit;
+      dp.status = a.status;
+      if (warp == 0) dstream::build_items<NT>(dp, s_expert, s_count, s_n, s_gi, s_di);
+      __syncthreads();
+      const dstream::Items its{s_expert, s_first, s_count, s_gi, s_di, s_n};
+      if (!s_abort) {
+        uint8_t* stages = smem + ((128u - (smem_addr(smem) & 127u)) & 127u);  // copy destinations: 128-aligned
+        const bool c_ok = dstream::run_stream<XT, WKG, NT>(maps, dp, its, stages, s_ring, s_sorted, s_w,
+                                                          a.w_s ? s_sgate : nullptr);
+        if (!c_ok) s_abort = 1;
+      }
+      ok = cta_grid_sync(a, &s_abort, &s_flag);
+      streamed = true;
+    }
   }
-  cta_grid_sync(a, &s_abort, &s_flag);
+  if (!streamed) {
+    // ---- G: gate/up
+    {
+      const Tables tb{s_expert, s_first, s_count, s_poff, s_coff, s_n};
+      if (warp == 0) build_prefix(tb, s_ph[0]);
+      __syncthreads();
+      int p0, p1;
+      cta_pairs(tb, s_ph[0], p0, p1);
+      if (!s_abort) run_phase<XT, WKG, true, MAXT>(s_ph[0], tb, p0, p1, sm);
+    }
+    cta_grid_sync(a, &s_abort, &s_flag);
 
-  // ---- D: down
-  {
-    const Tables tb{s_expert, s_first, s_count, s_poff, s_coff, s_n};
-    if (warp == 0) build_prefix(tb, s_ph[1]);
-    __syncthreads();
-    int p0, p1;
-    cta_pairs(tb, s_ph[1], p0, p1);
-    if (!s_abort) run_phase<float, WKD, false, MAXT>(s_ph[1], tb, p0, p1, sm);
+    // ---- D: down
+    {
+      const Tables tb{s_expert, s_first, s_count, s_poff, s_coff, s_n};
+      if (warp == 0) build_prefix(tb, s_ph[1]);
+      __syncthreads();
+      int p0, p1;
+      cta_pairs(tb, s_ph[1], p0, p1);
+      if (!s_abort) run_phase<float, WKD, false, MAXT>(s_ph[1], tb, p0, p1, sm);
+    }
+    ok = cta_grid_sync(a, &s_abort, &s_flag);
   }
-  const bool ok = cta_grid_sync(a, &s_abort, &s_flag);
 
   // ---- C: combine
   if (ok) {
@@ -412,8 +464,12 @@ int static_smem() {
 }
 
 template <typename XT, int WKG, int WKD, int MAXT>
-cudaError_t launch_fused_t(const Ctx& c, const DecodeArgs& a, int P) {
+cudaError_t launch_fused_t(const Ctx& c, const DecodeArgs& a0, int P, const dstream::Maps& maps) {
   auto kern = decode_layer_kernel<XT, WKG, WKD, MAXT>;
+  DecodeArgs a = a0;
+  if (!stream_format<WKG, WKD>()) a.tma = 0;
+  // the stream's per-warp rings reuse the stage area
+  if (a.tma) a.stage_bytes = std::max(a.stage_bytes, dstream::kRingBytes + 128);
   // more than half of an SM's shared memory, so one CTA per SM whatever the register count: a CTA of a later
   // grid then starts only after this grid's last barrier (the barrier counter is shared by all launches)
   const int smem = std::max(a.stage_bytes + 16 * P, c.smem_optin / 2 + 1024);
@@ -436,26 +492,108 @@ cudaError_t launch_fused_t(const Ctx& c, const DecodeArgs& a, int P) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  return cudaLaunchKernelEx(&cfg, kern, a, maps);
 }
 
 template <typename XT, int WKG, int WKD>
-cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P) {
-  if (a.T == 1) return launch_fused_t<XT, WKG, WKD, 1>(c, a, P);
-  return launch_fused_t<XT, WKG, WKD, kDecodeTok>(c, a, P);
+cudaError_t launch_fused(const Ctx& c, const DecodeArgs& a, int P, const dstream::Maps& maps) {
+  if (a.T == 1) return launch_fused_t<XT, WKG, WKD, 1>(c, a, P, maps);
+  return launch_fused_t<XT, WKG, WKD, kDecodeTok>(c, a, P, maps);
 }
 
 template <typename XT>
-cudaError_t launch_kinds(const Ctx& c, const DecodeArgs& a, int P, int wkg, int wkd) {
-  if (wkg == WK_F32) return launch_fused<XT, WK_F32, WK_F32>(c, a, P);
-  if (wkg == WK_BF16) return launch_fused<XT, WK_BF16, WK_BF16>(c, a, P);
-  if (wkg == WK_Q8) return launch_fused<XT, WK_Q8, WK_Q8>(c, a, P);
-  if (wkd == WK_Q6K) return launch_fused<XT, WK_Q4K, WK_Q6K>(c, a, P);
-  return launch_fused<XT, WK_Q4K, WK_Q4K>(c, a, P);
+cudaError_t launch_kinds(const Ctx& c, const DecodeArgs& a, int P, int wkg, int wkd, const dstream::Maps& maps) {
+  if (wkg == WK_F32) return launch_fused<XT, WK_F32, WK_F32>(c, a, P, maps);
+  if (wkg == WK_BF16) return launch_fused<XT, WK_BF16, WK_BF16>(c, a, P, maps);
+  if (wkg == WK_Q8) return launch_fused<XT, WK_Q8, WK_Q8>(c, a, P, maps);
+  if (wkd == WK_Q6K) return launch_fused<XT, WK_Q4K, WK_Q6K>(c, a, P, maps);
+  return launch_fused<XT, WK_Q4K, WK_Q4K>(c, a, P, maps);
 }
 
-cudaError_t launch_by_kind(const Ctx& c, const DecodeArgs& a, int P, bool x_f32, int wkg, int wkd) {
-  return x_f32 ? launch_kinds<float>(c, a, P, wkg, wkd) : launch_kinds<__nv_bfloat16>(c, a, P, wkg, wkd);
+cudaError_t launch_by_kind(const Ctx& c, const DecodeArgs& a, int P, bool x_f32, int wkg, int wkd,
+                           const dstream::Maps& maps) {
+  return x_f32 ? launch_kinds<float>(c, a, P, wkg, wkd, maps) : launch_kinds<__nv_bfloat16>(c, a, P, wkg, wkd, maps);
+}
+
+// ---- tensor maps of the stream, encoded once per (tensor, shape) and kept
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void* base;
+  int dtype;
+  uint64_t rows, cols;
+  uint32_t box_rows;
+  int dev;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && dtype == o.dtype && rows == o.rows && cols == o.cols && box_rows == o.box_rows &&
+           dev == o.dev;
+  }
+};
+
+// A row-major matrix [rows, cols] of `dtype` elements read in boxes of box_cols x box_rows
+// (zero fill past the edges).  The last few maps are kept, keyed by pointer, shape and box.
+bool stream_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int esize, uint64_t rows, uint64_t cols,
+                uint32_t box_cols, uint32_t box_rows) {
+  constexpr int kCache = 64;
+  static std::mutex mu;
+  static MapKey keys[kCache];
+  static CUtensorMap vals[kCache];
+  static int used = 0, next = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const MapKey key{base, static_cast<int>(dtype), rows, cols, box_cols * 1024u + box_rows, dev};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < used; ++i)
+      if (keys[i] == key) {
+        *m = vals[i];
+        return true;
+      }
+  }
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u) || (cols * esize) % 16) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * esize};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lk(mu);
+  keys[next] = key;
+  vals[next] = *m;
+  next = (next + 1) % kCache;
+  used = std::max(used, next == 0 ? kCache : next);
+  return true;
+}
+
+// Maps of one weight matrix [rows, K] (+ Q8_0 scale plane) for the stream; false if its layout does not fit
+// (rows too long for the 32-bit strides, scale rows not a multiple of 16 bytes, misaligned pointers).
+bool weight_maps(int wk, const void* w, const void* scale, uint64_t rows, uint64_t K, uint32_t box_rows,
+                 CUtensorMap* mw, CUtensorMap* ms) {
+  // a slot row: 256 elements of the map's type (f32, bf16, or Q8_0 codes as 32-bit words) and, for Q8_0, the
+  // 32 fp16 scales of those 1024 codes, one row per box
+  if (wk == WK_F32) return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, K, 256, box_rows);
+  if (wk == WK_BF16) return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 256, box_rows);
+  if (K % 256) return false;  // the fp16 scale rows (K / 16 bytes) must be whole 16-byte units
+  return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, rows, K / 4, 256, box_rows) &&
+         stream_map(ms, scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, K / 32, 32, box_rows);
 }
 
 }  // namespace
@@ -542,7 +680,29 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
   a.status = c.status;
   a.wait_limit = c.wait_limit;
   a.barrier_delay = c.barrier_delay;
-  return launch_by_kind(c, a, P, L.x_dtype == MOE_F32, wkg, wkd);
+  // gate/up and down as one TMA-fed stream: f32, bf16 or Q8_0 in both projections, every matrix mappable
+  dstream::Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  a.sync = static_cast<dstream::Sync*>(L.stream_sync);
+  // Q8_0 keeps the two phases: with ~1.5 tokens per expert its items are one or two stages long, and the
+  // stream's per-item and per-token work measured slower than the row-pair GEMV (q8_0_decode_t16: 315 against
+  // 233 us); moe_set_decode_stream(2) takes the stream for Q8_0 too
+  const int sw = stream_path_mode();
+  a.tma = L.stream_sync != nullptr && wkg == wkd && (wkg == WK_F32 || wkg == WK_BF16 || (wkg == WK_Q8 && sw == 2));
+  if (a.tma) {
+    using namespace dstream;
+    const uint64_t E = L.E, H = L.H, I = L.I, Is = L.Is;
+    constexpr uint32_t GR = kRows / 2, DR = kRows;  // boxes of 16 gate (or up) rows, 32 down rows
+    bool ok = weight_maps(wkg, L.gate, L.gate_scale, E * I, H, GR, &maps.w[M_GATE], &maps.s[M_GATE]) &&
+              weight_maps(wkg, L.up, L.up_scale, E * I, H, GR, &maps.w[M_UP], &maps.s[M_UP]) &&
+              weight_maps(wkd, L.down, L.down_scale, E * H, I, DR, &maps.w[M_DOWN], &maps.s[M_DOWN]);
+    if (ok && Is > 0)
+      ok = weight_maps(wkg, L.sh_gate, L.sh_gate_scale, Is, H, GR, &maps.w[M_SGATE], &maps.s[M_SGATE]) &&
+           weight_maps(wkg, L.sh_up, L.sh_up_scale, Is, H, GR, &maps.w[M_SUP], &maps.s[M_SUP]) &&
+           weight_maps(wkd, L.sh_down, L.sh_down_scale, H, Is, DR, &maps.w[M_SDOWN], &maps.s[M_SDOWN]);
+    a.tma = ok && sw != 0;
+  }
+  return launch_by_kind(c, a, P, L.x_dtype == MOE_F32, wkg, wkd, maps);
 }
 
 }  // namespace moe

@@ -108,7 +108,17 @@ struct KParams {
   int skip_stage;
   int head_mult;       // single-CTA kernel: skip each group's first floor(rows / head_mult) * head_mult rows
                        // (the CTA-pair kernel's full 256-row tiles); 0: all rows
+  const int32_t* gather_rows;  // A row r = row gather_rows[r] / gather_div of the map's tensor (nullptr: row r)
+  int gather_div;
 };
+
+// Token rows of A rows [a_row + 4 lane, a_row + 4 lane + 4) for a gathered A operand (rows past the last
+// logical row read the last one; the epilogue never writes them).
+__device__ __forceinline__ void gather_tokens(const KParams& p, int a_row, int (&tr)[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) tr[j] = p.gather_rows[min(a_row + 4 * lane + j, p.rows_single - 1)] / p.gather_div;
+}
 
 // Wait ignoring the abort flag (used to drain in-flight work before exit).
 __device__ __forceinline__ bool wait_cycles(uint64_t* bar, uint32_t parity, long long limit) {
@@ -327,7 +337,59 @@ __global__ void __launch_bounds__(THREADS, 1)
   const long long limit = p.wait_limit;
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (MT == 1 && p.gather_rows != nullptr) {
+      // ------------------------------------------------------------ TMA producer, gathered A rows (whole warp)
+      // Lane l gathers rows [4 l, 4 l + 4) of each 128-row A tile straight from the token rows
+      // (tile::gather4, one row per coordinate, into the 128-byte-swizzled tile as a box load would);
+      // lane 0 waits for the stage, expects its bytes and loads the weight tile.
+      uint32_t kbg = 0, outstanding = 0, out_phase = 0;
+      bool skipped = false;
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_a = l2_policy_evict_last();
+      for (int w = blockIdx.x; w < total; w += gridDim.x) {
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+        int g, mt, nm, nt, ks;
+        decode_item<MT>(aux, p.G, p.ksplit, w, g, mt, nm, nt, ks);
+        const int a_row = aux.row_off[g] + mt * BM;
+        int tr[4];
+        gather_tokens(p, a_row, tr);
+        const bool one_mtile = aux.cnt[g] <= BM;
+        const int b_row = g * p.N + nt * p.col_step;
+        const int kb0 = ks * p.kb_per_split, kb1 = min(nkb, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
+          const int s = kbg % STAGES;
+          const uint32_t ph = (kbg / STAGES) & 1u;
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait_bounded(&aux.empty[s], ph ^ 1u, limit, abort_flag);
+          if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+          outstanding &= ~(1u << s);
+          if (p.skip_stage && !skipped && blockIdx.x == 0) {  // debug: leave this stage unfilled
+            skipped = true;
+            continue;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          if (lane == 0) mbar_arrive_expect_tx(&aux.full[s], A_BYTES + B_BYTES);
+          __syncwarp();
+          tma_gather4(sa + lane * 4 * 128, &mapA, &aux.full[s], kb * BK, tr[0], tr[1], tr[2], tr[3], pol_a);
+          if (lane == 0) {
+            if (one_mtile) {
+              tma_load_2d_hint(sb, &mapB0, &aux.full[s], kb * BK, b_row, pol_w);
+              if (DUAL) tma_load_2d_hint(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row, pol_w);
+            } else {
+              tma_load_2d(sb, &mapB0, &aux.full[s], kb * BK, b_row);
+              if (DUAL) tma_load_2d(sb + B_BYTES / 2, &mapB1, &aux.full[s], kb * BK, b_row);
+            }
+          }
+          outstanding |= 1u << s;
+          out_phase = (out_phase & ~(1u << s)) | (ph << s);
+        }
+      }
+      if (lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (outstanding & (1u << s)) wait_cycles(&aux.full[s], (out_phase >> s) & 1u, limit);
+      }
+    } else if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
       uint32_t kbg = 0, outstanding = 0, out_phase = 0;
       bool skipped = false;
@@ -586,32 +648,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const long long limit = p.wait_limit;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ TMA producer (both CTAs)
+    // ------------------------------------------------------------ TMA producer (both CTAs; with gathered A
+    // rows the whole warp: lane l gathers rows [4 l, 4 l + 4) of the CTA's 128 A rows, as in the single-CTA
+    // kernel, and lane 0 does the rest)
+    const bool gather = p.gather_rows != nullptr;
+    if (gather || lane == 0) {
       uint32_t kbg = 0, outstanding = 0, out_phase = 0;
       const uint64_t pol_a = l2_policy_evict_last();    // activation rows: read by every column tile
       const uint64_t pol_b = l2_policy_evict_normal();  // weight tiles: read by each row tile of the group
       const CUtensorMap* mb = (DUAL && rank == 1) ? &mapB1 : &mapB0;
-      for (int w = pair; w < total && !*abort_flag; w += npairs) {
+      const unsigned mask = gather ? 0xffffffffu : 1u;
+      for (int w = pair; w < total; w += npairs) {
+        if (__shfl_sync(mask, *abort_flag, 0)) break;
         int g, mt, nt;
         decode_pair_item(aux, p.G, w, g, mt, nt);
         const int a_row = aux.row_off[g] + mt * PAIR_M + static_cast<int>(rank) * BM;
         const int b_row = g * p.N + nt * p.col_step + (DUAL ? 0 : static_cast<int>(rank) * 128);
+        int tr[4] = {0, 0, 0, 0};
+        if (gather) gather_tokens(p, a_row, tr);
         for (int kb = 0; kb < nkb; ++kb, ++kbg) {
           const int s = kbg % PAIR_STAGES;
           const uint32_t ph = (kbg / PAIR_STAGES) & 1u;
-          if (!mbar_wait_bounded(&aux.empty[s], ph ^ 1u, limit, abort_flag)) break;
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait_bounded(&aux.empty[s], ph ^ 1u, limit, abort_flag);
+          if (!__shfl_sync(mask, ok, 0)) break;
           outstanding &= ~(1u << s);
           uint8_t* sa = smem + s * PAIR_STAGE_BYTES;
           const uint32_t full_s = cluster_addr(&aux.full[s], 0);
-          if (rank == 0) mbar_arrive_expect_tx(&aux.full[s], 2 * PAIR_STAGE_BYTES);
-          tma_load_2d_pair(sa, &mapA, full_s, kb * BK, a_row, pol_a);
-          tma_load_2d_pair(sa + A_BYTES, mb, full_s, kb * BK, b_row, pol_b);
+          if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&aux.full[s], 2 * PAIR_STAGE_BYTES);
+          if (gather) {
+            __syncwarp();
+            tma_gather4_pair(sa + lane * 4 * 128, &mapA, full_s, kb * BK, tr[0], tr[1], tr[2], tr[3], pol_a);
+          } else {
+            tma_load_2d_pair(sa, &mapA, full_s, kb * BK, a_row, pol_a);
+          }
+          if (lane == 0) tma_load_2d_pair(sa + A_BYTES, mb, full_s, kb * BK, b_row, pol_b);
           outstanding |= 1u << s;
           out_phase = (out_phase & ~(1u << s)) | (ph << s);
         }
       }
-      if (*abort_flag && rank == 0) {  // let issued copies land before the pair exits
+      if (lane == 0 && *abort_flag && rank == 0) {  // let issued copies land before the pair exits
         for (int s = 0; s < PAIR_STAGES; ++s)
           if (outstanding & (1u << s)) wait_cycles(&aux.full[s], (out_phase >> s) & 1u, limit);
       }
@@ -747,14 +823,24 @@ KParams make_params(const Ctx& c, const GemmArgs& a, int col_step, int head_mult
   p.wait_limit = c.wait_limit;
   p.skip_stage = c.skip_stage;
   p.head_mult = head_mult;
+  p.gather_rows = a.gather_rows;
+  p.gather_div = a.gather_div > 0 ? a.gather_div : 1;
   return p;
+}
+
+// The A map: the operand's rows in 128-row boxes, or, for a gathered operand, the source rows one at a time
+// (tile::gather4 boxes are one row high).
+bool make_a_map(CUtensorMap* m, const GemmArgs& a) {
+  if (a.gather_rows)
+    return make_map(m, a.A_src, static_cast<uint64_t>(a.rows_src), static_cast<uint64_t>(a.Kdim), 1);
+  return make_map(m, a.A, static_cast<uint64_t>(a.rows_A), static_cast<uint64_t>(a.Kdim), BM);
 }
 
 template <bool DUAL, int BN, int MT>
 cudaError_t launch_tiled(const Ctx& c, const GemmArgs& a, int head_mult = 0) {
   CUtensorMap mA, mB0, mB1;
   const uint32_t brows = DUAL ? BN / 2 : BN;
-  if (!make_map(&mA, a.A, static_cast<uint64_t>(a.rows_A), static_cast<uint64_t>(a.Kdim), BM) ||
+  if (!make_a_map(&mA, a) ||
       !make_map(&mB0, a.B0, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), brows))
     return cudaErrorInvalidValue;
   if (DUAL) {
@@ -806,7 +892,7 @@ int pair_clusters(const Ctx& c) {
 template <bool DUAL>
 cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, int clusters) {
   CUtensorMap mA, mB0, mB1;
-  if (!make_map(&mA, a.A, static_cast<uint64_t>(a.rows_A), static_cast<uint64_t>(a.Kdim), BM) ||
+  if (!make_a_map(&mA, a) ||
       !make_map(&mB0, a.B0, static_cast<uint64_t>(a.G) * a.N, static_cast<uint64_t>(a.Kdim), 128))
     return cudaErrorInvalidValue;
   if (DUAL) {
@@ -844,6 +930,7 @@ double wave_waste(double items, int sms) {
 cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a) {
   if (a.G <= 0 || a.max_rows <= 0 || a.N <= 0 || a.rows_A <= 0) return cudaSuccess;
   if (a.G > MAX_G || a.N % 32) return cudaErrorInvalidValue;  // the epilogue writes whole 16-byte column chunks
+  if (a.gather_rows && (!a.dual || a.ksplit > 1 || !a.A_src)) return cudaErrorInvalidValue;
   const int groups = std::min(a.G, a.max_rows);
   const double rows_per_group = static_cast<double>(a.max_rows) / groups;
   // about half an M tile of padding per group

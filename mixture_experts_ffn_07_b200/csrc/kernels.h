@@ -64,6 +64,12 @@ struct GemmArgs {
   const char* name;        // trace label
   int ksplit = 1;          // single mode without row_map/row_scale only: K split into ranges whose
   size_t part_stride = 0;  // f32 results go to out_f32 + range * part_stride (summed by the caller)
+  // Row gather (the routed gate/up projection): A row r is row gather_rows[r] / gather_div of A_src
+  // [rows_src, Kdim]; rows_A then counts the logical rows.  nullptr: A is read as it is.
+  const int32_t* gather_rows = nullptr;
+  int gather_div = 1;
+  const __nv_bfloat16* A_src = nullptr;
+  int64_t rows_src = 0;
 };
 cudaError_t launch_grouped_gemm(const Ctx& c, const GemmArgs& a);
 bool pair_gemm_enabled();  // moe_set_pair_gemm
@@ -140,8 +146,11 @@ struct DecodeLayer {
   float* y_slots;
   float* y_s;
   void* out;
+  void* stream_sync;  // decode_stream_sync_bytes() of workspace for the gate/up + down stream (nullptr: two phases)
 };
 size_t decode_router_parts_floats(int T, int H, int E, bool shared_gate);
+constexpr size_t decode_stream_sync_bytes() { return 4 * (1 + 257); }
+int stream_path_mode();  // moe_set_decode_stream: 0 off, 1 f32 / bf16, 2 also Q8_0
 cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L);
 
 

@@ -2,7 +2,7 @@
 // workspace layout, the order of kernel launches for each entry point, the
 // device status word, and the host-side launch counter and event trace.
 //
-// Path choice: bf16 activations with bf16 expert weights and T >= 65 (moe_set_tensor_min_tokens) take the
+// Path choice: bf16 activations with bf16 expert weights and T >= 8 (moe_set_tensor_min_tokens) take the
 // tensor-core path (row gather + tcgen05 grouped GEMMs); everything else takes
 // the weight-streaming path (expert-major GEMV kernels), which reads each
 // touched expert's weights once and is the bandwidth-optimal form for small T.
@@ -39,6 +39,8 @@ std::atomic<long long> g_barrier_delay{0};
 std::atomic<int> g_fused_decode{1};
 std::atomic<int> g_fused_front{1};
 std::atomic<int> g_pair_gemm{1};
+std::atomic<int> g_decode_stream{1};
+std::atomic<int> g_tma_gather{0};
 
 struct TraceRec {
   const char* name;
@@ -82,8 +84,10 @@ inline size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255);
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Fewest tokens for which a bf16 layer takes the tensor-core path (moe_set_tensor_min_tokens).
-std::atomic<int> g_tensor_min_tokens{65};
+// Fewest tokens for which a bf16 layer takes the tensor-core path (moe_set_tensor_min_tokens).  Measured
+// on B200 (bench.py --op crossover): the tensor-core path is faster from 2-8 tokens on, depending on the
+// shape, so 8.
+std::atomic<int> g_tensor_min_tokens{8};
 
 bool tensor_path(const moe_desc& d) {
   return d.act_dtype == MOE_BF16 && d.w_dtype == MOE_BF16 && d.T >= g_tensor_min_tokens.load();
@@ -151,7 +155,7 @@ moe::RouteCfg route_cfg(const moe_desc& d) {
 }
 
 struct Layout {
-  size_t logits, logit_parts, router_parts, front_hist, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos,
+  size_t logits, logit_parts, router_parts, stream_sync, front_hist, ids, w, shared_gate, counts, offsets, sorted_pairs, pair_pos,
       y_slots, x_perm, h, h_s, y_s, total;
 };
 
@@ -168,6 +172,7 @@ Layout layout_of(const moe_desc& d) {
   L.logits = take(T * E * 4);
   L.logit_parts = tensor_router(d) ? take(router_ksplit(d) * T * E * 4) : 0;
   L.router_parts = fused_decode(d) ? take(moe::decode_router_parts_floats(d.T, d.H, d.E, shared_gated(d)) * 4) : 0;
+  L.stream_sync = fused_decode(d) ? take(moe::decode_stream_sync_bytes()) : 0;
   L.front_hist = fused_front(d) ? take(static_cast<size_t>(moe::kMaxFrontCtas) * E * 4) : 0;
   L.ids = take(P * 4);
   L.w = take(P * 4);
@@ -177,7 +182,7 @@ Layout layout_of(const moe_desc& d) {
   L.sorted_pairs = take(P * 4);
   L.pair_pos = take(P * 4);
   L.y_slots = take(P * H * 4);
-  L.x_perm = tc ? take(P * H * 2) : 0;
+  L.x_perm = tc && !g_tma_gather.load() ? take(P * H * 2) : 0;
   L.h = take(P * I * (tc ? 2 : 4));
   L.h_s = Is ? take(T * Is * (tc ? 2 : 4)) : 0;
   L.y_s = Is ? take(T * H * 4) : 0;
@@ -262,13 +267,20 @@ moe_status expert_impl(const moe::Ctx& c, const moe_desc& d, const void* x, cons
                        const Layout& L, bool rows_gathered = false, bool bf16_slots = false) {
   const int P = d.T * d.top_k;
   if (tensor_path(d)) {
-    __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.x_perm);
     __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
-    if (!rows_gathered)
-      MOE_TRY(moe::launch_gather_rows(c, static_cast<const __nv_bfloat16*>(x), sorted_pairs, offsets, d.E, d.top_k,
-                                      P, d.H, xp));
     moe::GemmArgs a{};
-    a.A = xp;
+    if (L.x_perm == 0) {  // the GEMM gathers each pair's x row itself (TMA tile::gather4)
+      a.gather_rows = sorted_pairs;
+      a.gather_div = d.top_k;
+      a.A_src = static_cast<const __nv_bfloat16*>(x);
+      a.rows_src = d.T;
+    } else {  // x rows copied into expert order first
+      __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.x_perm);
+      if (!rows_gathered)
+        MOE_TRY(moe::launch_gather_rows(c, static_cast<const __nv_bfloat16*>(x), sorted_pairs, offsets, d.E,
+                                        d.top_k, P, d.H, xp));
+      a.A = xp;
+    }
     a.rows_A = P;
     a.Kdim = d.H;
     a.B0 = static_cast<const __nv_bfloat16*>(w.gate);
@@ -421,6 +433,8 @@ cudaError_t allow_dynamic_smem(const void* kernel, int bytes) {
 // timeline groups the launches by step; without a profiler attached the NVTX
 // calls return at once.
 bool pair_gemm_enabled() { return g_pair_gemm.load() != 0; }
+
+int stream_path_mode() { return g_decode_stream.load(); }
 
 KernelScope::KernelScope(const Ctx& c, const char* name) : ctx(c), slot(-1) {
   g_launches.fetch_add(1);
@@ -599,6 +613,7 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
     f.sh_up_scale = w->sh_up_scale;
     f.sh_down_scale = w->sh_down_scale;
     f.router_parts = at<float>(ws, L.router_parts);
+    f.stream_sync = at<void>(ws, L.stream_sync);
     f.logits = logits;
     f.ids = ids;
     f.w = tw;
@@ -643,7 +658,7 @@ moe_status moe_layer(const moe_desc* d, const void* x, const moe_weights* w, voi
     f.offsets = offsets;
     f.sorted_pairs = sorted_pairs;
     f.pair_pos = at<int32_t>(ws, L.pair_pos);
-    f.x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+    f.x_perm = L.x_perm ? at<__nv_bfloat16>(ws, L.x_perm) : nullptr;
     f.hist = at<int32_t>(ws, L.front_hist);
     const cudaError_t e = moe::launch_prefill_front(c, f);
     bool gathered = e == cudaSuccess;
@@ -814,6 +829,10 @@ void moe_set_fused_decode(int enable) { g_fused_decode.store(enable ? 1 : 0); }
 void moe_set_fused_front(int enable) { g_fused_front.store(enable ? 1 : 0); }
 
 void moe_set_pair_gemm(int enable) { g_pair_gemm.store(enable ? 1 : 0); }
+
+void moe_set_decode_stream(int mode) { g_decode_stream.store(mode < 0 ? 0 : (mode > 2 ? 2 : mode)); }
+
+void moe_set_tma_gather(int enable) { g_tma_gather.store(enable ? 1 : 0); }
 
 void moe_set_tensor_min_tokens(int tokens) { g_tensor_min_tokens.store(std::max(1, tokens)); }
 

@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
       __syncwarp();
     }
   }
+  if (a.x_perm == nullptr) return;  // the expert GEMM gathers the rows itself
   __syncthreads();
   const int n16 = a.H / 8;  // 16-byte groups of a bf16 row
   const uint4* src = reinterpret_cast<const uint4*>(a.x);

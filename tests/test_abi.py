@@ -57,9 +57,15 @@ def test_workspace_bytes_host_only():
     d = moe.Desc(T=512, H=2048, E=64, I=1024, top_k=8)
     n = moe.workspace_bytes(d)
     P = 512 * 8
-    # routing + permutation + slots [P,H] f32 + gathered rows [P,H] bf16 + h [P,I] bf16
+    # routing + permutation + slots [P,H] f32 + the x rows in expert order [P,H] bf16 + h [P,I] bf16
     assert n >= P * 2048 * 4 + P * 2048 * 2 + P * 1024 * 2
     assert n % 256 == 0
+    # with the gate/up GEMM gathering the x rows itself: no [P,H] bf16 copy
+    moe.set_tma_gather(True)
+    try:
+        assert n - moe.workspace_bytes(d) >= P * 2048 * 2
+    finally:
+        moe.set_tma_gather(False)
     # affine in T without the tensor-core router; with it, plus at most 20480 * E * 4 bytes of split-K scratch
     # and 256 * E * 4 bytes of per-CTA expert counts (each region 256-byte aligned)
     ts = (1024, 2048, 3072, 4096, 8192)

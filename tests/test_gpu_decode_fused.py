@@ -82,6 +82,12 @@ def _bits(t):
     return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
 
 
+@pytest.fixture(autouse=True)
+def _bf16_on_the_streaming_path():
+    with _gpu.streaming_path():  # the bf16 cases are decode batches on the streaming path
+        yield
+
+
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_fused_matches_steps_and_oracle(case):
     s, opt = CASES[case]

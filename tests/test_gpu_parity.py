@@ -132,8 +132,19 @@ FFN_CASES = {
 }
 
 
+@pytest.fixture
+def path_for(request):
+    """Cases named stream_* run with bf16 batches of up to 64 tokens on the streaming path."""
+    case = request.node.callspec.params.get("case", "")
+    if case.startswith("stream_"):
+        with _gpu.streaming_path():
+            yield
+    else:
+        yield
+
+
 @pytest.mark.parametrize("case", sorted(FFN_CASES))
-def test_expert_ffn(case):
+def test_expert_ffn(case, path_for):
     s = FFN_CASES[case]
     wl = make(s, seed=5)
     desc, w, x = _gpu.upload(wl)
@@ -186,7 +197,7 @@ LAYER_CASES = {
 
 
 @pytest.mark.parametrize("case", sorted(LAYER_CASES))
-def test_layer(case):
+def test_layer(case, path_for):
     s, opt = LAYER_CASES[case]
     bias = None
     if opt.get("bias"):

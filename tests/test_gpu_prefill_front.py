@@ -1,11 +1,14 @@
-"""The tensor-core path's fused selection + permutation + row gather
-(route_permute_gather, one cooperative launch after the router GEMM) against
-the three separate launches it replaces, moe_route and the oracle.
+"""The tensor-core path's fused selection + permutation (route_permute_gather,
+one cooperative launch after the router GEMM) against the separate launches
+it replaces, moe_route and the oracle.  With the x rows copied into expert
+order first (the default) the fused kernel also does that copy and replaces
+three launches (router_topk, permute, gather_rows); with the expert GEMM
+gathering its rows itself (moe_set_tma_gather(1)) it replaces two.
 
 The fused kernel selects with the same code as router_topk_kernel and the
 permutation is a stable sort (unique), so logits, ids, weights, counts,
 offsets, sorted pairs and their inverse must be bit-identical to the
-three-launch path, and so must the output (the GEMMs then see the same rows).
+separate-launch path, and so must the output (the GEMMs then see the same rows).
 """
 import numpy as np
 import pytest
@@ -82,7 +85,7 @@ def test_fused_front_matches_three_launches(case):
     desc, w, x = _gpu.upload(wl)
     out_f, rf, nf = _run(desc, w, x, True)
     out_s, rs, ns = _run(desc, w, x, False)
-    assert ns - nf == 2  # three launches become one
+    assert ns - nf == 2  # selection, permutation and the row copy: three launches become one
     for k in rs:
         assert torch.equal(_bits(rf[k]), _bits(rs[k])), f"{case}: {k}"
     assert torch.equal(_bits(out_f), _bits(out_s))
@@ -108,3 +111,22 @@ def test_fused_front_back_to_back():
     torch.cuda.synchronize()
     assert moe.last_device_status() == moe.MOE_OK
     assert torch.equal(_bits(out), _bits(ref))
+
+
+def test_fused_front_with_gathering_gemm():
+    """With the gate/up GEMM gathering its x rows itself (moe_set_tma_gather(1)) the fused kernel writes no
+    copy: two launches become one, and the layer has the same bits as with the copied rows."""
+    s, opt = CASES["T333_E64_shared_ungated"]
+    wl = _workload(s, opt, seed=57)
+    desc, w, x = _gpu.upload(wl)
+    out_c, _, n_c = _run(desc, w, x, True)
+    moe.set_tma_gather(True)
+    try:
+        out_f, _, nf = _run(desc, w, x, True)
+        out_s, _, ns = _run(desc, w, x, False)
+    finally:
+        moe.set_tma_gather(False)
+    assert ns - nf == 1
+    assert nf == n_c
+    assert torch.equal(out_f.view(torch.int16), out_s.view(torch.int16))
+    assert torch.equal(out_f.view(torch.int16), out_c.view(torch.int16))
