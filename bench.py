@@ -335,7 +335,7 @@ def run_ours(args, spec):
     from mixture_experts_ffn_07_b200 import host
 
     moe.set_pair_gemm(bool(args.pair_gemm))
-    moe.set_decode_stream(args.decode_stream)
+    moe.set_decode_stream(bool(args.decode_stream))
     wl = workloads.make(spec)
     desc, w, x = host.upload(wl)
     T, H = spec.T, spec.H
@@ -489,7 +489,7 @@ def run_ours(args, spec):
             "data": "synthetic",
             "config": {"workload": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "I": spec.I, "top_k": spec.K,
                        "act": spec.act, "shared_I": spec.shared_I, "parallelism": f"replicas{ws_n}",
-                       "pair_gemm": bool(args.pair_gemm), "decode_stream": args.decode_stream,
+                       "pair_gemm": bool(args.pair_gemm), "decode_stream": bool(args.decode_stream),
                        "l2": f"no flush: inputs larger than L2; x rotates over {NROT} token batches, so consecutive "
                              "steps route to different experts"},
             "e2e": {"value": job_throughput(ws_n, T, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
@@ -775,9 +775,9 @@ def main():
                          "crossover: both paths of bf16 layers over batch sizes 8..256")
     ap.add_argument("--pair-gemm", type=int, default=1, choices=[0, 1],
                     help="0: compute-bound expert GEMMs on single CTAs only (moe_set_pair_gemm), for comparison")
-    ap.add_argument("--decode-stream", type=int, default=1, choices=[0, 1, 2],
-                    help="moe_set_decode_stream mode: 0 two phases for every format, 1 stream for f32/bf16 "
-                         "(default), 2 stream for Q8_0 too; for comparison")
+    ap.add_argument("--decode-stream", type=int, default=1, choices=[0, 1],
+                    help="0: the decode kernel's gate/up and down as two phases for every format "
+                         "(moe_set_decode_stream), for comparison")
     ap.add_argument("--dist-selftest", action="store_true",
                     help="ranks only: gloo process group, max over ranks of a rank-dependent time, no GPU work")
     args = ap.parse_args()

@@ -227,11 +227,10 @@ def set_pair_gemm(enable: bool) -> None:
     _lib.lib().moe_set_pair_gemm(int(enable))
 
 
-def set_decode_stream(mode) -> None:
-    """moe_set_decode_stream: gate/up and down of the cooperative decode kernel as one TMA-fed stream of
-    work items for f32 / bf16 weights (1 or True, default), for Q8_0 too (2), or two phases with a grid
-    barrier for every format (0 or False)."""
-    _lib.lib().moe_set_decode_stream(int(mode))
+def set_decode_stream(enable: bool) -> None:
+    """moe_set_decode_stream: gate/up and down of the cooperative decode kernel for f32 / bf16 weights as one
+    TMA-fed stream of work items (True, default) or two phases with a grid barrier (False)."""
+    _lib.lib().moe_set_decode_stream(int(enable))
 
 
 def set_tma_gather(enable: bool) -> None:

@@ -225,6 +225,7 @@ __device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+
 // L2 policies: data read once (streamed weights) goes first when L2 needs
 // room; data read again soon (activation rows, the next kernel's inputs) last.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {

@@ -76,10 +76,13 @@ struct DecodeArgs {
   dstream::Sync* sync;     // queue and per-group counters of the stream (workspace)
 };
 
-// The stream instance of a weight format: one format for gate/up and down, f32, bf16 or Q8_0.
+// The formats the stream serves: one format for gate/up and down, f32 or bf16.  (A Q8_0 stream measured
+// slower than the Q8_0 row-pair GEMV -- q8_0_decode_t16 315 against 233 us: with ~1.5 tokens per expert its
+// items are one or two stages long and the per-item and per-token work dominates -- so Q8_0 and the
+// k-quant stacks keep the two phases.)
 template <int WKG, int WKD>
 __host__ __device__ constexpr bool stream_format() {
-  return WKG == WKD && (WKG == WK_F32 || WKG == WK_BF16 || WKG == WK_Q8);
+  return WKG == WKD && (WKG == WK_F32 || WKG == WK_BF16);
 }
 
 __device__ __forceinline__ bool cta_grid_sync(const DecodeArgs& a, int* s_abort, int* s_flag) {
@@ -583,17 +586,11 @@ bool stream_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int
   return true;
 }
 
-// Maps of one weight matrix [rows, K] (+ Q8_0 scale plane) for the stream; false if its layout does not fit
-// (rows too long for the 32-bit strides, scale rows not a multiple of 16 bytes, misaligned pointers).
-bool weight_maps(int wk, const void* w, const void* scale, uint64_t rows, uint64_t K, uint32_t box_rows,
-                 CUtensorMap* mw, CUtensorMap* ms) {
-  // a slot row: 256 elements of the map's type (f32, bf16, or Q8_0 codes as 32-bit words) and, for Q8_0, the
-  // 32 fp16 scales of those 1024 codes, one row per box
+// The map of one weight matrix [rows, K] (f32 or bf16) for the stream, in boxes of 256 elements x box_rows;
+// false if its layout does not fit (misaligned pointer).
+bool weight_map(int wk, const void* w, uint64_t rows, uint64_t K, uint32_t box_rows, CUtensorMap* mw) {
   if (wk == WK_F32) return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, K, 256, box_rows);
-  if (wk == WK_BF16) return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 256, box_rows);
-  if (K % 256) return false;  // the fp16 scale rows (K / 16 bytes) must be whole 16-byte units
-  return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, rows, K / 4, 256, box_rows) &&
-         stream_map(ms, scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, K / 32, 32, box_rows);
+  return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 256, box_rows);
 }
 
 }  // namespace
@@ -680,26 +677,23 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
   a.status = c.status;
   a.wait_limit = c.wait_limit;
   a.barrier_delay = c.barrier_delay;
-  // gate/up and down as one TMA-fed stream: f32, bf16 or Q8_0 in both projections, every matrix mappable
+  // gate/up and down as one TMA-fed stream: f32 or bf16 in both projections, every matrix mappable
   dstream::Maps maps;
   memset(&maps, 0, sizeof(maps));
   a.sync = static_cast<dstream::Sync*>(L.stream_sync);
-  // Q8_0 keeps the two phases: with ~1.5 tokens per expert its items are one or two stages long, and the
-  // stream's per-item and per-token work measured slower than the row-pair GEMV (q8_0_decode_t16: 315 against
-  // 233 us); moe_set_decode_stream(2) takes the stream for Q8_0 too
   const int sw = stream_path_mode();
-  a.tma = L.stream_sync != nullptr && wkg == wkd && (wkg == WK_F32 || wkg == WK_BF16 || (wkg == WK_Q8 && sw == 2));
+  a.tma = L.stream_sync != nullptr && wkg == wkd && (wkg == WK_F32 || wkg == WK_BF16);
   if (a.tma) {
     using namespace dstream;
     const uint64_t E = L.E, H = L.H, I = L.I, Is = L.Is;
     constexpr uint32_t GR = kRows / 2, DR = kRows;  // boxes of 16 gate (or up) rows, 32 down rows
-    bool ok = weight_maps(wkg, L.gate, L.gate_scale, E * I, H, GR, &maps.w[M_GATE], &maps.s[M_GATE]) &&
-              weight_maps(wkg, L.up, L.up_scale, E * I, H, GR, &maps.w[M_UP], &maps.s[M_UP]) &&
-              weight_maps(wkd, L.down, L.down_scale, E * H, I, DR, &maps.w[M_DOWN], &maps.s[M_DOWN]);
+    bool ok = weight_map(wkg, L.gate, E * I, H, GR, &maps.w[M_GATE]) &&
+              weight_map(wkg, L.up, E * I, H, GR, &maps.w[M_UP]) &&
+              weight_map(wkd, L.down, E * H, I, DR, &maps.w[M_DOWN]);
     if (ok && Is > 0)
-      ok = weight_maps(wkg, L.sh_gate, L.sh_gate_scale, Is, H, GR, &maps.w[M_SGATE], &maps.s[M_SGATE]) &&
-           weight_maps(wkg, L.sh_up, L.sh_up_scale, Is, H, GR, &maps.w[M_SUP], &maps.s[M_SUP]) &&
-           weight_maps(wkd, L.sh_down, L.sh_down_scale, H, Is, DR, &maps.w[M_SDOWN], &maps.s[M_SDOWN]);
+      ok = weight_map(wkg, L.sh_gate, Is, H, GR, &maps.w[M_SGATE]) &&
+           weight_map(wkg, L.sh_up, Is, H, GR, &maps.w[M_SUP]) &&
+           weight_map(wkd, L.sh_down, H, Is, DR, &maps.w[M_SDOWN]);
     a.tma = ok && sw != 0;
   }
   return launch_by_kind(c, a, P, L.x_dtype == MOE_F32, wkg, wkd, maps);

@@ -34,14 +34,15 @@
 // groups found complete, so later items of the group do not ask again.  The queue hands out all gate/up items first, expert by expert, so
 // the first down items find their experts finished long before; there is no
 // grid barrier between the two projections, and a CTA moves from gate/up rows
-// to down rows without draining its ring.  A group with more than NT tokens
+// to down rows without draining its ring.  (Asking L2 for a batch of items
+// ahead of their copies measured slower: the prefetched rows of 148 CTAs
+// evict one another.)  A group with more than NT tokens
 // has one item per chunk of NT tokens, the chunks of a row block next to each
 // other in the queue so that the repeated weight rows come from L2.
 //
-// Formats: f32 and bf16 weight rows, and Q8_0 in the split form (int8 codes
-// [rows, K], fp16 scales [rows, K/32]): a lane's 16-code chunk is half a
-// block, so partial = sum q*x over the chunk, then acc += d * partial.
-// Activations f32 or bf16.
+// Formats: f32 and bf16 weight rows, f32 or bf16 activations.  (A Q8_0 form
+// of the stream measured slower than the row-pair GEMV of stream_core.cuh,
+// so Q8_0 and the k-quant stacks keep the two phases.)
 #pragma once
 
 #include "stream_core.cuh"
@@ -52,39 +53,34 @@ namespace dstream {
 using stream::kWarps;
 using stream::WK_BF16;
 using stream::WK_F32;
-using stream::WK_Q8;
 
 constexpr int kStages = 4;            // ring depth
 constexpr int kRows = 32;             // weight rows per stage (and per item)
 constexpr int kRowBytes = 1024;       // bytes of one weight row in a stage (f32: 256 values)
-constexpr int kScaleBox = 64;         // Q8_0: bytes of the 32 fp16 scales of one row in a stage
-constexpr int kStageWBytes = kRows * kRowBytes;   // 32 KB
-constexpr int kStageSBytes = kRows * kScaleBox;   // 2 KB
-constexpr int kStageBytes = kStageWBytes + kStageSBytes;
+constexpr int kStageBytes = kRows * kRowBytes;    // 32 KB
 constexpr int kRingBytes = kStages * kStageBytes;
-static_assert(kStageWBytes % 128 == 0 && kStageBytes % 128 == 0 && (kRows / 2) * kScaleBox % 128 == 0,
+static_assert(kStageBytes % 128 == 0 && (kRows / 2) * 512 % 128 == 0,
               "every copy into the ring starts at a 128-byte boundary");
 
-// Elements of a row per stage (KC: 256 elements of the map's type), bytes of
-// a row per stage (RB) and 16-byte chunks per lane and row (NCH).
+// Elements of a row per stage (KC: 256, the widest box), bytes of a row per
+// stage (RB) and 16-byte chunks per lane and row (NCH).
 template <int WK>
 struct Fmt {
-  static constexpr int EB = WK == WK_F32 ? 4 : (WK == WK_BF16 ? 2 : 1);
-  static constexpr int KC = WK == WK_Q8 ? 1024 : 256;  // row elements per stage (Q8_0: codes)
+  static_assert(WK == WK_F32 || WK == WK_BF16, "the stream serves f32 and bf16 weights");
+  static constexpr int EB = WK == WK_F32 ? 4 : 2;
+  static constexpr int KC = 256;                       // row elements per stage
   static constexpr int RB = KC * EB;                   // bytes of a row in a stage
   static constexpr int NCH = RB / 512;                 // 16-byte chunks per lane and row
   static constexpr int E16 = 16 / EB;                  // elements per chunk
   static_assert(RB % 512 == 0 && RB <= kRowBytes, "a stage row is whole 512-byte runs");
 };
 
-// Tensor maps of one layer: weights and Q8_0 scale planes of gate, up, down,
-// shared gate, shared up, shared down.  Weight boxes are 256 elements wide
-// (Q8_0 codes as 32-bit words), 16 rows high for gate/up and 32 for down;
-// scale boxes 32 fp16 wide and as high.
+// Tensor maps of one layer: the weights of gate, up, down, shared gate, shared
+// up, shared down, in boxes 256 elements wide, 16 rows high for gate/up and
+// 32 for down.
 enum { M_GATE = 0, M_UP, M_DOWN, M_SGATE, M_SUP, M_SDOWN, M_COUNT };
 struct Maps {
   CUtensorMap w[M_COUNT];
-  CUtensorMap s[M_COUNT];
 };
 
 // Per-launch synchronisation words in the caller's workspace, zeroed by the
@@ -204,33 +200,20 @@ __device__ __forceinline__ Item decode_item(const Params& p, const Items& it, in
   return m;
 }
 
-// Lane 0 of warp 0: requests stage kc of item m (32 rows; Q8_0 also their
-// scales) into `st`, completing on `bar`.
+// Thread 0: requests stage kc of item m (its 32 rows) into `st`, completing on `bar`.
 template <int WK>
 __device__ __forceinline__ void issue_stage(const Maps& maps, const Params& p, const Item& m, int kc, uint8_t* st,
                                             uint64_t* bar) {
-  constexpr int KC = Fmt<WK>::KC;
   constexpr int RB = Fmt<WK>::RB;
-  const int kx = WK == WK_Q8 ? kc * (KC / 4) : kc * KC;  // Q8_0 codes as 32-bit words
-  const int ks = kc * (KC / 32);
-  uint8_t* sc = st + kStageWBytes;
-  constexpr uint32_t bytes = kRows * RB + (WK == WK_Q8 ? kRows * kScaleBox : 0);
-  mbar_arrive_expect_tx(bar, bytes);
+  const int kx = kc * Fmt<WK>::KC;
+  mbar_arrive_expect_tx(bar, kRows * RB);
   const uint64_t pol = l2_policy_evict_first();  // weight rows are read once (a repeated chunk: from L2 at once)
   if (!m.down) {
-    const int mg = m.e < 0 ? M_SGATE : M_GATE, mu = m.e < 0 ? M_SUP : M_UP;
     const int row = (m.e < 0 ? 0 : m.e * p.I) + m.r0;
-    tma_load_2d_hint(st, &maps.w[mg], bar, kx, row, pol);
-    tma_load_2d_hint(st + (kRows / 2) * RB, &maps.w[mu], bar, kx, row, pol);
-    if (WK == WK_Q8) {
-      tma_load_2d_hint(sc, &maps.s[mg], bar, ks, row, pol);
-      tma_load_2d_hint(sc + (kRows / 2) * kScaleBox, &maps.s[mu], bar, ks, row, pol);
-    }
+    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SGATE : M_GATE], bar, kx, row, pol);
+    tma_load_2d_hint(st + (kRows / 2) * RB, &maps.w[m.e < 0 ? M_SUP : M_UP], bar, kx, row, pol);
   } else {
-    const int md = m.e < 0 ? M_SDOWN : M_DOWN;
-    const int row = (m.e < 0 ? 0 : m.e * p.H) + m.r0;
-    tma_load_2d_hint(st, &maps.w[md], bar, kx, row, pol);
-    if (WK == WK_Q8) tma_load_2d_hint(sc, &maps.s[md], bar, ks, row, pol);
+    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SDOWN : M_DOWN], bar, kx, (m.e < 0 ? 0 : m.e * p.H) + m.r0, pol);
   }
 }
 
@@ -269,16 +252,11 @@ __device__ __forceinline__ void w_chunk(uint32_t a, float2 (&w)[Fmt<WK>::E16 / 2
   if constexpr (WK == WK_F32) {
     w[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
     w[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
-  } else if constexpr (WK == WK_BF16) {
+  } else {
     w[0] = stream::bf16x2_f2(v.x);
     w[1] = stream::bf16x2_f2(v.y);
     w[2] = stream::bf16x2_f2(v.z);
     w[3] = stream::bf16x2_f2(v.w);
-  } else {
-    stream::q8_quad(v.x, w[0], w[1]);
-    stream::q8_quad(v.y, w[2], w[3]);
-    stream::q8_quad(v.z, w[4], w[5]);
-    stream::q8_quad(v.w, w[6], w[7]);
   }
 }
 
@@ -371,7 +349,8 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
       if (++is_item >= is_end) {
         is_item = is_next;
         is_end = min(total, is_item + kBatch);
-        if (is_item < is_end) is_next = static_cast<int>(atomicAdd(&p.sync->queue, 1u)) * kBatch;
+        if (is_item < is_end)  // the batch after it, asked for now
+          is_next = static_cast<int>(atomicAdd(&p.sync->queue, 1u)) * kBatch;
       }
       is_kc = 0;
       if (is_item < is_end) is_m = decode_item<NT, WK>(p, it, is_item);
@@ -443,7 +422,6 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
     const uint32_t st = smem_addr(stages + s * kStageBytes);
     const int ra = m.down ? 2 * warp : warp, rb = m.down ? 2 * warp + 1 : kRows / 2 + warp;
     const uint32_t wa_s = st + ra * RB, wb_s = st + rb * RB;
-    const uint8_t* scs = stages + s * kStageBytes + kStageWBytes;
 #pragma unroll
     for (int ch = 0; ch < NCH; ++ch) {
       const int k = kc * KC + (ch * 512 + lane * 16) / Fmt<WK>::EB;
@@ -451,12 +429,6 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
         float2 wa[E16 / 2], wb[E16 / 2];
         w_chunk<WK>(wa_s + ch * 512 + lane * 16, wa);
         w_chunk<WK>(wb_s + ch * 512 + lane * 16, wb);
-        float sa = 1.f, sb = 1.f;
-        if constexpr (WK == WK_Q8) {  // the fp16 scale of the chunk's block
-          const int blk = (ch * 512 + lane * 16) / 32;
-          sa = __half2float(*reinterpret_cast<const __half*>(scs + ra * kScaleBox + blk * 2));
-          sb = __half2float(*reinterpret_cast<const __half*>(scs + rb * kScaleBox + blk * 2));
-        }
 #pragma unroll
         for (int c = 0; c < NT; ++c) {
           if (c < m.nt) {
@@ -467,21 +439,10 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
                                           k, xv);
             else
               act_chunk<XT, false, E16>(static_cast<const XT*>(p.x) + static_cast<size_t>(arow[c]) * p.H, k, xv);
-            if constexpr (WK == WK_Q8) {
-              float2 pa = __fmul2_rn(wa[0], xv[0]), pb = __fmul2_rn(wb[0], xv[0]);
 #pragma unroll
-              for (int i = 1; i < E16 / 2; ++i) {
-                pa = __ffma2_rn(wa[i], xv[i], pa);
-                pb = __ffma2_rn(wb[i], xv[i], pb);
-              }
-              acc_a[c] = __ffma2_rn(make_float2(sa, sa), pa, acc_a[c]);
-              acc_b[c] = __ffma2_rn(make_float2(sb, sb), pb, acc_b[c]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < E16 / 2; ++i) {
-                acc_a[c] = __ffma2_rn(wa[i], xv[i], acc_a[c]);
-                acc_b[c] = __ffma2_rn(wb[i], xv[i], acc_b[c]);
-              }
+            for (int i = 0; i < E16 / 2; ++i) {
+              acc_a[c] = __ffma2_rn(wa[i], xv[i], acc_a[c]);
+              acc_b[c] = __ffma2_rn(wb[i], xv[i], acc_b[c]);
             }
           }
         }

@@ -830,7 +830,7 @@ void moe_set_fused_front(int enable) { g_fused_front.store(enable ? 1 : 0); }
 
 void moe_set_pair_gemm(int enable) { g_pair_gemm.store(enable ? 1 : 0); }
 
-void moe_set_decode_stream(int mode) { g_decode_stream.store(mode < 0 ? 0 : (mode > 2 ? 2 : mode)); }
+void moe_set_decode_stream(int enable) { g_decode_stream.store(enable ? 1 : 0); }
 
 void moe_set_tma_gather(int enable) { g_tma_gather.store(enable ? 1 : 0); }
 
