@@ -360,14 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (stream_format<WKG, WKD>()) {
     if (a.tma) {
       // ---- G + D as one stream of items (decode_stream.cuh); then one barrier before the combine
-      constexpr int NT = MAXT == 1 ? 1 : 4;
+      constexpr int NT = dstream::item_tokens(MAXT);
       dstream::Params dp;
       dp.H = a.H;
       dp.K = a.K;
       dp.I = a.g.plan[0].Nout;
       dp.Is = a.has_shared ? a.g.plan[1].Nout : 0;
       dp.act = a.g.act_fn;
-      dp.x = a.x;
       dp.h = a.g.src[0].out;
       dp.h_s = a.g.src[1].out;
       dp.y_slots = a.d.src[0].out;
@@ -694,6 +693,18 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
       ok = weight_map(wkg, L.sh_gate, Is, H, GR, &maps.w[M_SGATE]) &&
            weight_map(wkg, L.sh_up, Is, H, GR, &maps.w[M_SUP]) &&
            weight_map(wkd, L.sh_down, H, Is, DR, &maps.w[M_SDOWN]);
+    // activation rows: x in boxes of one row; h and h_s in boxes of the item's tokens (no taller than the
+    // matrix), the same kernel instance launch_fused picks for T
+    const uint32_t nt = static_cast<uint32_t>(item_tokens(L.T == 1 ? 1 : kDecodeTok));
+    const uint64_t T = L.T, P = T * L.K;
+    maps.h_box = static_cast<int>(std::min<uint64_t>(nt, P));
+    maps.hs_box = static_cast<int>(std::min<uint64_t>(nt, T));
+    if (ok)
+      ok = (L.x_dtype == MOE_F32 ? stream_map(&maps.w[M_X], L.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, H, 256, 1)
+                                 : stream_map(&maps.w[M_X], L.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, H, 256, 1)) &&
+           stream_map(&maps.w[M_H], L.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P, I, 256, maps.h_box);
+    if (ok && Is > 0)
+      ok = stream_map(&maps.w[M_HS], L.h_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, Is, 256, maps.hs_box);
     a.tma = ok && sw != 0;
   }
   return launch_by_kind(c, a, P, L.x_dtype == MOE_F32, wkg, wkd, maps);

@@ -9,36 +9,44 @@
 // group:
 //   gate/up: gate rows j..j+15 and up rows j..j+15 of an expert (16 features);
 //   down:    down rows n..n+31.
-// Every CTA takes the next item from a device-wide counter; lane 0 of warp 0
-// streams the items' rows through the copy engine (cp.async.bulk.tensor.2d,
-// one box of 16 or 32 rows x 256 elements per copy -- 16 to 32 KB, so the
-// copy engine's cost per copy stays small -- no multicast) into a ring of
-// kStages stages, each on its own pair of mbarriers (full: the copies landed;
-// empty: all 16 warps are done with it).  Warp w takes two rows of every
-// stage (gate/up: gate row w and up row 16 + w, i.e. feature j + w; down: rows
-// 2w and 2w + 1); lane l owns 16-byte chunks l and 32 + l of each row (512
-// bytes apart, so every shared-memory load of the warp reads 512 contiguous
-// bytes), loads its activation values for those elements once per token (x
-// from the input through L1, h from L2) and uses them for both rows,
-// accumulating 2 x NT partial sums in registers.  At the item's last stage
-// the warp adds its lanes' partial sums (a butterfly over the 2*NT values)
+// Every CTA takes its next batch of items from a device-wide counter.  The
+// CTA is warp specialised: lane 0 of warp 8 streams each item's weight rows
+// through the copy engine (cp.async.bulk.tensor.2d, one box of 16 or 32 rows x
+// 256 elements per copy; no multicast) into a ring of kStages stages of 32 KB,
+// each on a full and an empty mbarrier, and the same stage receives the item's
+// activation rows for its 256 elements (the x rows of the chunk's tokens for
+// gate/up, a box of h rows for down), so no consumer waits on a global load.
+// The issuing thread sleeps on a stage's empty barrier until the 8 consumer
+// warps have released it and the consumers sleep on the full barriers:
+// nothing polls (a polling issuer measured ~4.3 TB/s on a bare stream of such
+// stages, a sleeping one ~5.1).  Consumer warp w takes four rows of every
+// stage as two row pairs -- gate/up: features 2w and 2w + 1 (gate row f with
+// up row 16 + f); down: rows 4w .. 4w + 3 -- lane l owns 16-byte chunks l and
+// 32 + l of each row (512 bytes apart, so every shared-memory load of the
+// warp reads 512 contiguous bytes), reads its activation values for those
+// elements once per token and uses them for all four rows, accumulating
+// 2 x 2 x NT partial sums in registers.  At the item's last stage the warp
+// adds its lanes' partial sums (a butterfly over the 2*NT values of each pair)
 // and writes
-//   gate/up: h[r, j + w] = act(g) * u   (f32 rows of the hidden activation)
-//   down:    y[dest_r, n + 2w + i] = scale_r * d_i (the pairs' slot rows
-//            weighted by the routing weight, or the shared expert's rows by
-//            its gate).
-// A down item of expert e needs the whole h rows of e: when all 16 warps of a
-// gate/up item have stored their h values (counted in shared memory), the
-// last one fences and adds 1 to the group's counter; a down item's warps wait
-// (bounded) until the count is complete before they read h, and remember
-// groups found complete, so later items of the group do not ask again.  The queue hands out all gate/up items first, expert by expert, so
-// the first down items find their experts finished long before; there is no
-// grid barrier between the two projections, and a CTA moves from gate/up rows
-// to down rows without draining its ring.  (Asking L2 for a batch of items
-// ahead of their copies measured slower: the prefetched rows of 148 CTAs
-// evict one another.)  A group with more than NT tokens
-// has one item per chunk of NT tokens, the chunks of a row block next to each
-// other in the queue so that the repeated weight rows come from L2.
+//   gate/up: h[r, j + f] = act(g) * u   (f32 rows of the hidden activation)
+//   down:    y[dest_r, n] = scale_r * d  (the pairs' slot rows weighted by
+//            the routing weight, or the shared expert's rows by its gate).
+// A down item of expert e needs the whole h rows of e: when the 8 consumer
+// warps of a gate/up item have stored their h values (counted in shared
+// memory), the last one fences and adds 1 to the group's counter.  Before the
+// issuing thread requests the first stage of a down item it waits (bounded)
+// until its group's count is complete, with an acquiring load; a proxy fence
+// then orders the copy engine's reads of h after the stores that count
+// published, and the group is remembered as complete.  While it waits, the
+// consumers go on with the stages already in the ring.  The queue hands out
+// all gate/up items first, expert by expert, and each CTA takes its items in
+// queue order, so a down item only waits for gate/up items ahead of it:
+// there is no grid barrier between the two projections, and a CTA moves from
+// gate/up rows to down rows without draining its ring.  (Asking L2 for a
+// batch of items ahead of their copies measured slower: the prefetched rows
+// of 148 CTAs evict one another.)  A group with more than NT tokens has one
+// item per chunk of NT tokens, the chunks of a row block next to each other
+// in the queue so that the repeated weight rows come from L2.
 //
 // Formats: f32 and bf16 weight rows, f32 or bf16 activations.  (A Q8_0 form
 // of the stream measured slower than the row-pair GEMV of stream_core.cuh,
@@ -57,10 +65,16 @@ using stream::WK_F32;
 constexpr int kStages = 4;            // ring depth
 constexpr int kRows = 32;             // weight rows per stage (and per item)
 constexpr int kRowBytes = 1024;       // bytes of one weight row in a stage (f32: 256 values)
-constexpr int kStageBytes = kRows * kRowBytes;    // 32 KB
+constexpr int kMaxNT = 4;             // most tokens per item
+constexpr int kActRow = 1024;         // bytes of one activation row in a stage (256 values, f32 or bf16)
+constexpr int kStageWBytes = kRows * kRowBytes;                // 32 KB of weight rows
+constexpr int kStageBytes = kStageWBytes + kMaxNT * kActRow;   // + the item's activation rows
 constexpr int kRingBytes = kStages * kStageBytes;
-static_assert(kStageBytes % 128 == 0 && (kRows / 2) * 512 % 128 == 0,
+static_assert(kStageWBytes % 128 == 0 && kStageBytes % 128 == 0 && kActRow % 128 == 0 && (kRows / 2) * 512 % 128 == 0,
               "every copy into the ring starts at a 128-byte boundary");
+
+// Tokens per item of a kernel instance built for at most maxt tokens (host and device).
+__host__ __device__ constexpr int item_tokens(int maxt) { return maxt == 1 ? 1 : kMaxNT; }
 
 // Elements of a row per stage (KC: 256, the widest box), bytes of a row per
 // stage (RB) and 16-byte chunks per lane and row (NCH).
@@ -77,10 +91,12 @@ struct Fmt {
 
 // Tensor maps of one layer: the weights of gate, up, down, shared gate, shared
 // up, shared down, in boxes 256 elements wide, 16 rows high for gate/up and
-// 32 for down.
-enum { M_GATE = 0, M_UP, M_DOWN, M_SGATE, M_SUP, M_SDOWN, M_COUNT };
+// 32 for down; the input x [T, H] in boxes of 256 x 1 row; the hidden rows h
+// [P, I] and h_s [T, Is] (f32) in boxes of 256 x h_box (hs_box) rows.
+enum { M_GATE = 0, M_UP, M_DOWN, M_SGATE, M_SUP, M_SDOWN, M_X, M_H, M_HS, M_COUNT };
 struct Maps {
   CUtensorMap w[M_COUNT];
+  int h_box, hs_box;
 };
 
 // Per-launch synchronisation words in the caller's workspace, zeroed by the
@@ -93,7 +109,6 @@ struct Sync {
 
 struct Params {
   int H, K, I, Is, act;
-  const void* x;       // [T, H] activations (XT)
   float* h;            // [P, I] hidden rows in expert-sorted order
   float* h_s;          // [T, Is] shared expert hidden rows
   float* y_slots;      // [P, H] weighted expert outputs, row = pair id
@@ -200,43 +215,53 @@ __device__ __forceinline__ Item decode_item(const Params& p, const Items& it, in
   return m;
 }
 
-// Thread 0: requests stage kc of item m (its 32 rows) into `st`, completing on `bar`.
-template <int WK>
-__device__ __forceinline__ void issue_stage(const Maps& maps, const Params& p, const Item& m, int kc, uint8_t* st,
-                                            uint64_t* bar) {
+// The issuing thread: requests stage kc of item m into `st`, completing on
+// `bar`: its 32 weight rows (wrow: first row of the item in its matrix) and
+// its activation rows -- gate/up: the x rows xrow[0..nt) of the item's
+// tokens; down: the box of h (or h_s) rows from row xrow[0].
+template <typename XT, int WK, int NT>
+__device__ __forceinline__ void issue_stage(const Maps& maps, const Item& m, int kc, int wrow, const int (&xrow)[NT],
+                                            uint8_t* st, uint64_t* bar) {
   constexpr int RB = Fmt<WK>::RB;
-  const int kx = kc * Fmt<WK>::KC;
-  mbar_arrive_expect_tx(bar, kRows * RB);
+  constexpr int KC = Fmt<WK>::KC;
+  const int kx = kc * KC;
   const uint64_t pol = l2_policy_evict_first();  // weight rows are read once (a repeated chunk: from L2 at once)
+  const uint64_t apol = l2_policy_evict_last();  // activation rows are read by many items
+  uint8_t* act = st + kStageWBytes;
   if (!m.down) {
-    const int row = (m.e < 0 ? 0 : m.e * p.I) + m.r0;
-    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SGATE : M_GATE], bar, kx, row, pol);
-    tma_load_2d_hint(st + (kRows / 2) * RB, &maps.w[m.e < 0 ? M_SUP : M_UP], bar, kx, row, pol);
+    mbar_arrive_expect_tx(bar, kRows * RB + m.nt * KC * static_cast<int>(sizeof(XT)));
+    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SGATE : M_GATE], bar, kx, wrow, pol);
+    tma_load_2d_hint(st + (kRows / 2) * RB, &maps.w[m.e < 0 ? M_SUP : M_UP], bar, kx, wrow, pol);
+#pragma unroll
+    for (int c = 0; c < NT; ++c)
+      if (c < m.nt) tma_load_2d_hint(act + c * kActRow, &maps.w[M_X], bar, kx, xrow[c], apol);
   } else {
-    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SDOWN : M_DOWN], bar, kx, (m.e < 0 ? 0 : m.e * p.H) + m.r0, pol);
+    const int hb = m.e < 0 ? maps.hs_box : maps.h_box;
+    mbar_arrive_expect_tx(bar, kRows * RB + hb * KC * 4);
+    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SDOWN : M_DOWN], bar, kx, wrow, pol);
+    tma_load_2d_hint(act, &maps.w[m.e < 0 ? M_HS : M_H], bar, kx, xrow[0], apol);
   }
 }
 
-// E16 activation values of a row at element k, as f32 pairs (L1 for the
-// layer's input x, L2 only for the h rows this kernel writes).
-template <typename AT, bool L2ONLY, int E16>
-__device__ __forceinline__ void act_chunk(const AT* row, int k, float2 (&x)[E16 / 2]) {
+// E16 activation values (type AT) at shared address `a`, as f32 pairs.
+template <typename AT, int E16>
+__device__ __forceinline__ void act_smem(uint32_t a, float2 (&x)[E16 / 2]) {
   if constexpr (sizeof(AT) == 4) {
 #pragma unroll
     for (int q = 0; q < E16 / 4; ++q) {
-      const float4* p4 = reinterpret_cast<const float4*>(row + k) + q;
-      const float4 a = L2ONLY ? __ldcg(p4) : __ldg(p4);
-      x[2 * q] = make_float2(a.x, a.y);
-      x[2 * q + 1] = make_float2(a.z, a.w);
+      const uint4 v = stream::lds16(a + 16 * q);
+      x[2 * q] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+      x[2 * q + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
     }
   } else if constexpr (E16 == 4) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(row + k));
-    x[0] = stream::bf16x2_f2(v.x);
-    x[1] = stream::bf16x2_f2(v.y);
+    uint32_t v0, v1;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(a));
+    x[0] = stream::bf16x2_f2(v0);
+    x[1] = stream::bf16x2_f2(v1);
   } else {
 #pragma unroll
     for (int q = 0; q < E16 / 8; ++q) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + k) + q);
+      const uint4 v = stream::lds16(a + 16 * q);
       x[4 * q] = stream::bf16x2_f2(v.x);
       x[4 * q + 1] = stream::bf16x2_f2(v.y);
       x[4 * q + 2] = stream::bf16x2_f2(v.z);
@@ -286,10 +311,20 @@ __device__ __forceinline__ float warp_reduce_many(float (&v)[V]) {
   return v[0];
 }
 
-// Wait until phase `parity` of `bar` completed; false after `limit` cycles
-// (decided by lane 0, so the outcome is warp-uniform).  All lanes.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit) {
-  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+// Shared state of the stream in one CTA (shared memory).
+constexpr int kMaxBatch = 4;  // most items handed out per queue step (fewer when there are few items per warp)
+constexpr int kCW = 8;        // consumer warps; warp kCW issues the copies; the rest sit the stream out
+struct Ring {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  Item item[kStages];      // the item a stage belongs to
+  int kc[kStages];         // the stage's index within its item; -1: the queue is empty
+  int done_warps[kStages]; // consumer warps done with the gate/up item ending in this stage
+};
+
+// Waits (bounded) until phase `parity` of `bar` completes, asleep on the barrier.  Every lane of the warp;
+// false (warp-uniform) if the wait gave up.
+__device__ __forceinline__ bool warp_sleep_wait(uint64_t* bar, uint32_t parity, long long limit) {
   const long long t0 = clock64();
   for (;;) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
@@ -297,21 +332,18 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
-// Shared state of the stream in one CTA (shared memory).
-constexpr int kMaxBatch = 4;  // most items handed out per queue step (fewer when there are few items per warp)
-struct Ring {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  Item item[kStages];      // the item a stage belongs to (decoded once, by the producer)
-  int kc[kStages];         // the stage's index within its item; -1: the queue is empty
-  int done_warps[kStages]; // warps of the gate/up item ending in this stage that have stored their h values
-  unsigned gdone[(kMaxGroups + 31) / 32];  // groups whose gate/up items are all finished (known to this CTA)
-};
-
 // The stream of one CTA, until the queue is empty.  All threads of the CTA
 // (16 warps).  Returns false if a wait gave up (MOE_ERR_TIMEOUT recorded).
 //   stages: kRingBytes of shared memory, 128-byte aligned
 //   pairs:  sorted pair ids;  wpair: routing weight per pair id;  sgate: shared-expert gate per token or nullptr
+//
+// Warp specialised: lane 0 of warp kCW issues every copy, asleep on a stage's empty barrier until the kCW
+// consumer warps have released it; the consumers sleep on the full barriers.  Nothing polls, and the
+// issuing thread may wait for the device-wide counters (the queue, a group's gate/up count) without
+// holding up the consumers, which go on with the stages already in the ring.  The queue puts every gate/up
+// item before every down item and each CTA takes items in queue order, so a down item only ever waits for
+// gate/up items that are ahead of it in some CTA's ring or queue order: none waits on a stage that waits
+// on it.
 template <typename XT, int WK, int NT>
 __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, const Items& it, uint8_t* stages,
                                            Ring& ring, const int32_t* pairs, const float* wpair, const float* sgate) {
@@ -319,65 +351,124 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
   constexpr int RB = Fmt<WK>::RB;
   constexpr int NCH = Fmt<WK>::NCH;
   constexpr int E16 = Fmt<WK>::E16;
+  constexpr int EB = Fmt<WK>::EB;
   constexpr int NV = 2 * NT;
+  static_assert(NT <= kMaxNT, "an item's activation rows fit its stage");
+  static_assert(kCW * 4 == kRows && kCW < kWarps, "a consumer warp takes four rows of a stage");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int total = it.gi[it.n] + it.di[it.n];
-  const bool producer = threadIdx.x == 0;
   // items per queue step: about 16 steps per CTA, at most kMaxBatch (large items are few: batching them
-  // would leave the CTAs unevenly loaded)
-  const int kBatch = max(1, min(kMaxBatch, total / (static_cast<int>(gridDim.x) * 16)));
-
-  // ---- issue side (thread 0): a cursor over (item, stage of the item) in queue order; items come in
-  // batches of kBatch consecutive ones, the next batch asked for while the current one is issued
-  int is_item = 0, is_end = 0, is_next = 0, is_kc = 0;
-  Item is_m{};
-  if (producer) {
+  // would leave the CTAs unevenly loaded).  The first batch is the CTA's own (batch blockIdx.x), the next
+  // ones come from the counter.
+  const int batch = max(1, min(kMaxBatch, total / (static_cast<int>(gridDim.x) * 16)));
+  if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ring.full[s], 1);
-      mbar_init(&ring.empty[s], kWarps);
+      mbar_init(&ring.empty[s], kCW);
+      ring.done_warps[s] = 0;
     }
-    for (int s = 0; s < kStages; ++s) ring.done_warps[s] = 0;
-    for (int i = 0; i < (kMaxGroups + 31) / 32; ++i) ring.gdone[i] = 0;
     fence_mbar_init();
-    is_item = static_cast<int>(atomicAdd(&p.sync->queue, 1u)) * kBatch;
-    is_end = min(total, is_item + kBatch);
-    is_next = static_cast<int>(atomicAdd(&p.sync->queue, 1u)) * kBatch;
-    if (is_item < is_end) is_m = decode_item<NT, WK>(p, it, is_item);
   }
-  auto issue = [&](int s) {  // thread 0: the next stage in queue order into ring stage s, or an end mark
-    while (is_item < is_end && is_kc >= is_m.nkc) {
-      if (++is_item >= is_end) {
-        is_item = is_next;
-        is_end = min(total, is_item + kBatch);
-        if (is_item < is_end)  // the batch after it, asked for now
-          is_next = static_cast<int>(atomicAdd(&p.sync->queue, 1u)) * kBatch;
-      }
-      is_kc = 0;
-      if (is_item < is_end) is_m = decode_item<NT, WK>(p, it, is_item);
-    }
-    if (is_item >= is_end) {
-      ring.kc[s] = -1;
-      mbar_arrive(&ring.full[s]);  // the end mark is published through the same barrier
-      return;
-    }
-    ring.item[s] = is_m;
-    ring.kc[s] = is_kc;
-    issue_stage<WK>(maps, p, is_m, is_kc, stages + s * kStageBytes, &ring.full[s]);
-    ++is_kc;
-  };
-  if (producer)
-    for (int s = 0; s < kStages; ++s) issue(s);
   __syncthreads();
-
-  // ---- compute side (every warp)
-  Item m{};
-  int arow[NT];  // activation row of each token of the chunk (x row for gate/up, h row for down)
-  float2 acc_a[NT], acc_b[NT];
   bool ok = true;
+
+  if (warp == kCW) {
+    // ---- the issuing thread: items in queue order, each batch's successor claimed when the batch starts
+    if (lane == 0) {
+      int item = static_cast<int>(blockIdx.x) * batch;
+      int end = min(total, item + batch);
+      int next = item < end ? (static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(&p.sync->queue, 1u))) * batch
+                            : total;
+      unsigned gdone[(kMaxGroups + 31) / 32];  // groups whose gate/up items are all finished (known here)
+#pragma unroll
+      for (int i = 0; i < (kMaxGroups + 31) / 32; ++i) gdone[i] = 0;
+      Item m{};
+      int kc = 0, wrow = 0;
+      int xr[NT];
+      bool have = false;
+      const long long t0 = clock64();
+      for (uint32_t seq = 0;; ++seq) {
+        const int s = static_cast<int>(seq % kStages);
+        if (seq >= kStages) {
+          while (!mbar_try_wait(&ring.empty[s], (seq / kStages - 1) & 1u))
+            if (clock64() - t0 > p.wait_limit) {
+              ok = false;
+              break;
+            }
+          if (!ok) break;
+        }
+        if (!have || kc >= m.nkc) {  // the next item, from this batch or the next
+          if (have && ++item >= end) {
+            item = next;
+            end = min(total, item + batch);
+            if (item < end) next = (static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(&p.sync->queue, 1u))) * batch;
+          }
+          have = true;
+          kc = 0;
+          if (item < end) {
+            m = decode_item<NT, WK>(p, it, item);
+            const int first = it.first[m.g];
+            if (!m.down) {
+              wrow = (m.e < 0 ? 0 : m.e * p.I) + m.r0;
+#pragma unroll
+              for (int k = 0; k < NT; ++k) {
+                const int t = m.t0 + min(k, m.nt - 1);
+                xr[k] = m.e < 0 ? t : pairs[first + t] / p.K;
+              }
+            } else {
+              wrow = (m.e < 0 ? 0 : m.e * p.H) + m.r0;
+#pragma unroll
+              for (int k = 0; k < NT; ++k) xr[k] = m.e < 0 ? m.t0 : first + m.t0;
+              if (!(gdone[m.g >> 5] >> (m.g & 31) & 1u)) {
+                // the item reads the h rows of its group: once every gate/up item of the group has counted
+                // itself; then a proxy fence orders the copy engine's reads after the stores it published
+                const unsigned need = static_cast<unsigned>(g_items(p, m.e, it.count[m.g], NT));
+                for (;;) {
+                  unsigned v;
+                  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&p.sync->done[m.g]) : "memory");
+                  if (v >= need) break;
+                  if (clock64() - t0 > p.wait_limit) {
+                    ok = false;
+                    break;
+                  }
+                  __nanosleep(200);
+                }
+                if (!ok) {  // the slot is free: an end mark stops the consumers at once
+                  ring.kc[s] = -1;
+                  mbar_arrive(&ring.full[s]);
+                  break;
+                }
+                fence_proxy_async_global();
+                gdone[m.g >> 5] |= 1u << (m.g & 31);
+              }
+            }
+          }
+        }
+        if (item >= end) {
+          ring.kc[s] = -1;
+          mbar_arrive(&ring.full[s]);  // the end mark is published through the same barrier
+          break;
+        }
+        ring.item[s] = m;
+        ring.kc[s] = kc;
+        issue_stage<XT, WK, NT>(maps, m, kc, wrow, xr, stages + s * kStageBytes, &ring.full[s]);
+        ++kc;
+      }
+      if (!ok) record_status(p.status, MOE_ERR_TIMEOUT);
+    }
+    __syncwarp();
+    return ok;
+  }
+  if (warp > kCW) return true;
+
+  // ---- consumers (warps 0 .. kCW-1): rows of pairs pi = 0, 1 -- gate/up: features f = 2w + pi (gate row f,
+  // up row 16 + f); down: rows 4w + 2pi and 4w + 2pi + 1
+  Item m{};
+  float2 acc_a[2][NT], acc_b[2][NT];
   for (uint32_t q = 0;; ++q) {
     const int s = static_cast<int>(q % kStages);
     const uint32_t par = (q / kStages) & 1u;
-    if (!warp_wait(&ring.full[s], par, p.wait_limit)) {
+    if (!warp_sleep_wait(&ring.full[s], par, p.wait_limit)) {
       record_status(p.status, MOE_ERR_TIMEOUT);
       ok = false;
       break;
@@ -386,127 +477,102 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
     if (kc < 0) break;
     if (kc == 0) {  // ---- the item begins
       m = ring.item[s];
-      const int first = it.first[m.g];
 #pragma unroll
-      for (int c = 0; c < NT; ++c) {
-        const int t = m.t0 + min(c, m.nt - 1);
-        arow[c] = m.e < 0 ? t : (m.down ? first + t : pairs[first + t] / p.K);
-        acc_a[c] = acc_b[c] = make_float2(0.f, 0.f);
-      }
-      if (m.down && !(ring.gdone[m.g >> 5] >> (m.g & 31) & 1u)) {
-        // the group's gate/up items are not known to be finished here: wait until the count is complete
-        const unsigned need = static_cast<unsigned>(g_items(p, m.e, it.count[m.g], NT));
-        int waited = 1;
-        if (lane == 0) {
-          const long long t0 = clock64();
-          for (;;) {
-            unsigned v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&p.sync->done[m.g]) : "memory");
-            if (v >= need) break;
-            if (clock64() - t0 > p.wait_limit) {
-              waited = 0;
-              break;
-            }
-          }
-          if (waited) atomicOr_block(&ring.gdone[m.g >> 5], 1u << (m.g & 31));
-        }
-        waited = __shfl_sync(0xffffffffu, waited, 0);
-        __syncwarp();
-        if (!waited) {
-          record_status(p.status, MOE_ERR_TIMEOUT);
-          ok = false;
-        }
-      }
+      for (int pi = 0; pi < 2; ++pi)
+#pragma unroll
+        for (int c = 0; c < NT; ++c) acc_a[pi][c] = acc_b[pi][c] = make_float2(0.f, 0.f);
     }
-    // ---- this stage: the warp's rows a and b, lane chunks ch = 0..NCH-1 at bytes ch*512 + lane*16
+    // ---- this stage: lane chunks ch = 0..NCH-1 at bytes ch*512 + lane*16 of the warp's rows; the
+    // activation rows of the item's tokens follow the weight rows
     const uint32_t st = smem_addr(stages + s * kStageBytes);
-    const int ra = m.down ? 2 * warp : warp, rb = m.down ? 2 * warp + 1 : kRows / 2 + warp;
-    const uint32_t wa_s = st + ra * RB, wb_s = st + rb * RB;
+    const uint32_t act = st + kStageWBytes;
 #pragma unroll
     for (int ch = 0; ch < NCH; ++ch) {
-      const int k = kc * KC + (ch * 512 + lane * 16) / Fmt<WK>::EB;
-      if (ok && k < m.kdim) {  // past the row (the last stage's tail): nothing to add
-        float2 wa[E16 / 2], wb[E16 / 2];
-        w_chunk<WK>(wa_s + ch * 512 + lane * 16, wa);
-        w_chunk<WK>(wb_s + ch * 512 + lane * 16, wb);
+      const int kl = (ch * 512 + lane * 16) / EB;  // element within the stage
+      if (kc * KC + kl < m.kdim) {  // past the row (the last stage's tail): nothing to add
+        float2 xv[NT][E16 / 2];
 #pragma unroll
         for (int c = 0; c < NT; ++c) {
           if (c < m.nt) {
-            float2 xv[E16 / 2];
             if (m.down)
-              act_chunk<float, true, E16>(m.e >= 0 ? p.h + static_cast<size_t>(arow[c]) * p.I
-                                                    : p.h_s + static_cast<size_t>(arow[c]) * p.Is,
-                                          k, xv);
+              act_smem<float, E16>(act + c * kActRow + kl * 4, xv[c]);
             else
-              act_chunk<XT, false, E16>(static_cast<const XT*>(p.x) + static_cast<size_t>(arow[c]) * p.H, k, xv);
+              act_smem<XT, E16>(act + c * kActRow + kl * static_cast<int>(sizeof(XT)), xv[c]);
+          }
+        }
 #pragma unroll
-            for (int i = 0; i < E16 / 2; ++i) {
-              acc_a[c] = __ffma2_rn(wa[i], xv[i], acc_a[c]);
-              acc_b[c] = __ffma2_rn(wb[i], xv[i], acc_b[c]);
+        for (int pi = 0; pi < 2; ++pi) {
+          const int ra = m.down ? 4 * warp + 2 * pi : 2 * warp + pi;
+          const int rb = m.down ? ra + 1 : kRows / 2 + ra;
+          float2 wa[E16 / 2], wb[E16 / 2];
+          w_chunk<WK>(st + ra * RB + ch * 512 + lane * 16, wa);
+          w_chunk<WK>(st + rb * RB + ch * 512 + lane * 16, wb);
+#pragma unroll
+          for (int c = 0; c < NT; ++c) {
+            if (c < m.nt) {
+#pragma unroll
+              for (int i = 0; i < E16 / 2; ++i) {
+                acc_a[pi][c] = __ffma2_rn(wa[i], xv[c][i], acc_a[pi][c]);
+                acc_b[pi][c] = __ffma2_rn(wb[i], xv[c][i], acc_b[pi][c]);
+              }
             }
           }
         }
       }
     }
-    if (ok && kc == m.nkc - 1) {  // ---- the item ends: add the lanes' sums and store
-      float v[NV];
-#pragma unroll
-      for (int c = 0; c < NT; ++c) {
-        v[c] = acc_a[c].x + acc_a[c].y;
-        v[NT + c] = acc_b[c].x + acc_b[c].y;
-      }
-      const float tot = warp_reduce_many<NV>(v);
-      constexpr int per = 32 / NV;  // lanes holding each total; value i sits in lanes [i*per, i*per + per)
-      const int vi = lane / per;
-      const int c = vi % NT;
+    if (kc == m.nkc - 1) {  // ---- the item ends: add the lanes' sums and store, pair by pair
       const int first = it.first[m.g];
-      const int t = m.t0 + min(c, m.nt - 1);
-      const int pr = m.e < 0 ? t : pairs[first + t];
-      if (!m.down) {
-        // row a (gate) totals are values [0, NT), row b (up) [NT, 2 NT): 16 lanes higher
-        const float u = __shfl_down_sync(0xffffffffu, tot, 16);
-        if (lane < 16 && lane % per == 0 && c < m.nt) {
-          const float hv = act_fn(p.act, tot) * u;
-          const int f = m.r0 + warp;
+#pragma unroll
+      for (int pi = 0; pi < 2; ++pi) {
+        float v[NV];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+          v[c] = acc_a[pi][c].x + acc_a[pi][c].y;
+          v[NT + c] = acc_b[pi][c].x + acc_b[pi][c].y;
+        }
+        const float tot = warp_reduce_many<NV>(v);
+        constexpr int per = 32 / NV;  // lanes holding each total; value i sits in lanes [i*per, i*per + per)
+        const int vi = lane / per;
+        const int c = vi % NT;
+        const int t = m.t0 + min(c, m.nt - 1);
+        const int pr = m.e < 0 ? t : pairs[first + t];
+        if (!m.down) {
+          // row a (gate) totals are values [0, NT), row b (up) [NT, 2 NT): 16 lanes higher
+          const float u = __shfl_down_sync(0xffffffffu, tot, 16);
+          if (lane < 16 && lane % per == 0 && c < m.nt) {
+            const float hv = act_fn(p.act, tot) * u;
+            const int f = m.r0 + 2 * warp + pi;
+            if (m.e < 0)
+              p.h_s[static_cast<size_t>(t) * p.Is + f] = hv;
+            else
+              p.h[static_cast<size_t>(first + t) * p.I + f] = hv;
+          }
+        } else if (lane % per == 0 && c < m.nt) {
+          const int n = m.r0 + 4 * warp + 2 * pi + vi / NT;  // rows 4w + 2pi, 4w + 2pi + 1 of the block
           if (m.e < 0)
-            p.h_s[static_cast<size_t>(t) * p.Is + f] = hv;
+            p.y_s[static_cast<size_t>(t) * p.H + n] = (sgate ? sgate[t] : 1.f) * tot;
           else
-            p.h[static_cast<size_t>(first + t) * p.I + f] = hv;
+            p.y_slots[static_cast<size_t>(pr) * p.H + n] = wpair[pr] * tot;
         }
-        // the item's 16 warps count themselves in shared memory; the last one makes all their h stores
-        // visible GPU-wide (the fence is cumulative over what it observed) and counts the item for its group
-        __threadfence_block();
+      }
+      if (!m.down) {
+        // the item's consumer warps count themselves in shared memory; the last one makes all their h
+        // stores visible GPU-wide (the fence is cumulative over what it observed) and counts the item for
+        // its group
         __syncwarp();
-        if (lane == 0 && atomicAdd_block(&ring.done_warps[s], 1) == kWarps - 1) {
-          ring.done_warps[s] = 0;  // ready for the next item ending in this stage (after the refill)
-          __threadfence();
-          atomicAdd(&p.sync->done[m.g], 1u);
+        if (lane == 0) {
+          __threadfence_block();
+          if (atomicAdd_block(&ring.done_warps[s], 1) == kCW - 1) {
+            ring.done_warps[s] = 0;  // ready for the next item ending in this stage (after the refill)
+            __threadfence();
+            atomicAdd(&p.sync->done[m.g], 1u);
+          }
         }
-      } else if (lane % per == 0 && c < m.nt) {
-        const int n = m.r0 + 2 * warp + vi / NT;  // rows 2w, 2w + 1 of the block
-        if (m.e < 0)
-          p.y_s[static_cast<size_t>(t) * p.H + n] = (sgate ? sgate[t] : 1.f) * tot;
-        else
-          p.y_slots[static_cast<size_t>(pr) * p.H + n] = wpair[pr] * tot;
       }
     }
-    // the warp is done with the stage (its shared memory, and the item-end count kept for it)
+    // the warp is done with the stage
     __syncwarp();
     if (lane == 0) mbar_arrive(&ring.empty[s]);
-    // thread 0 refills the stage once every warp has released it
-    if (producer) {
-      const long long t0 = clock64();
-      while (!mbar_try_wait(&ring.empty[s], par)) {
-        if (clock64() - t0 > p.wait_limit) {
-          record_status(p.status, MOE_ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
-      }
-      if (ok) issue(s);
-    }
-    ok = __shfl_sync(0xffffffffu, static_cast<int>(ok), 0) != 0;
-    if (!ok) break;
   }
   return ok;
 }
