@@ -107,6 +107,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// 4 bytes global -> shared without holding the thread (cp.async); cp_async_wait_all() before the data is used.
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(smem_dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Whether phase `parity` of `bar` has completed, without waiting (try_wait may suspend the thread for a
 // while before it answers no).
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {

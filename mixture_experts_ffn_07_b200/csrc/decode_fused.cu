@@ -89,13 +89,9 @@ __device__ __forceinline__ bool cta_grid_sync(const DecodeArgs& a, int* s_abort,
   return grid_sync(&g_decode_barrier, a.wait_limit, a.status, s_abort, s_flag);
 }
 
-// Partial logits of a block of router rows for one (hidden chunk, token group):
-// the CTA has staged the group's x chunk in shared memory as f32 (xs, rows of
-// kRouterChunk); warp w takes row r0 + w.  The chunk arithmetic is that of
-// route_util.cuh.  The row's chunk is requested whole before any product.
+// Router row r0 + warp's chunk ch into registers (requested whole; zeros past the row or past R).
 template <typename WT>
-__device__ __forceinline__ void router_rows(const DecodeArgs& a, const float* xs, int r0, int ch, int t0, int nt,
-                                            int R) {
+__device__ __forceinline__ void router_load(const DecodeArgs& a, int r0, int ch, int R, Raw8<WT> (&wr)[kRouterSteps]) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = r0 + warp;
   if (r >= R) return;
@@ -103,10 +99,22 @@ __device__ __forceinline__ void router_rows(const DecodeArgs& a, const float* xs
   const WT* wrow = (r < a.E ? static_cast<const WT*>(a.router) + static_cast<size_t>(r) * a.H
                             : static_cast<const WT*>(a.w_s)) +
                    h0;
-  Raw8<WT> wr[kRouterSteps];
 #pragma unroll
   for (int u = 0; u < kRouterSteps; ++u)
     if (lane * 8 + 256 * u < hc) raw_load(wrow + lane * 8 + 256 * u, wr[u]);
+}
+
+// Partial logits of a block of router rows for one (hidden chunk, token group):
+// the CTA has staged the group's x chunk in shared memory as f32 (xs, rows of
+// kRouterChunk); warp w takes row r0 + w, whose chunk it loaded into wr (router_load) before the
+// staging, so both loads are in flight together.  The chunk arithmetic is that of route_util.cuh.
+template <typename WT>
+__device__ __forceinline__ void router_rows(const DecodeArgs& a, const float* xs, int r0, int ch, int t0, int nt,
+                                            int R, const Raw8<WT> (&wr)[kRouterSteps]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = r0 + warp;
+  if (r >= R) return;
+  const int hc = min(kRouterChunk, a.H - ch * kRouterChunk);
   float acc[kTokGroup];
 #pragma unroll
   for (int c = 0; c < kTokGroup; ++c) acc[c] = 0.f;
@@ -137,17 +145,6 @@ __device__ __forceinline__ void router_rows(const DecodeArgs& a, const float* xs
   }
 }
 
-// Asks L2 for router row r's chunk ch (lane 0; skipped unless 16-byte aligned).
-__device__ __forceinline__ void router_prefetch_row(const DecodeArgs& a, int r, int ch, int R) {
-  if ((threadIdx.x & 31) != 0 || r >= R) return;
-  const size_t es = a.router_bf16 ? 2 : 4;
-  const int h0 = ch * kRouterChunk, hc = min(kRouterChunk, a.H - h0);
-  const uint8_t* p = r < a.E ? static_cast<const uint8_t*>(a.router) + (static_cast<size_t>(r) * a.H + h0) * es
-                             : static_cast<const uint8_t*>(a.w_s) + h0 * es;
-  const uint32_t bytes = static_cast<uint32_t>(hc * es);
-  if (((reinterpret_cast<uintptr_t>(p) | bytes) & 15u) == 0) prefetch_l2(p, bytes);
-}
-
 // Stages x[t0 .. t0+nt) [h0 .. h0+hc) as f32 rows of kRouterChunk.  All threads.
 template <typename XT>
 __device__ __forceinline__ void router_stage_x(const DecodeArgs& a, float* xs, int ch, int t0, int nt) {
@@ -163,6 +160,22 @@ __device__ __forceinline__ void router_stage_x(const DecodeArgs& a, float* xs, i
     dst[0] = make_float4(v[0], v[1], v[2], v[3]);
     dst[1] = make_float4(v[4], v[5], v[6], v[7]);
   }
+}
+
+// One R work item of a CTA: the row block's chunk requested, the x chunk staged (when it differs from the
+// one staged last), then the partial logits.  All threads.
+template <typename XT, typename WT>
+__device__ __forceinline__ void router_item(const DecodeArgs& a, float* xs, int rb, int cg, int ch, int t0, int nt,
+                                            int R, int& staged) {
+  Raw8<WT> wr[kRouterSteps];
+  router_load<WT>(a, rb * kWarps, ch, R, wr);
+  if (cg != staged) {
+    __syncthreads();
+    router_stage_x<XT>(a, xs, ch, t0, nt);
+    __syncthreads();
+    staged = cg;
+  }
+  router_rows<WT>(a, xs, rb * kWarps, ch, t0, nt, R, wr);
 }
 
 // MAXT: the most tokens of one expert batch (1 when T = 1: only single-token code, more loads in flight).
@@ -182,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_n, s_flag, s_abort;
   __shared__ int s_gi[kMaxGroups + 1], s_di[kMaxGroups + 1];
   __shared__ dstream::Ring s_ring;
+  __shared__ float s_bias[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = a.T, E = a.E, K = a.K, P = T * K;
   const int R = E + (a.w_s ? 1 : 0);
@@ -205,6 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (blockIdx.x == 0 && a.tma)  // the stream's queue and counters start at zero (visible after the barrier)
     for (int i = threadIdx.x; i < 1 + dstream::kMaxGroups; i += blockDim.x) reinterpret_cast<unsigned*>(a.sync)[i] = 0;
 
+  // the routing bias, copied to shared memory while R runs (it is read in S)
+  if (a.bias)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cp_async4(&s_bias[e], a.bias + e);
+
   // ---- R: partial router logits; a CTA item is (hidden chunk, token group, block of kWarps rows)
   {
     const int nch = (a.H + kRouterChunk - 1) / kRouterChunk;
@@ -217,19 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rb = i % nrb, cg = i / nrb;  // consecutive items of a CTA share their x chunk when they can
       const int ch = cg % nch, tg = cg / nch;
       const int t0 = tg * kTokGroup, nt = min(kTokGroup, T - t0);
-      if (cg != staged) {
-        router_prefetch_row(a, rb * kWarps + warp, ch, R);  // the row chunk's fetch overlaps the x staging
-        __syncthreads();
-        router_stage_x<XT>(a, xs, ch, t0, nt);
-        __syncthreads();
-        staged = cg;
-      }
       if (a.router_bf16)
-        router_rows<__nv_bfloat16>(a, xs, rb * kWarps, ch, t0, nt, R);
+        router_item<XT, __nv_bfloat16>(a, xs, rb, cg, ch, t0, nt, R, staged);
       else
-        router_rows<float>(a, xs, rb * kWarps, ch, t0, nt, R);
+        router_item<XT, float>(a, xs, rb, cg, ch, t0, nt, R, staged);
     }
   }
+  cp_async_wait_all();  // the bias copies (long done); the barrier's block sync publishes them
   debug_delay_cta0(a.barrier_delay);
   cta_grid_sync(a, &s_abort, &s_flag);
 
@@ -261,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane + 32 * i < R) row[lane + 32 * i] = l[i];
       __syncwarp();
       float* lout = blockIdx.x == 0 ? a.logits + static_cast<size_t>(t) * E : row;
-      warp_topk(row, a.bias, a.rc, lout, s_ids + t * K, s_w + t * K);
+      warp_topk(row, a.bias ? s_bias : nullptr, a.rc, lout, s_ids + t * K, s_w + t * K);
       if (a.w_s && lane == 0) {
         const float sg = 1.0f / (1.0f + expf(-row[E]));
         s_sgate[t] = sg;
