@@ -387,15 +387,15 @@ void moe_set_fused_front(int enable);
 void moe_set_pair_gemm(int enable);
 
 /* How the cooperative decode kernel (moe_set_fused_decode) runs gate/up and
- * down for f32 and bf16 weights: enable = 1 (default) as one stream of work
- * items (32 weight rows each, fed through the copy engine into a ring of 32 KB
- * stages per CTA, taken from a device-wide queue that hands out all gate/up
- * items, expert by expert, before the down items; a down item waits only for
- * its own expert's gate/up items); 0 as two phases separated by a grid
- * barrier, each CTA streaming a contiguous slice of the rows, which is how
- * Q8_0 and the k-quant stacks always run.  Same routing and the same values
- * up to the order of f32 additions.  Process-wide; takes effect at the next
- * call. */
+ * down for f32, bf16 and Q8_0 weights: enable = 1 (default) as one stream of
+ * work items (32 weight rows each, fed through the copy engine by one issuing
+ * warp into a ring of stages per CTA, taken from a device-wide queue that
+ * hands out all gate/up items, expert by expert, before the down items; a down
+ * item waits only for its own expert's gate/up items); 0 as two phases
+ * separated by a grid barrier, each CTA streaming a contiguous slice of the
+ * rows, which is how the k-quant stacks always run (and Q8_0 whose H, I or
+ * shared I is not a multiple of 256).  Same routing and the same values up to
+ * the order of f32 additions.  Process-wide; takes effect at the next call. */
 void moe_set_decode_stream(int enable);
 
 /* How the tensor-core path feeds the routed gate/up GEMM its x rows in expert

@@ -228,8 +228,8 @@ def set_pair_gemm(enable: bool) -> None:
 
 
 def set_decode_stream(enable: bool) -> None:
-    """moe_set_decode_stream: gate/up and down of the cooperative decode kernel for f32 / bf16 weights as one
-    TMA-fed stream of work items (True, default) or two phases with a grid barrier (False)."""
+    """moe_set_decode_stream: gate/up and down of the cooperative decode kernel for f32 / bf16 / Q8_0 weights
+    as one TMA-fed stream of work items (True, default) or two phases with a grid barrier (False)."""
     _lib.lib().moe_set_decode_stream(int(enable))
 
 

@@ -76,13 +76,11 @@ struct DecodeArgs {
   dstream::Sync* sync;     // queue and per-group counters of the stream (workspace)
 };
 
-// The formats the stream serves: one format for gate/up and down, f32 or bf16.  (A Q8_0 stream measured
-// slower than the Q8_0 row-pair GEMV -- q8_0_decode_t16 315 against 233 us: with ~1.5 tokens per expert its
-// items are one or two stages long and the per-item and per-token work dominates -- so Q8_0 and the
-// k-quant stacks keep the two phases.)
+// The formats the stream serves: one format for gate/up and down, f32, bf16 or Q8_0 (the k-quant stacks
+// keep the two phases).
 template <int WKG, int WKD>
 __host__ __device__ constexpr bool stream_format() {
-  return WKG == WKD && (WKG == WK_F32 || WKG == WK_BF16);
+  return WKG == WKD && (WKG == WK_F32 || WKG == WK_BF16 || WKG == WK_Q8);
 }
 
 __device__ __forceinline__ bool cta_grid_sync(const DecodeArgs& a, int* s_abort, int* s_flag) {
@@ -482,12 +480,14 @@ cudaError_t launch_fused_t(const Ctx& c, const DecodeArgs& a0, int P, const dstr
   auto kern = decode_layer_kernel<XT, WKG, WKD, MAXT>;
   DecodeArgs a = a0;
   if (!stream_format<WKG, WKD>()) a.tma = 0;
-  // the stream's per-warp rings reuse the stage area
-  if (a.tma) a.stage_bytes = std::max(a.stage_bytes, dstream::kRingBytes + 128);
+  const int st = static_smem<XT, WKG, WKD, MAXT>();
+  // the stream's ring reuses the stage area (the two phases take over if it does not fit)
+  const int ring = dstream::ring_bytes(WKG) + 128;
+  if (a.tma && std::max(a.stage_bytes, ring) + 16 * P + st > c.smem_optin) a.tma = 0;
+  if (a.tma) a.stage_bytes = std::max(a.stage_bytes, ring);
   // more than half of an SM's shared memory, so one CTA per SM whatever the register count: a CTA of a later
   // grid then starts only after this grid's last barrier (the barrier counter is shared by all launches)
   const int smem = std::max(a.stage_bytes + 16 * P, c.smem_optin / 2 + 1024);
-  const int st = static_smem<XT, WKG, WKD, MAXT>();
   if (st < 0 || smem + st > c.smem_optin) return cudaErrorInvalidValue;
   cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -597,11 +597,16 @@ bool stream_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int
   return true;
 }
 
-// The map of one weight matrix [rows, K] (f32 or bf16) for the stream, in boxes of 256 elements x box_rows;
-// false if its layout does not fit (misaligned pointer).
-bool weight_map(int wk, const void* w, uint64_t rows, uint64_t K, uint32_t box_rows, CUtensorMap* mw) {
+// The map of one weight matrix [rows, K] for the stream, in boxes of 256 elements (Q8_0: 256 32-bit words
+// of codes) x box_rows, and for Q8_0 the map of its fp16 scale plane [rows, K / 32] in boxes of 32 x box_rows;
+// false if the layout does not fit (misaligned pointer, K not whole 256-code units for Q8_0).
+bool weight_map(int wk, const void* w, const void* scale, uint64_t rows, uint64_t K, uint32_t box_rows,
+                CUtensorMap* mw, CUtensorMap* ms) {
   if (wk == WK_F32) return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, K, 256, box_rows);
-  return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 256, box_rows);
+  if (wk == WK_BF16) return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 256, box_rows);
+  if (K % 256) return false;
+  return stream_map(mw, w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, rows, K / 4, 256, box_rows) &&
+         stream_map(ms, scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, K / 32, 32, box_rows);
 }
 
 }  // namespace
@@ -693,30 +698,42 @@ cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L) {
   memset(&maps, 0, sizeof(maps));
   a.sync = static_cast<dstream::Sync*>(L.stream_sync);
   const int sw = stream_path_mode();
-  a.tma = L.stream_sync != nullptr && wkg == wkd && (wkg == WK_F32 || wkg == WK_BF16);
+  a.tma = L.stream_sync != nullptr && wkg == wkd && (wkg == WK_F32 || wkg == WK_BF16 || wkg == WK_Q8);
   if (a.tma) {
     using namespace dstream;
     const uint64_t E = L.E, H = L.H, I = L.I, Is = L.Is;
     constexpr uint32_t GR = kRows / 2, DR = kRows;  // boxes of 16 gate (or up) rows, 32 down rows
-    bool ok = weight_map(wkg, L.gate, E * I, H, GR, &maps.w[M_GATE]) &&
-              weight_map(wkg, L.up, E * I, H, GR, &maps.w[M_UP]) &&
-              weight_map(wkd, L.down, E * H, I, DR, &maps.w[M_DOWN]);
+    bool ok = weight_map(wkg, L.gate, L.gate_scale, E * I, H, GR, &maps.w[M_GATE], &maps.s[M_GATE]) &&
+              weight_map(wkg, L.up, L.up_scale, E * I, H, GR, &maps.w[M_UP], &maps.s[M_UP]) &&
+              weight_map(wkd, L.down, L.down_scale, E * H, I, DR, &maps.w[M_DOWN], &maps.s[M_DOWN]);
     if (ok && Is > 0)
-      ok = weight_map(wkg, L.sh_gate, Is, H, GR, &maps.w[M_SGATE]) &&
-           weight_map(wkg, L.sh_up, Is, H, GR, &maps.w[M_SUP]) &&
-           weight_map(wkd, L.sh_down, H, Is, DR, &maps.w[M_SDOWN]);
-    // activation rows: x in boxes of one row; h and h_s in boxes of the item's tokens (no taller than the
-    // matrix), the same kernel instance launch_fused picks for T
-    const uint32_t nt = static_cast<uint32_t>(item_tokens(L.T == 1 ? 1 : kDecodeTok));
+      ok = weight_map(wkg, L.sh_gate, L.sh_gate_scale, Is, H, GR, &maps.w[M_SGATE], &maps.s[M_SGATE]) &&
+           weight_map(wkg, L.sh_up, L.sh_up_scale, Is, H, GR, &maps.w[M_SUP], &maps.s[M_SUP]) &&
+           weight_map(wkd, L.sh_down, L.sh_down_scale, H, Is, DR, &maps.w[M_SDOWN], &maps.s[M_SDOWN]);
     const uint64_t T = L.T, P = T * L.K;
-    maps.h_box = static_cast<int>(std::min<uint64_t>(nt, P));
-    maps.hs_box = static_cast<int>(std::min<uint64_t>(nt, T));
-    if (ok)
-      ok = (L.x_dtype == MOE_F32 ? stream_map(&maps.w[M_X], L.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, H, 256, 1)
-                                 : stream_map(&maps.w[M_X], L.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, H, 256, 1)) &&
-           stream_map(&maps.w[M_H], L.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P, I, 256, maps.h_box);
-    if (ok && Is > 0)
-      ok = stream_map(&maps.w[M_HS], L.h_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, Is, 256, maps.hs_box);
+    const bool xf = L.x_dtype == MOE_F32;
+    const CUtensorMapDataType xdt = xf ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int xes = xf ? 4 : 2;
+    if (wkg == WK_Q8) {
+      // activations as rows of 256 values, four of them (one token's 1024 values) per box
+      ok = ok && H % 256 == 0 && I % 256 == 0 && Is % 256 == 0;
+      if (ok)
+        ok = stream_map(&maps.w[M_X], L.x, xdt, xes, T * H / 256, 256, 256, 4) &&
+             stream_map(&maps.w[M_H], L.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P * I / 256, 256, 256, 4);
+      if (ok && Is > 0)
+        ok = stream_map(&maps.w[M_HS], L.h_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T * Is / 256, 256, 256, 4);
+    } else {
+      // x in boxes of one row; h and h_s in boxes of the item's tokens (no taller than the matrix), the same
+      // kernel instance launch_fused picks for T
+      const uint32_t nt = static_cast<uint32_t>(item_tokens(L.T == 1 ? 1 : kDecodeTok));
+      maps.h_box = static_cast<int>(std::min<uint64_t>(nt, P));
+      maps.hs_box = static_cast<int>(std::min<uint64_t>(nt, T));
+      if (ok)
+        ok = stream_map(&maps.w[M_X], L.x, xdt, xes, T, H, 256, 1) &&
+             stream_map(&maps.w[M_H], L.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P, I, 256, maps.h_box);
+      if (ok && Is > 0)
+        ok = stream_map(&maps.w[M_HS], L.h_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, Is, 256, maps.hs_box);
+    }
     a.tma = ok && sw != 0;
   }
   return launch_by_kind(c, a, P, L.x_dtype == MOE_F32, wkg, wkd, maps);

@@ -61,41 +61,56 @@ namespace dstream {
 using stream::kWarps;
 using stream::WK_BF16;
 using stream::WK_F32;
+using stream::WK_Q8;
 
 constexpr int kStages = 4;            // ring depth
 constexpr int kRows = 32;             // weight rows per stage (and per item)
-constexpr int kRowBytes = 1024;       // bytes of one weight row in a stage (f32: 256 values)
+constexpr int kRowBytes = 1024;       // bytes of one weight row in a stage (f32: 256 values, Q8_0: 1024 codes)
 constexpr int kMaxNT = 4;             // most tokens per item
-constexpr int kActRow = 1024;         // bytes of one activation row in a stage (256 values, f32 or bf16)
-constexpr int kStageWBytes = kRows * kRowBytes;                // 32 KB of weight rows
-constexpr int kStageBytes = kStageWBytes + kMaxNT * kActRow;   // + the item's activation rows
-constexpr int kRingBytes = kStages * kStageBytes;
-static_assert(kStageWBytes % 128 == 0 && kStageBytes % 128 == 0 && kActRow % 128 == 0 && (kRows / 2) * 512 % 128 == 0,
-              "every copy into the ring starts at a 128-byte boundary");
+constexpr int kStageWBytes = kRows * kRowBytes;  // 32 KB of weight rows
 
 // Tokens per item of a kernel instance built for at most maxt tokens (host and device).
 __host__ __device__ constexpr int item_tokens(int maxt) { return maxt == 1 ? 1 : kMaxNT; }
 
-// Elements of a row per stage (KC: 256, the widest box), bytes of a row per
-// stage (RB) and 16-byte chunks per lane and row (NCH).
+// Geometry of a stage by weight format.  KC: row elements per stage (256 f32 / bf16 values -- a box is at
+// most 256 wide --, 1024 Q8_0 codes as 256 words); RB: bytes of a row in a stage (bf16 rows fill half of
+// kRowBytes); NCH: 16-byte chunks per lane and row; E16: elements per chunk;
+// AR: bytes of one activation row of the stage (KC values, room for f32); SR: bytes of the fp16 scales of
+// one row (Q8_0: 32 blocks).  A stage is [kRows weight rows][kMaxNT activation rows][kRows scale rows].
 template <int WK>
 struct Fmt {
-  static_assert(WK == WK_F32 || WK == WK_BF16, "the stream serves f32 and bf16 weights");
-  static constexpr int EB = WK == WK_F32 ? 4 : 2;
-  static constexpr int KC = 256;                       // row elements per stage
-  static constexpr int RB = KC * EB;                   // bytes of a row in a stage
-  static constexpr int NCH = RB / 512;                 // 16-byte chunks per lane and row
-  static constexpr int E16 = 16 / EB;                  // elements per chunk
-  static_assert(RB % 512 == 0 && RB <= kRowBytes, "a stage row is whole 512-byte runs");
+  static_assert(WK == WK_F32 || WK == WK_BF16 || WK == WK_Q8, "the stream serves f32, bf16 and Q8_0 weights");
+  static constexpr int EB = WK == WK_F32 ? 4 : (WK == WK_BF16 ? 2 : 1);
+  static constexpr int KC = WK == WK_Q8 ? 1024 : 256;
+  static constexpr int RB = KC * EB;
+  static constexpr int NCH = RB / 512;
+  static constexpr int E16 = 16 / EB;
+  static constexpr int AR = KC * 4;
+  static constexpr int SR = WK == WK_Q8 ? KC / 32 * 2 : 0;
+  static constexpr int ACT = kStageWBytes;                  // offset of the activation rows
+  static constexpr int SCL = ACT + kMaxNT * AR;             // offset of the scale rows
+  static constexpr int SB = (SCL + kRows * SR + 127) / 128 * 128;  // stage bytes
+  static_assert(RB % 512 == 0 && RB <= kRowBytes && AR % 128 == 0 && SCL % 128 == 0 && (kRows / 2) * SR % 64 == 0,
+                "every copy into the ring starts at a 128-byte boundary (scale halves at 64)");
 };
 
+// Shared memory of the ring by weight format (host and device).
+__host__ __device__ constexpr int ring_bytes(int wk) {
+  return kStages * (wk == WK_Q8 ? Fmt<WK_Q8>::SB : (wk == WK_BF16 ? Fmt<WK_BF16>::SB : Fmt<WK_F32>::SB));
+}
+
 // Tensor maps of one layer: the weights of gate, up, down, shared gate, shared
-// up, shared down, in boxes 256 elements wide, 16 rows high for gate/up and
-// 32 for down; the input x [T, H] in boxes of 256 x 1 row; the hidden rows h
-// [P, I] and h_s [T, Is] (f32) in boxes of 256 x h_box (hs_box) rows.
+// up, shared down, in boxes 256 elements wide (Q8_0: 256 32-bit words of codes),
+// 16 rows high for gate/up and 32 for down, and for Q8_0 their fp16 scale
+// planes in boxes of 32 x as many rows; the input x; the hidden rows h [P, I]
+// and h_s [T, Is] (f32).  For f32 / bf16 weights x comes in boxes of 256 x 1
+// row and h (h_s) in boxes of 256 x h_box (hs_box) rows; for Q8_0 all three are
+// seen as rows of 256 values ([T * H / 256, 256] and so on) in boxes of 4 such
+// rows: the 1024 values of one token that a stage needs.
 enum { M_GATE = 0, M_UP, M_DOWN, M_SGATE, M_SUP, M_SDOWN, M_X, M_H, M_HS, M_COUNT };
 struct Maps {
   CUtensorMap w[M_COUNT];
+  CUtensorMap s[M_SDOWN + 1];
   int h_box, hs_box;
 };
 
@@ -186,20 +201,26 @@ struct Item {
   int nkc;    // stages of the item
 };
 
+// Item idx of the queue; `hint` is a group to try before searching (the previous item's: consecutive items
+// of a CTA are mostly in one group).
 template <int NT, int WK>
-__device__ __forceinline__ Item decode_item(const Params& p, const Items& it, int idx) {
+__device__ __forceinline__ Item decode_item(const Params& p, const Items& it, int idx, int hint = 0) {
   Item m;
   const int ng = it.gi[it.n];
   m.down = idx >= ng;
   const int* off = m.down ? it.di : it.gi;
   const int v = m.down ? idx - ng : idx;
   int lo = 0, hi = it.n - 1;  // largest g with off[g] <= v
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (off[mid] <= v)
-      lo = mid;
-    else
-      hi = mid - 1;
+  if (hint >= 0 && hint < it.n && off[hint] <= v && v < off[hint + 1]) {
+    lo = hint;
+  } else {
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off[mid] <= v)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
   }
   m.g = lo;
   m.e = it.expert[lo];
@@ -216,30 +237,51 @@ __device__ __forceinline__ Item decode_item(const Params& p, const Items& it, in
 }
 
 // The issuing thread: requests stage kc of item m into `st`, completing on
-// `bar`: its 32 weight rows (wrow: first row of the item in its matrix) and
-// its activation rows -- gate/up: the x rows xrow[0..nt) of the item's
-// tokens; down: the box of h (or h_s) rows from row xrow[0].
+// `bar`: its 32 weight rows (wrow: first row of the item in its matrix; Q8_0
+// also their scales) and its activation rows -- gate/up: the x rows xrow[0..nt)
+// of the item's tokens; down: the h (or h_s) rows from row xrow[0].
+//   pol: L2 policy of the weight rows (evict first: read once; a repeated chunk comes from L2 at once);
+//   apol: of the activation rows (evict last: read by many items)
 template <typename XT, int WK, int NT>
-__device__ __forceinline__ void issue_stage(const Maps& maps, const Item& m, int kc, int wrow, const int (&xrow)[NT],
-                                            uint8_t* st, uint64_t* bar) {
-  constexpr int RB = Fmt<WK>::RB;
-  constexpr int KC = Fmt<WK>::KC;
-  const int kx = kc * KC;
-  const uint64_t pol = l2_policy_evict_first();  // weight rows are read once (a repeated chunk: from L2 at once)
-  const uint64_t apol = l2_policy_evict_last();  // activation rows are read by many items
-  uint8_t* act = st + kStageWBytes;
+__device__ __forceinline__ void issue_stage(const Maps& maps, const Params& p, const Item& m, int kc, int wrow,
+                                            const int (&xrow)[NT], uint8_t* st, uint64_t* bar, uint64_t pol,
+                                            uint64_t apol) {
+  using F = Fmt<WK>;
+  constexpr bool Q8 = WK == WK_Q8;
+  const int kx = kc * (Q8 ? F::KC / 4 : F::KC);  // Q8_0 codes as 32-bit words
+  uint8_t* act = st + F::ACT;
+  uint8_t* sc = st + F::SCL;
+  const int ax = Q8 ? 0 : kx;  // activation copies: Q8_0 reads 4 rows of the 256-value view
   if (!m.down) {
-    mbar_arrive_expect_tx(bar, kRows * RB + m.nt * KC * static_cast<int>(sizeof(XT)));
-    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SGATE : M_GATE], bar, kx, wrow, pol);
-    tma_load_2d_hint(st + (kRows / 2) * RB, &maps.w[m.e < 0 ? M_SUP : M_UP], bar, kx, wrow, pol);
+    const int xb = F::KC * static_cast<int>(sizeof(XT));
+    mbar_arrive_expect_tx(bar, kRows * F::RB + kRows * F::SR + m.nt * xb);
+    const int mg = m.e < 0 ? M_SGATE : M_GATE, mu = m.e < 0 ? M_SUP : M_UP;
+    tma_load_2d_hint(st, &maps.w[mg], bar, kx, wrow, pol);
+    tma_load_2d_hint(st + (kRows / 2) * F::RB, &maps.w[mu], bar, kx, wrow, pol);
+    if constexpr (Q8) {
+      tma_load_2d_hint(sc, &maps.s[mg], bar, kc * 32, wrow, pol);
+      tma_load_2d_hint(sc + (kRows / 2) * F::SR, &maps.s[mu], bar, kc * 32, wrow, pol);
+    }
 #pragma unroll
     for (int c = 0; c < NT; ++c)
-      if (c < m.nt) tma_load_2d_hint(act + c * kActRow, &maps.w[M_X], bar, kx, xrow[c], apol);
+      if (c < m.nt)
+        tma_load_2d_hint(act + c * F::AR, &maps.w[M_X], bar, ax, Q8 ? xrow[c] * (p.H / 256) + kc * 4 : xrow[c], apol);
   } else {
-    const int hb = m.e < 0 ? maps.hs_box : maps.h_box;
-    mbar_arrive_expect_tx(bar, kRows * RB + hb * KC * 4);
-    tma_load_2d_hint(st, &maps.w[m.e < 0 ? M_SDOWN : M_DOWN], bar, kx, wrow, pol);
-    tma_load_2d_hint(act, &maps.w[m.e < 0 ? M_HS : M_H], bar, kx, xrow[0], apol);
+    const int md = m.e < 0 ? M_SDOWN : M_DOWN, mh = m.e < 0 ? M_HS : M_H;
+    if constexpr (Q8) {
+      mbar_arrive_expect_tx(bar, kRows * F::RB + kRows * F::SR + m.nt * F::AR);
+      tma_load_2d_hint(st, &maps.w[md], bar, kx, wrow, pol);
+      tma_load_2d_hint(sc, &maps.s[md], bar, kc * 32, wrow, pol);
+      const int per = (m.e < 0 ? p.Is : p.I) / 256;
+#pragma unroll
+      for (int c = 0; c < NT; ++c)
+        if (c < m.nt) tma_load_2d_hint(act + c * F::AR, &maps.w[mh], bar, 0, (xrow[0] + c) * per + kc * 4, apol);
+    } else {
+      const int hb = m.e < 0 ? maps.hs_box : maps.h_box;
+      mbar_arrive_expect_tx(bar, kRows * F::RB + hb * F::KC * 4);
+      tma_load_2d_hint(st, &maps.w[md], bar, kx, wrow, pol);
+      tma_load_2d_hint(act, &maps.w[mh], bar, kx, xrow[0], apol);
+    }
   }
 }
 
@@ -277,11 +319,16 @@ __device__ __forceinline__ void w_chunk(uint32_t a, float2 (&w)[Fmt<WK>::E16 / 2
   if constexpr (WK == WK_F32) {
     w[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
     w[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
-  } else {
+  } else if constexpr (WK == WK_BF16) {
     w[0] = stream::bf16x2_f2(v.x);
     w[1] = stream::bf16x2_f2(v.y);
     w[2] = stream::bf16x2_f2(v.z);
     w[3] = stream::bf16x2_f2(v.w);
+  } else {  // Q8_0 codes, widened exactly
+    stream::q8_quad(v.x, w[0], w[1]);
+    stream::q8_quad(v.y, w[2], w[3]);
+    stream::q8_quad(v.z, w[4], w[5]);
+    stream::q8_quad(v.w, w[6], w[7]);
   }
 }
 
@@ -314,12 +361,15 @@ __device__ __forceinline__ float warp_reduce_many(float (&v)[V]) {
 // Shared state of the stream in one CTA (shared memory).
 constexpr int kMaxBatch = 4;  // most items handed out per queue step (fewer when there are few items per warp)
 constexpr int kCW = 8;        // consumer warps; warp kCW issues the copies; the rest sit the stream out
+constexpr int kDoneQ = 32;    // finished gate/up items waiting to be counted (at most one per stage in flight)
 struct Ring {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   Item item[kStages];      // the item a stage belongs to
   int kc[kStages];         // the stage's index within its item; -1: the queue is empty
   int done_warps[kStages]; // consumer warps done with the gate/up item ending in this stage
+  int dq[kDoneQ];          // group + 1 of each finished gate/up item, in claim order (0: not yet written)
+  int dq_tail;             // items claimed a place in dq (consumers)
 };
 
 // Waits (bounded) until phase `parity` of `bar` completes, asleep on the barrier.  Every lane of the warp;
@@ -334,7 +384,7 @@ __device__ __forceinline__ bool warp_sleep_wait(uint64_t* bar, uint32_t parity, 
 
 // The stream of one CTA, until the queue is empty.  All threads of the CTA
 // (16 warps).  Returns false if a wait gave up (MOE_ERR_TIMEOUT recorded).
-//   stages: kRingBytes of shared memory, 128-byte aligned
+//   stages: ring_bytes(WK) of shared memory, 128-byte aligned
 //   pairs:  sorted pair ids;  wpair: routing weight per pair id;  sgate: shared-expert gate per token or nullptr
 //
 // Warp specialised: lane 0 of warp kCW issues every copy, asleep on a stage's empty barrier until the kCW
@@ -367,6 +417,8 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
       mbar_init(&ring.empty[s], kCW);
       ring.done_warps[s] = 0;
     }
+    for (int i = 0; i < kDoneQ; ++i) ring.dq[i] = 0;
+    ring.dq_tail = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -375,10 +427,17 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
   if (warp == kCW) {
     // ---- the issuing thread: items in queue order, each batch's successor claimed when the batch starts
     if (lane == 0) {
+      auto claim = [&]() {
+        return (static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(&p.sync->queue, 1u))) * batch;
+      };
       int item = static_cast<int>(blockIdx.x) * batch;
       int end = min(total, item + batch);
-      int next = item < end ? (static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(&p.sync->queue, 1u))) * batch
-                            : total;
+      // the batches after this one, claimed two ahead so that the counter's answer is there when needed
+      // (claims of one CTA only grow: a claim past the end ends its stream)
+      int next = item < end ? claim() : total;
+      int next2 = next < total ? claim() : total;
+      const uint64_t pol = l2_policy_evict_first(), apol = l2_policy_evict_last();
+      const int kshift = (p.K & (p.K - 1)) == 0 ? __ffs(p.K) - 1 : -1;  // pair -> token without a division
       unsigned gdone[(kMaxGroups + 31) / 32];  // groups whose gate/up items are all finished (known here)
 #pragma unroll
       for (int i = 0; i < (kMaxGroups + 31) / 32; ++i) gdone[i] = 0;
@@ -386,9 +445,30 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
       int kc = 0, wrow = 0;
       int xr[NT];
       bool have = false;
+      int dq_head = 0;
+      // finished gate/up items, counted for their groups: the consumers' last warp of an item wrote the
+      // entry after its item's h stores (ordered by a block fence); this thread observes the entry, and its
+      // GPU fence, cumulative over what it observed, makes those stores visible before the count
+      auto drain = [&]() {
+        for (;;) {
+          const int g1 = *reinterpret_cast<volatile int*>(&ring.dq[dq_head % kDoneQ]);
+          if (g1 == 0) return;
+          __threadfence_block();
+          *reinterpret_cast<volatile int*>(&ring.dq[dq_head % kDoneQ]) = 0;
+          ++dq_head;
+          __threadfence();
+          atomicAdd(&p.sync->done[g1 - 1], 1u);
+        }
+      };
       const long long t0 = clock64();
+      // no CTA issues more stages than the whole queue holds: a bound that ends the loop whatever happens
+      const long long most = static_cast<long long>(total) * ((max(p.H, max(p.I, p.Is)) + KC - 1) / KC) + kStages;
       for (uint32_t seq = 0;; ++seq) {
         const int s = static_cast<int>(seq % kStages);
+        if (seq > most) {
+          ok = false;
+          break;
+        }
         if (seq >= kStages) {
           while (!mbar_try_wait(&ring.empty[s], (seq / kStages - 1) & 1u))
             if (clock64() - t0 > p.wait_limit) {
@@ -397,23 +477,27 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
             }
           if (!ok) break;
         }
+        drain();
         if (!have || kc >= m.nkc) {  // the next item, from this batch or the next
           if (have && ++item >= end) {
             item = next;
+            next = next2;
             end = min(total, item + batch);
-            if (item < end) next = (static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(&p.sync->queue, 1u))) * batch;
+            if (next2 < total) next2 = claim();
           }
+          const int hint = have ? m.g : 0;
           have = true;
           kc = 0;
           if (item < end) {
-            m = decode_item<NT, WK>(p, it, item);
+            m = decode_item<NT, WK>(p, it, item, hint);
             const int first = it.first[m.g];
             if (!m.down) {
               wrow = (m.e < 0 ? 0 : m.e * p.I) + m.r0;
 #pragma unroll
               for (int k = 0; k < NT; ++k) {
                 const int t = m.t0 + min(k, m.nt - 1);
-                xr[k] = m.e < 0 ? t : pairs[first + t] / p.K;
+                const int pr = pairs[first + t];
+                xr[k] = m.e < 0 ? t : (kshift >= 0 ? pr >> kshift : pr / p.K);
               }
             } else {
               wrow = (m.e < 0 ? 0 : m.e * p.H) + m.r0;
@@ -424,6 +508,7 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
                 // itself; then a proxy fence orders the copy engine's reads after the stores it published
                 const unsigned need = static_cast<unsigned>(g_items(p, m.e, it.count[m.g], NT));
                 for (;;) {
+                  drain();  // this CTA's own finished items may be what the group waits for
                   unsigned v;
                   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&p.sync->done[m.g]) : "memory");
                   if (v >= need) break;
@@ -447,11 +532,20 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
         if (item >= end) {
           ring.kc[s] = -1;
           mbar_arrive(&ring.full[s]);  // the end mark is published through the same barrier
+          // the stages still in flight may end gate/up items: once the consumers have released every one
+          // of them, count the last finished items
+          for (uint32_t n = seq > kStages ? seq - kStages : 0; n < seq && ok; ++n)
+            while (!mbar_try_wait(&ring.empty[n % kStages], (n / kStages) & 1u))
+              if (clock64() - t0 > p.wait_limit) {
+                ok = false;
+                break;
+              }
+          drain();
           break;
         }
         ring.item[s] = m;
         ring.kc[s] = kc;
-        issue_stage<XT, WK, NT>(maps, m, kc, wrow, xr, stages + s * kStageBytes, &ring.full[s]);
+        issue_stage<XT, WK, NT>(maps, p, m, kc, wrow, xr, stages + s * Fmt<WK>::SB, &ring.full[s], pol, apol);
         ++kc;
       }
       if (!ok) record_status(p.status, MOE_ERR_TIMEOUT);
@@ -483,89 +577,168 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
         for (int c = 0; c < NT; ++c) acc_a[pi][c] = acc_b[pi][c] = make_float2(0.f, 0.f);
     }
     // ---- this stage: lane chunks ch = 0..NCH-1 at bytes ch*512 + lane*16 of the warp's rows; the
-    // activation rows of the item's tokens follow the weight rows
-    const uint32_t st = smem_addr(stages + s * kStageBytes);
-    const uint32_t act = st + kStageWBytes;
+    // activation rows of the item's tokens follow the weight rows, then (Q8_0) the rows' scales
+    const uint32_t st = smem_addr(stages + s * Fmt<WK>::SB);
+    const uint32_t act = st + Fmt<WK>::ACT;
+    if constexpr (WK == WK_Q8) {
+      // a lane's 16 codes of a row are half a block: partial = sum q * x over them, then acc += d * partial.
+      // Token by token, the four rows' chains side by side (the codes are widened again per token: most
+      // items have one or two tokens).
+      const int r0 = m.down ? 4 * warp : 2 * warp, r1 = m.down ? r0 + 1 : kRows / 2 + r0;
+      const int r2 = m.down ? r0 + 2 : r0 + 1, r3 = m.down ? r0 + 3 : kRows / 2 + r0 + 1;
+      const int rows[4] = {r0, r1, r2, r3};
+      float d[NCH][4];
 #pragma unroll
-    for (int ch = 0; ch < NCH; ++ch) {
-      const int kl = (ch * 512 + lane * 16) / EB;  // element within the stage
-      if (kc * KC + kl < m.kdim) {  // past the row (the last stage's tail): nothing to add
-        float2 xv[NT][E16 / 2];
+      for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
-        for (int c = 0; c < NT; ++c) {
-          if (c < m.nt) {
-            if (m.down)
-              act_smem<float, E16>(act + c * kActRow + kl * 4, xv[c]);
-            else
-              act_smem<XT, E16>(act + c * kActRow + kl * static_cast<int>(sizeof(XT)), xv[c]);
-          }
+        for (int j = 0; j < 4; ++j) {
+          uint16_t hv;
+          asm volatile("ld.shared.u16 %0, [%1];"
+                       : "=h"(hv)
+                       : "r"(st + Fmt<WK>::SCL + rows[j] * Fmt<WK>::SR + ((ch * 512 + lane * 16) / 32) * 2));
+          d[ch][j] = __half2float(__ushort_as_half(hv));
         }
 #pragma unroll
-        for (int pi = 0; pi < 2; ++pi) {
-          const int ra = m.down ? 4 * warp + 2 * pi : 2 * warp + pi;
-          const int rb = m.down ? ra + 1 : kRows / 2 + ra;
-          float2 wa[E16 / 2], wb[E16 / 2];
-          w_chunk<WK>(st + ra * RB + ch * 512 + lane * 16, wa);
-          w_chunk<WK>(st + rb * RB + ch * 512 + lane * 16, wb);
+      for (int c = 0; c < NT; ++c) {
+        if (c >= m.nt) break;
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) {
+          const int kl = ch * 512 + lane * 16;  // code within the stage
+          if (kc * KC + kl < m.kdim) {
+            float2 xv[8];
+            if (m.down)
+              act_smem<float, 16>(act + c * Fmt<WK>::AR + kl * 4, xv);
+            else
+              act_smem<XT, 16>(act + c * Fmt<WK>::AR + kl * static_cast<int>(sizeof(XT)), xv);
+            float2 pr[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float2 w[8];
+              w_chunk<WK>(st + rows[j] * RB + kl, w);
+              float2 e = __fmul2_rn(w[0], xv[0]), o = __fmul2_rn(w[1], xv[1]);
+#pragma unroll
+              for (int i = 2; i < 8; i += 2) {
+                e = __ffma2_rn(w[i], xv[i], e);
+                o = __ffma2_rn(w[i + 1], xv[i + 1], o);
+              }
+              pr[j] = __fadd2_rn(e, o);
+            }
+            acc_a[0][c] = __ffma2_rn(make_float2(d[ch][0], d[ch][0]), pr[0], acc_a[0][c]);
+            acc_b[0][c] = __ffma2_rn(make_float2(d[ch][1], d[ch][1]), pr[1], acc_b[0][c]);
+            acc_a[1][c] = __ffma2_rn(make_float2(d[ch][2], d[ch][2]), pr[2], acc_a[1][c]);
+            acc_b[1][c] = __ffma2_rn(make_float2(d[ch][3], d[ch][3]), pr[3], acc_b[1][c]);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        const int kl = (ch * 512 + lane * 16) / EB;  // element within the stage
+        if (kc * KC + kl < m.kdim) {  // past the row (the last stage's tail): nothing to add
+          float2 xv[NT][E16 / 2];
 #pragma unroll
           for (int c = 0; c < NT; ++c) {
             if (c < m.nt) {
+              if (m.down)
+                act_smem<float, E16>(act + c * Fmt<WK>::AR + kl * 4, xv[c]);
+              else
+                act_smem<XT, E16>(act + c * Fmt<WK>::AR + kl * static_cast<int>(sizeof(XT)), xv[c]);
+            }
+          }
 #pragma unroll
-              for (int i = 0; i < E16 / 2; ++i) {
-                acc_a[pi][c] = __ffma2_rn(wa[i], xv[c][i], acc_a[pi][c]);
-                acc_b[pi][c] = __ffma2_rn(wb[i], xv[c][i], acc_b[pi][c]);
+          for (int pi = 0; pi < 2; ++pi) {
+            const int ra = m.down ? 4 * warp + 2 * pi : 2 * warp + pi;
+            const int rb = m.down ? ra + 1 : kRows / 2 + ra;
+            float2 wa[E16 / 2], wb[E16 / 2];
+            w_chunk<WK>(st + ra * RB + ch * 512 + lane * 16, wa);
+            w_chunk<WK>(st + rb * RB + ch * 512 + lane * 16, wb);
+#pragma unroll
+            for (int c = 0; c < NT; ++c) {
+              if (c < m.nt) {
+#pragma unroll
+                for (int i = 0; i < E16 / 2; ++i) {
+                  acc_a[pi][c] = __ffma2_rn(wa[i], xv[c][i], acc_a[pi][c]);
+                  acc_b[pi][c] = __ffma2_rn(wb[i], xv[c][i], acc_b[pi][c]);
+                }
               }
             }
           }
         }
       }
     }
-    if (kc == m.nkc - 1) {  // ---- the item ends: add the lanes' sums and store, pair by pair
+    if (kc == m.nkc - 1) {  // ---- the item ends: add the lanes' sums and store
       const int first = it.first[m.g];
-#pragma unroll
-      for (int pi = 0; pi < 2; ++pi) {
-        float v[NV];
-#pragma unroll
-        for (int c = 0; c < NT; ++c) {
-          v[c] = acc_a[pi][c].x + acc_a[pi][c].y;
-          v[NT + c] = acc_b[pi][c].x + acc_b[pi][c].y;
-        }
-        const float tot = warp_reduce_many<NV>(v);
-        constexpr int per = 32 / NV;  // lanes holding each total; value i sits in lanes [i*per, i*per + per)
-        const int vi = lane / per;
-        const int c = vi % NT;
-        const int t = m.t0 + min(c, m.nt - 1);
-        const int pr = m.e < 0 ? t : pairs[first + t];
+      if (NT == 1 || m.nt == 1) {
+        // one token: the four rows' sums in one butterfly; rows a0, b0, a1, b1 land in lanes 0, 8, 16, 24
+        float v[4] = {acc_a[0][0].x + acc_a[0][0].y, acc_b[0][0].x + acc_b[0][0].y, acc_a[1][0].x + acc_a[1][0].y,
+                      acc_b[1][0].x + acc_b[1][0].y};
+        const float tot = warp_reduce_many<4>(v);
+        const int t = m.t0;
         if (!m.down) {
-          // row a (gate) totals are values [0, NT), row b (up) [NT, 2 NT): 16 lanes higher
-          const float u = __shfl_down_sync(0xffffffffu, tot, 16);
-          if (lane < 16 && lane % per == 0 && c < m.nt) {
+          const float u = __shfl_down_sync(0xffffffffu, tot, 8);  // the up row's sum beside its gate row's
+          if ((lane & 15) == 0) {
             const float hv = act_fn(p.act, tot) * u;
-            const int f = m.r0 + 2 * warp + pi;
+            const int f = m.r0 + 2 * warp + (lane >> 4);
             if (m.e < 0)
               p.h_s[static_cast<size_t>(t) * p.Is + f] = hv;
             else
               p.h[static_cast<size_t>(first + t) * p.I + f] = hv;
           }
-        } else if (lane % per == 0 && c < m.nt) {
-          const int n = m.r0 + 4 * warp + 2 * pi + vi / NT;  // rows 4w + 2pi, 4w + 2pi + 1 of the block
-          if (m.e < 0)
+        } else if ((lane & 7) == 0) {
+          const int n = m.r0 + 4 * warp + (lane >> 3);
+          if (m.e < 0) {
             p.y_s[static_cast<size_t>(t) * p.H + n] = (sgate ? sgate[t] : 1.f) * tot;
-          else
+          } else {
+            const int pr = pairs[first + t];
             p.y_slots[static_cast<size_t>(pr) * p.H + n] = wpair[pr] * tot;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int pi = 0; pi < 2; ++pi) {
+          float v[NV];
+#pragma unroll
+          for (int c = 0; c < NT; ++c) {
+            v[c] = acc_a[pi][c].x + acc_a[pi][c].y;
+            v[NT + c] = acc_b[pi][c].x + acc_b[pi][c].y;
+          }
+          const float tot = warp_reduce_many<NV>(v);
+          constexpr int per = 32 / NV;  // lanes holding each total; value i sits in lanes [i*per, i*per + per)
+          const int vi = lane / per;
+          const int c = vi % NT;
+          const int t = m.t0 + min(c, m.nt - 1);
+          const int pr = m.e < 0 ? t : pairs[first + t];
+          if (!m.down) {
+            // row a (gate) totals are values [0, NT), row b (up) [NT, 2 NT): 16 lanes higher
+            const float u = __shfl_down_sync(0xffffffffu, tot, 16);
+            if (lane < 16 && lane % per == 0 && c < m.nt) {
+              const float hv = act_fn(p.act, tot) * u;
+              const int f = m.r0 + 2 * warp + pi;
+              if (m.e < 0)
+                p.h_s[static_cast<size_t>(t) * p.Is + f] = hv;
+              else
+                p.h[static_cast<size_t>(first + t) * p.I + f] = hv;
+            }
+          } else if (lane % per == 0 && c < m.nt) {
+            const int n = m.r0 + 4 * warp + 2 * pi + vi / NT;  // rows 4w + 2pi, 4w + 2pi + 1 of the block
+            if (m.e < 0)
+              p.y_s[static_cast<size_t>(t) * p.H + n] = (sgate ? sgate[t] : 1.f) * tot;
+            else
+              p.y_slots[static_cast<size_t>(pr) * p.H + n] = wpair[pr] * tot;
+          }
         }
       }
       if (!m.down) {
-        // the item's consumer warps count themselves in shared memory; the last one makes all their h
-        // stores visible GPU-wide (the fence is cumulative over what it observed) and counts the item for
-        // its group
+        // the item's consumer warps count themselves in shared memory; the last one (which has observed
+        // the others' h stores through the count) queues the item for the issuing thread to count
         __syncwarp();
         if (lane == 0) {
           __threadfence_block();
           if (atomicAdd_block(&ring.done_warps[s], 1) == kCW - 1) {
             ring.done_warps[s] = 0;  // ready for the next item ending in this stage (after the refill)
-            __threadfence();
-            atomicAdd(&p.sync->done[m.g], 1u);
+            const int slot = atomicAdd_block(&ring.dq_tail, 1);
+            __threadfence_block();
+            *reinterpret_cast<volatile int*>(&ring.dq[slot % kDoneQ]) = m.g + 1;
           }
         }
       }

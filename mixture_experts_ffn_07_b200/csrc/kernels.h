@@ -150,7 +150,7 @@ struct DecodeLayer {
 };
 size_t decode_router_parts_floats(int T, int H, int E, bool shared_gate);
 constexpr size_t decode_stream_sync_bytes() { return 4 * (1 + 257); }
-int stream_path_mode();  // moe_set_decode_stream: 0 two phases, 1 the stream (f32 / bf16 weights)
+int stream_path_mode();  // moe_set_decode_stream: 0 two phases, 1 the stream (f32 / bf16 / Q8_0 weights)
 cudaError_t launch_decode_layer(const Ctx& c, const DecodeLayer& L);
 
 

@@ -1,8 +1,9 @@
-"""The fused decode kernel's gate/up + down stream (a ring of 32 KB stages per CTA fed by the copy engine, work
-items from a device-wide queue, down items waiting on their expert's gate/up counter) against the two-phase form
-of the same kernel and against the oracle, for f32 and bf16 weights (f32 or bf16 activations): one token,
-several tokens per expert (token chunks), the shared expert (gated), rows longer than one stage, the most
-pairs (E = 256, K = 32), and all pairs on two experts."""
+"""The fused decode kernel's gate/up + down stream (a ring of stages per CTA fed by the copy engine from one
+issuing warp, work items from a device-wide queue, down items waiting on their expert's gate/up counter)
+against the two-phase form of the same kernel and against the oracle, for f32, bf16 and Q8_0 weights (f32 or
+bf16 activations): one token, several tokens per expert (token chunks), the shared expert (gated and not),
+rows longer than one stage, Q8_0 rows of 1024-code stages with a partial last stage, the most pairs (E = 256,
+K = 32), and all pairs on two experts."""
 import numpy as np
 import pytest
 
@@ -24,6 +25,13 @@ CASES = {
     "f32x_bf16w_T3": (spec(3, 384, 8, 64, 2, dt="f32", w_dt="bf16", r_dt="f32"), {}),
     "max_pairs_E256_K32": (spec(64, 128, 256, 32, 32, dt="f32"), {}),
     "skew_all_to_two": (spec(48, 256, 8, 64, 2, dt="f32"), dict(skew=True)),
+    "q8_T1": (spec(1, 1024, 16, 512, 4, dt="f32", w_dt="q8_0", r_dt="f32"), {}),
+    "q8_T16": (spec(16, 512, 32, 256, 8, dt="f32", w_dt="q8_0", r_dt="f32"), {}),
+    "q8_T16_long_rows_shared": (spec(16, 2048, 32, 768, 8, dt="f32", w_dt="q8_0", r_dt="f32", shared=256,
+                                     gated=True), {}),
+    "q8_T5_ungated_shared_bf16_router": (spec(5, 512, 16, 256, 2, dt="f32", w_dt="q8_0", r_dt="bf16",
+                                              shared=256), {}),
+    "q8_skew_chunks": (spec(40, 512, 8, 256, 2, dt="f32", w_dt="q8_0", r_dt="f32"), dict(skew=True)),
 }
 
 
@@ -78,7 +86,8 @@ def test_stream_matches_two_phases_and_oracle(case):
     print(f"\n{case}: max|stream-oracle| {err_a:.3e}, max|two phases-oracle| {err_b:.3e}, {flagged} flagged")
 
 
-@pytest.mark.parametrize("case", ["f32_T64_shared_gated_bias", "f32_T1_long_rows", "f32_skew_chunks"])
+@pytest.mark.parametrize("case", ["f32_T64_shared_gated_bias", "f32_T1_long_rows", "f32_skew_chunks",
+                                  "q8_T16_long_rows_shared", "q8_skew_chunks"])
 def test_stream_is_deterministic(case):
     """Whichever warp takes an item, its arithmetic is fixed: the same bits on every call."""
     s, opt = CASES[case]
