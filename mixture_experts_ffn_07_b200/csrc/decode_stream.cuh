@@ -581,53 +581,65 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
     const uint32_t st = smem_addr(stages + s * Fmt<WK>::SB);
     const uint32_t act = st + Fmt<WK>::ACT;
     if constexpr (WK == WK_Q8) {
-      // a lane's 16 codes of a row are half a block: partial = sum q * x over them, then acc += d * partial.
-      // Token by token, the four rows' chains side by side (the codes are widened again per token: most
-      // items have one or two tokens).
+      // In each 512-code half of a row, lane l takes the 4-code groups at 4l + 128q (q = 0..3): the loads of
+      // the codes (32-bit words) and of the activations (4 values) of a group are then adjacent across the
+      // lanes, free of shared-memory bank conflicts (16 contiguous codes per lane would put the lanes' f32
+      // activations 64 bytes apart, four to a bank).  Each group lies in one block: partial = sum q * x over
+      // it, then acc += d * partial.  Token by token, the four rows' chains side by side (the codes are
+      // widened again per token: most items have one or two tokens).
       const int r0 = m.down ? 4 * warp : 2 * warp, r1 = m.down ? r0 + 1 : kRows / 2 + r0;
       const int r2 = m.down ? r0 + 2 : r0 + 1, r3 = m.down ? r0 + 3 : kRows / 2 + r0 + 1;
       const int rows[4] = {r0, r1, r2, r3};
-      float d[NCH][4];
+      constexpr int AB = 4 * sizeof(XT);  // activation bytes of a group (gate/up); down reads f32 h
 #pragma unroll
-      for (int ch = 0; ch < NCH; ++ch)
+      for (int ch = 0; ch < NCH; ++ch) {
+        if (kc * KC + ch * 512 >= m.kdim) break;  // past the row: nothing to add (rows are whole 256-code units)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint16_t hv;
-          asm volatile("ld.shared.u16 %0, [%1];"
-                       : "=h"(hv)
-                       : "r"(st + Fmt<WK>::SCL + rows[j] * Fmt<WK>::SR + ((ch * 512 + lane * 16) / 32) * 2));
-          d[ch][j] = __half2float(__ushort_as_half(hv));
-        }
+        for (int c = 0; c < NT; ++c) {
+          if (c >= m.nt) break;
+          float sj[4] = {0.f, 0.f, 0.f, 0.f};  // the four rows' sums over this half
 #pragma unroll
-      for (int c = 0; c < NT; ++c) {
-        if (c >= m.nt) break;
+          for (int qh = 0; qh < 2; ++qh) {  // two groups' activations at a time
+            float2 xv[2][2];
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) {
-          const int kl = ch * 512 + lane * 16;  // code within the stage
-          if (kc * KC + kl < m.kdim) {
-            float2 xv[8];
-            if (m.down)
-              act_smem<float, 16>(act + c * Fmt<WK>::AR + kl * 4, xv);
-            else
-              act_smem<XT, 16>(act + c * Fmt<WK>::AR + kl * static_cast<int>(sizeof(XT)), xv);
-            float2 pr[4];
+            for (int qq = 0; qq < 2; ++qq) {
+              const int e = ch * 512 + 4 * lane + 128 * (2 * qh + qq);  // the group's first code
+              if (m.down || sizeof(XT) == 4) {
+                const uint4 v = stream::lds16(act + c * Fmt<WK>::AR + e * 4);
+                xv[qq][0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+                xv[qq][1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+              } else {
+                uint32_t v0, v1;
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                             : "=r"(v0), "=r"(v1)
+                             : "r"(act + c * Fmt<WK>::AR + e * AB / 4));
+                xv[qq][0] = stream::bf16x2_f2(v0);
+                xv[qq][1] = stream::bf16x2_f2(v1);
+              }
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              float2 w[8];
-              w_chunk<WK>(st + rows[j] * RB + kl, w);
-              float2 e = __fmul2_rn(w[0], xv[0]), o = __fmul2_rn(w[1], xv[1]);
 #pragma unroll
-              for (int i = 2; i < 8; i += 2) {
-                e = __ffma2_rn(w[i], xv[i], e);
-                o = __ffma2_rn(w[i + 1], xv[i + 1], o);
+              for (int qq = 0; qq < 2; ++qq) {
+                const int q = 2 * qh + qq;
+                uint16_t hv;  // the group's block scale
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(hv)
+                             : "r"(st + Fmt<WK>::SCL + rows[j] * Fmt<WK>::SR + (ch * 16 + (lane >> 3) + 4 * q) * 2));
+                uint32_t wv;
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(wv) : "r"(st + rows[j] * RB + ch * 512 + 4 * lane + 128 * q));
+                float2 lo, hi;
+                stream::q8_quad(wv, lo, hi);
+                const float2 pq = __ffma2_rn(hi, xv[qq][1], __fmul2_rn(lo, xv[qq][0]));
+                sj[j] = fmaf(__half2float(__ushort_as_half(hv)), pq.x + pq.y, sj[j]);
               }
-              pr[j] = __fadd2_rn(e, o);
             }
-            acc_a[0][c] = __ffma2_rn(make_float2(d[ch][0], d[ch][0]), pr[0], acc_a[0][c]);
-            acc_b[0][c] = __ffma2_rn(make_float2(d[ch][1], d[ch][1]), pr[1], acc_b[0][c]);
-            acc_a[1][c] = __ffma2_rn(make_float2(d[ch][2], d[ch][2]), pr[2], acc_a[1][c]);
-            acc_b[1][c] = __ffma2_rn(make_float2(d[ch][3], d[ch][3]), pr[3], acc_b[1][c]);
           }
+          // Q8_0 sums in the .x halves of the accumulators (the .y halves stay zero)
+          acc_a[0][c].x += sj[0];
+          acc_b[0][c].x += sj[1];
+          acc_a[1][c].x += sj[2];
+          acc_b[1][c].x += sj[3];
         }
       }
     } else {
