@@ -217,6 +217,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (blockIdx.x == 0 && a.tma)  // the stream's queue and counters start at zero (visible after the barrier)
     for (int i = threadIdx.x; i < 1 + dstream::kMaxGroups; i += blockDim.x) reinterpret_cast<unsigned*>(a.sync)[i] = 0;
 
+  // the stream's tensor maps into the copy engine's descriptor cache while R and S run, by the warp that
+  // will issue the copies (only the maps this layer uses)
+  if constexpr (stream_format<WKG, WKD>()) {
+    using namespace dstream;
+    if (a.tma && warp == kCW && lane < M_COUNT) {
+      const bool sh = lane == M_SGATE || lane == M_SUP || lane == M_SDOWN || lane == M_HS;
+      if (!sh || a.has_shared) {
+        prefetch_tensormap(&maps.w[lane]);
+        if (WKG == WK_Q8 && lane <= M_SDOWN) prefetch_tensormap(&maps.s[lane]);
+      }
+    }
+  }
+
   // the routing bias, copied to shared memory while R runs (it is read in S)
   if (a.bias)
     for (int e = threadIdx.x; e < E; e += blockDim.x) cp_async4(&s_bias[e], a.bias + e);

@@ -96,6 +96,13 @@ __device__ __forceinline__ void warp_select(const float (&v)[8], float m, const 
     }
   }
 
+  // K rounds: each lane's best eligible logit (lower expert on ties), then over the warp the largest value
+  // (as an order-preserving 32-bit key, one redux) and the lowest expert holding it (a second redux).
+  // The same selection as a pairwise (value, lower index) maximum; -0 counts as +0, as in a float compare.
+  auto key = [](float f) {
+    const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  };
   int my_e = 0;
   float my_v = 0.f;
   for (int k = 0; k < K; ++k) {
@@ -109,15 +116,10 @@ __device__ __forceinline__ void warp_select(const float (&v)[8], float m, const 
         be = e;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
+    const uint32_t kb = key(bv);
+    const uint32_t km = __reduce_max_sync(0xffffffffu, kb);
+    be = static_cast<int>(__reduce_min_sync(0xffffffffu, kb == km ? static_cast<uint32_t>(be) : 0xFFFFFFFFu));
+    bv = __uint_as_float((km & 0x80000000u) ? (km & 0x7FFFFFFFu) : ~km);
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
     if (lane == k) {
       my_e = be;
