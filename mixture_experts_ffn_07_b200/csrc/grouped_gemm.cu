@@ -35,6 +35,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstring>
 
 #include "kernels.h"
 
@@ -887,6 +888,15 @@ int pair_clusters(const Ctx& c) {
   return n;
 }
 
+// The trace name of a CTA-pair launch's tail launch ("<name>_tail").
+inline const char* tail_name(const char* name) {
+  if (!std::strcmp(name, "expert_gate_up_gemm")) return "expert_gate_up_gemm_tail";
+  if (!std::strcmp(name, "expert_down_gemm")) return "expert_down_gemm_tail";
+  if (!std::strcmp(name, "shared_gate_up_gemm")) return "shared_gate_up_gemm_tail";
+  if (!std::strcmp(name, "shared_down_gemm")) return "shared_down_gemm_tail";
+  return "grouped_gemm_tail";
+}
+
 // The full 256-row tiles of every group on CTA pairs (M = 256, N = 256 per
 // MMA), then the rows left in each group on the single-CTA kernel.
 template <bool DUAL>
@@ -911,7 +921,7 @@ cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, int clusters) {
     if (e != cudaSuccess) return e;
   }
   GemmArgs tail = a;
-  if (a.name) tail.name = DUAL ? "expert_gate_up_gemm_tail" : "expert_down_gemm_tail";
+  if (a.name) tail.name = tail_name(a.name);
   return launch_tiled<DUAL, 256, 1>(c, tail, PAIR_M);
 }
 
