@@ -600,6 +600,9 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
           float sj[4] = {0.f, 0.f, 0.f, 0.f};  // the four rows' sums over this half
 #pragma unroll
           for (int qh = 0; qh < 2; ++qh) {  // two groups' activations at a time
+            // groups q = 2 qh, 2 qh + 1 lie in the stage's 256-code unit 2 ch + qh: past the row, nothing to add
+            // (their codes are zero fill, but the activations there belong to other rows and may be anything)
+            if (kc * KC + ch * 512 + qh * 256 >= m.kdim) break;
             float2 xv[2][2];
 #pragma unroll
             for (int qq = 0; qq < 2; ++qq) {

@@ -196,17 +196,22 @@ __global__ void __launch_bounds__(kThreads, 1) front_kernel(const FrontArgs a) {
   const int n16 = a.H / 8;  // 16-byte groups of a bf16 row
   const uint4* src = reinterpret_cast<const uint4*>(a.x);
   uint4* dst = reinterpret_cast<uint4*>(a.x_perm);
-  for (int p = p0 + warp; p < p1; p += kWarps) {
-    const uint4* s = src + static_cast<size_t>(p / K) * n16;
-    uint4* d = dst + static_cast<size_t>(pos_in_smem ? s_pos[p - p0] : a.pair_pos[p]) * n16;
+  // a warp per token: each 4 KB of its row is loaded once and stored at the places of all the token's pairs
+  // in this CTA's range (a token's K pairs are consecutive in pair order)
+  for (int t = p0 / K + warp; t * K < p1; t += kWarps) {
+    const int q0 = max(p0, t * K), q1 = min(p1, t * K + K);
+    const uint4* s = src + static_cast<size_t>(t) * n16;
     for (int o = lane; o < n16; o += 32 * 8) {  // a 4 KB row (H = 2048) in one round of loads
       uint4 v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         if (o + 32 * j < n16) v[j] = __ldg(s + o + 32 * j);
+      for (int q = q0; q < q1; ++q) {
+        uint4* d = dst + static_cast<size_t>(pos_in_smem ? s_pos[q - p0] : a.pair_pos[q]) * n16;
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (o + 32 * j < n16) d[o + 32 * j] = v[j];
+        for (int j = 0; j < 8; ++j)
+          if (o + 32 * j < n16) d[o + 32 * j] = v[j];
+      }
     }
   }
 }

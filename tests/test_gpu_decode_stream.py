@@ -48,7 +48,8 @@ def _run(desc, w, x, stream: bool):
     moe.set_decode_stream(stream)
     try:
         out = torch.full((desc.T, desc.H), float("nan"), dtype=x.dtype, device="cuda")
-        ws = torch.empty(max(moe.workspace_bytes(desc), 256), dtype=torch.uint8, device="cuda")
+        # every workspace byte 0xFF (NaN as f32): a read of a row before it is written shows in the output
+        ws = torch.full((max(moe.workspace_bytes(desc), 256),), 0xFF, dtype=torch.uint8, device="cuda")
         n0 = moe.launch_count()
         moe.layer(desc, x, w, out, ws)
         torch.cuda.synchronize()

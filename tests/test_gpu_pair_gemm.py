@@ -30,6 +30,8 @@ CASES = {
     "exact_tiles": (spec(512, 256, 2, 256, 2), None),
     # I = 160 (dual tiles of 128 features: a ragged last column tile), H = 352 (ragged 256-column tile)
     "ragged_columns": (spec(900, 352, 4, 160, 2, act="gelu_tanh"), None),
+    # two large experts (pair tiles and a remainder each) beside six small ones (single-CTA kernel only)
+    "mixed_sizes": (spec(900, 256, 8, 128, 2), [4.0, 3.0] + [0.0] * 6),
     # shared expert: one group of T = 600 rows (two pair tiles + 88 rows); routed groups of ~300 rows
     "shared_expert": (spec(600, 256, 8, 64, 4, shared=256, gated=True), None),
 }
