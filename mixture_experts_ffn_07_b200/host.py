@@ -75,8 +75,10 @@ def upload(src):
 
 
 def run_layer(desc, w, x):
-    out = torch.empty((desc.T, desc.H), dtype=x.dtype, device="cuda")
-    ws = torch.empty(max(workspace_bytes(desc), 256), dtype=torch.uint8, device="cuda")
+    """One moe_layer call on fresh buffers; the output starts as NaN and every workspace byte as 0xFF (NaN as
+    f32), so a row read before it is written, or an output never written, shows in the result."""
+    out = torch.full((desc.T, desc.H), float("nan"), dtype=x.dtype, device="cuda")
+    ws = torch.full((max(workspace_bytes(desc), 256),), 0xFF, dtype=torch.uint8, device="cuda")
     layer(desc, x, w, out, ws)
     torch.cuda.synchronize()
     st = last_device_status()

@@ -134,7 +134,7 @@ def test_fused_back_to_back_calls_share_the_barrier():
     desc, w, x = _gpu.upload(wl)
     ref, _, _ = _run(desc, w, x, True)
     out = torch.empty_like(ref)
-    ws = torch.empty(max(moe.workspace_bytes(desc), 256), dtype=torch.uint8, device="cuda")
+    ws = torch.full((max(moe.workspace_bytes(desc), 256),), 0xFF, dtype=torch.uint8, device="cuda")
     for _ in range(50):
         moe.layer(desc, x, w, out, ws)
     torch.cuda.synchronize()

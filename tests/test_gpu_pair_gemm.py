@@ -94,7 +94,7 @@ def test_pair_expert_ffn_f32_slots():
     moe.permute(desc, d_ids, counts, offsets, sp, pp)
     assert int(counts.min()) >= 256  # every expert has a full pair tile
     y = torch.full((P, s.H), float("nan"), dtype=torch.float32, device="cuda")
-    ws = torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    ws = torch.full((moe.workspace_bytes(desc),), 0xFF, dtype=torch.uint8, device="cuda")
     moe.expert_ffn(desc, x, w, offsets, sp, tw, y, ws)
     torch.cuda.synchronize()
     assert moe.last_device_status() == moe.MOE_OK

@@ -160,7 +160,7 @@ def test_expert_ffn(case, path_for):
     pp = torch.empty(P, dtype=torch.int32, device="cuda")
     moe.permute(desc, d_ids, counts, offsets, sp, pp)
     y = torch.full((P, s.H), float("nan"), dtype=torch.float32, device="cuda")
-    ws = torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    ws = torch.full((moe.workspace_bytes(desc),), 0xFF, dtype=torch.uint8, device="cuda")
     moe.expert_ffn(desc, x, w, offsets, sp, tw, y, ws)
     torch.cuda.synchronize()
     assert moe.last_device_status() == moe.MOE_OK
@@ -220,7 +220,7 @@ def test_empty_batch():
     _, w, _ = _gpu.upload(wl)
     x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
     out = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(max(moe.workspace_bytes(desc), 256), dtype=torch.uint8, device="cuda")
+    ws = torch.full((max(moe.workspace_bytes(desc), 256),), 0xFF, dtype=torch.uint8, device="cuda")
     n0 = moe.launch_count()
     moe.layer(desc, x, w, out, ws)
     assert moe.launch_count() == n0
@@ -247,7 +247,7 @@ def test_layer_host_matches_device_call():
     oh = torch.empty_like(xh).pin_memory()
     xd = torch.empty_like(x)
     od = torch.empty_like(x)
-    ws = torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    ws = torch.full((moe.workspace_bytes(desc),), 0xFF, dtype=torch.uint8, device="cuda")
     moe.layer_host(desc, xh, w, oh, xd, od, ws)
     torch.cuda.synchronize()
     assert torch.equal(oh.view(torch.int16), ref.cpu().view(torch.int16))
@@ -275,7 +275,7 @@ def test_two_streams_alternating_host_calls(case):
     ref = _gpu.run_layer(desc, w, x)
     xh = x.cpu().pin_memory()
     sets = [dict(oh=torch.empty_like(xh).pin_memory(), xd=torch.empty_like(x), od=torch.empty_like(x),
-                 ws=torch.empty(moe.workspace_bytes(desc), dtype=torch.uint8, device="cuda"),
+                 ws=torch.full((moe.workspace_bytes(desc),), 0xFF, dtype=torch.uint8, device="cuda"),
                  stream=torch.cuda.Stream()) for _ in range(2)]
     outs = []
     for i in range(8):
