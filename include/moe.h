@@ -412,8 +412,8 @@ void moe_set_tma_gather(int enable);
 
 /* The fewest tokens for which a bf16 layer (bf16 activations and expert
  * weights) takes the tensor-core path (router GEMM, grouped tcgen05 GEMMs)
- * instead of the weight-streaming path; default 8 (the streaming path for 1..7
- * tokens), where the two paths cross on B200 (between 2 and 8 tokens on the
+ * instead of the weight-streaming path; default 16 (the streaming path for 1..15
+ * tokens), where the two paths cross on B200 (between 8 and 16 tokens on the
  * measured shapes).  Values below 1 count as 1.  moe_workspace_bytes follows
  * the current setting, so size workspaces after changing it.  Process-wide. */
 void moe_set_tensor_min_tokens(int tokens);

@@ -241,7 +241,7 @@ def set_tma_gather(enable: bool) -> None:
 
 def set_tensor_min_tokens(tokens: int) -> None:
     """moe_set_tensor_min_tokens: bf16 layers of at least `tokens` tokens take the tensor-core path
-    (default 8); size workspaces after changing it."""
+    (default 16); size workspaces after changing it."""
     _lib.lib().moe_set_tensor_min_tokens(int(tokens))
 
 

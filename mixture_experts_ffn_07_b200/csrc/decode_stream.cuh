@@ -72,17 +72,22 @@ constexpr int kStageWBytes = kRows * kRowBytes;  // 32 KB of weight rows
 // Tokens per item of a kernel instance built for at most maxt tokens (host and device).
 __host__ __device__ constexpr int item_tokens(int maxt) { return maxt == 1 ? 1 : kMaxNT; }
 
-// Geometry of a stage by weight format.  KC: row elements per stage (256 f32 / bf16 values -- a box is at
-// most 256 wide --, 1024 Q8_0 codes as 256 words); RB: bytes of a row in a stage (bf16 rows fill half of
-// kRowBytes); NCH: 16-byte chunks per lane and row; E16: elements per chunk;
+// Geometry of a stage by weight format.  KC: row elements per stage (256 f32, 512 bf16 values in two
+// 256-wide boxes, 1024 Q8_0 codes as 256 words); RB: bytes of a row in a stage (kRowBytes for all three);
+// NCH: 16-byte chunks per lane and row; E16: elements per chunk;
 // AR: bytes of one activation row of the stage (KC values, room for f32); SR: bytes of the fp16 scales of
 // one row (Q8_0: 32 blocks).  A stage is [kRows weight rows][kMaxNT activation rows][kRows scale rows].
 template <int WK>
 struct Fmt {
   static_assert(WK == WK_F32 || WK == WK_BF16 || WK == WK_Q8, "the stream serves f32, bf16 and Q8_0 weights");
   static constexpr int EB = WK == WK_F32 ? 4 : (WK == WK_BF16 ? 2 : 1);
-  static constexpr int KC = WK == WK_Q8 ? 1024 : 256;
+  static constexpr int KC = WK == WK_Q8 ? 1024 : (WK == WK_BF16 ? 512 : 256);
   static constexpr int RB = KC * EB;
+  // bf16: a stage holds two 256-column chunks, each as its own plane of kRows rows of 512 bytes (a box is
+  // at most 256 wide), and the activation rows likewise as two planes of kMaxNT rows of 1 KB
+  static constexpr bool SPLIT = WK == WK_BF16;
+  static constexpr int PLANE = kRows * 512;
+  static constexpr int APLANE = kMaxNT * 1024;
   static constexpr int NCH = RB / 512;
   static constexpr int E16 = 16 / EB;
   static constexpr int AR = KC * 4;
@@ -252,6 +257,31 @@ __device__ __forceinline__ void issue_stage(const Maps& maps, const Params& p, c
   uint8_t* act = st + F::ACT;
   uint8_t* sc = st + F::SCL;
   const int ax = Q8 ? 0 : kx;  // activation copies: Q8_0 reads 4 rows of the 256-value view
+  if constexpr (F::SPLIT) {
+    if (!m.down) {
+      mbar_arrive_expect_tx(bar, kRows * F::RB + m.nt * 2 * 256 * static_cast<int>(sizeof(XT)));
+      const int mg = m.e < 0 ? M_SGATE : M_GATE, mu = m.e < 0 ? M_SUP : M_UP;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int kxc = kx + ch * 256;
+        tma_load_2d_hint(st + ch * F::PLANE, &maps.w[mg], bar, kxc, wrow, pol);
+        tma_load_2d_hint(st + ch * F::PLANE + (kRows / 2) * 512, &maps.w[mu], bar, kxc, wrow, pol);
+#pragma unroll
+        for (int c = 0; c < NT; ++c)
+          if (c < m.nt) tma_load_2d_hint(act + ch * F::APLANE + c * 1024, &maps.w[M_X], bar, kxc, xrow[c], apol);
+      }
+    } else {
+      const int hb = m.e < 0 ? maps.hs_box : maps.h_box;
+      mbar_arrive_expect_tx(bar, kRows * F::RB + 2 * hb * 256 * 4);
+      const int md = m.e < 0 ? M_SDOWN : M_DOWN, mh = m.e < 0 ? M_HS : M_H;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        tma_load_2d_hint(st + ch * F::PLANE, &maps.w[md], bar, kx + ch * 256, wrow, pol);
+        tma_load_2d_hint(act + ch * F::APLANE, &maps.w[mh], bar, kx + ch * 256, xrow[0], apol);
+      }
+    }
+    return;
+  }
   if (!m.down) {
     const int xb = F::KC * static_cast<int>(sizeof(XT));
     mbar_arrive_expect_tx(bar, kRows * F::RB + kRows * F::SR + m.nt * xb);
@@ -651,13 +681,17 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
         const int kl = (ch * 512 + lane * 16) / EB;  // element within the stage
         if (kc * KC + kl < m.kdim) {  // past the row (the last stage's tail): nothing to add
           float2 xv[NT][E16 / 2];
+          // bf16: chunk ch is its own plane (element kl = 256 ch + 8 lane)
+          const uint32_t arow = Fmt<WK>::SPLIT ? act + ch * Fmt<WK>::APLANE : act;
+          const int apitch = Fmt<WK>::SPLIT ? 1024 : Fmt<WK>::AR;
+          const int ael = Fmt<WK>::SPLIT ? lane * 8 : kl;
 #pragma unroll
           for (int c = 0; c < NT; ++c) {
             if (c < m.nt) {
               if (m.down)
-                act_smem<float, E16>(act + c * Fmt<WK>::AR + kl * 4, xv[c]);
+                act_smem<float, E16>(arow + c * apitch + ael * 4, xv[c]);
               else
-                act_smem<XT, E16>(act + c * Fmt<WK>::AR + kl * static_cast<int>(sizeof(XT)), xv[c]);
+                act_smem<XT, E16>(arow + c * apitch + ael * static_cast<int>(sizeof(XT)), xv[c]);
             }
           }
 #pragma unroll
@@ -665,8 +699,13 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
             const int ra = m.down ? 4 * warp + 2 * pi : 2 * warp + pi;
             const int rb = m.down ? ra + 1 : kRows / 2 + ra;
             float2 wa[E16 / 2], wb[E16 / 2];
-            w_chunk<WK>(st + ra * RB + ch * 512 + lane * 16, wa);
-            w_chunk<WK>(st + rb * RB + ch * 512 + lane * 16, wb);
+            if constexpr (Fmt<WK>::SPLIT) {
+              w_chunk<WK>(st + ch * Fmt<WK>::PLANE + ra * 512 + lane * 16, wa);
+              w_chunk<WK>(st + ch * Fmt<WK>::PLANE + rb * 512 + lane * 16, wb);
+            } else {
+              w_chunk<WK>(st + ra * RB + ch * 512 + lane * 16, wa);
+              w_chunk<WK>(st + rb * RB + ch * 512 + lane * 16, wb);
+            }
 #pragma unroll
             for (int c = 0; c < NT; ++c) {
               if (c < m.nt) {

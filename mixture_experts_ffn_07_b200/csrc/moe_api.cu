@@ -2,7 +2,7 @@
 // workspace layout, the order of kernel launches for each entry point, the
 // device status word, and the host-side launch counter and event trace.
 //
-// Path choice: bf16 activations with bf16 expert weights and T >= 8 (moe_set_tensor_min_tokens) take the
+// Path choice: bf16 activations with bf16 expert weights and T >= 16 (moe_set_tensor_min_tokens) take the
 // tensor-core path (row gather + tcgen05 grouped GEMMs); everything else takes
 // the weight-streaming path (expert-major GEMV kernels), which reads each
 // touched expert's weights once and is the bandwidth-optimal form for small T.
@@ -85,9 +85,9 @@ inline size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255);
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Fewest tokens for which a bf16 layer takes the tensor-core path (moe_set_tensor_min_tokens).  Measured
-// on B200 (bench.py --op crossover): the tensor-core path is faster from 2-8 tokens on, depending on the
-// shape, so 8.
-std::atomic<int> g_tensor_min_tokens{8};
+// on B200 (bench.py --op crossover): the decode stream is faster up to 8 tokens on every measured shape,
+// the tensor-core path from 16 on two of the three, so 16.
+std::atomic<int> g_tensor_min_tokens{16};
 
 bool tensor_path(const moe_desc& d) {
   return d.act_dtype == MOE_BF16 && d.w_dtype == MOE_BF16 && d.T >= g_tensor_min_tokens.load();

@@ -15,16 +15,19 @@ F32_TOL = (1e-3, 1e-5)   # |gpu - oracle|_inf <= 1e-3 * max|oracle| + 1e-5   (f3
 from mixture_experts_ffn_07_b200.host import run_layer, run_route, split_q8_0 as q8_split, to_device as dev, upload  # noqa: E402,F401
 
 
+DEFAULT_TENSOR_MIN_TOKENS = 16  # moe_set_tensor_min_tokens' default
+
+
 class streaming_path:
     """Within the block, bf16 layers of up to 64 tokens take the weight-streaming path (the tensor-core path
-    starts at 65 tokens instead of the default 8), for tests of that path."""
+    starts at 65 tokens instead of the default 16), for tests of that path."""
 
     def __enter__(self):
         moe.set_tensor_min_tokens(65)
         return self
 
     def __exit__(self, *exc):
-        moe.set_tensor_min_tokens(8)
+        moe.set_tensor_min_tokens(DEFAULT_TENSOR_MIN_TOKENS)
         return False
 
 

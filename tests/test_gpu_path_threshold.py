@@ -1,4 +1,4 @@
-"""Both paths of a bf16 layer on either side of the default 65-token threshold (moe_set_tensor_min_tokens):
+"""Both paths of a bf16 layer on either side of a token threshold (moe_set_tensor_min_tokens):
 the tensor-core path on 16..64 tokens and the weight-streaming path on more than 64, each against the oracle,
 so the threshold can be set anywhere the measured crossover puts it."""
 import numpy as np
@@ -26,7 +26,7 @@ def test_layer_on_either_path(T, threshold):
         _gpu.run_layer(desc, w, x)
         launches = moe.launch_count() - n0
     finally:
-        moe.set_tensor_min_tokens(65)
+        moe.set_tensor_min_tokens(_gpu.DEFAULT_TENSOR_MIN_TOKENS)
     assert moe.last_device_status() == moe.MOE_OK
     L = oracle.from_workload(wl)
     exp, flagged = _gpu.expected_layer(L, ids.cpu().numpy(), gpu_logits=logits.cpu().numpy().astype(np.float64))
