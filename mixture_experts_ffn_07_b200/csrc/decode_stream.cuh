@@ -627,7 +627,7 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
 #pragma unroll
         for (int c = 0; c < NT; ++c) {
           if (c >= m.nt) break;
-          float sj[4] = {0.f, 0.f, 0.f, 0.f};  // the four rows' sums over this half
+          float2 sj[4] = {};  // the four rows' sums over this half, as pairs
 #pragma unroll
           for (int qh = 0; qh < 2; ++qh) {  // two groups' activations at a time
             // groups q = 2 qh, 2 qh + 1 lie in the stage's 256-code unit 2 ch + qh: past the row, nothing to add
@@ -664,15 +664,16 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
                 float2 lo, hi;
                 stream::q8_quad(wv, lo, hi);
                 const float2 pq = __ffma2_rn(hi, xv[qq][1], __fmul2_rn(lo, xv[qq][0]));
-                sj[j] = fmaf(__half2float(__ushort_as_half(hv)), pq.x + pq.y, sj[j]);
+                const float d = __half2float(__ushort_as_half(hv));
+                sj[j] = __ffma2_rn(make_float2(d, d), pq, sj[j]);
               }
             }
           }
           // Q8_0 sums in the .x halves of the accumulators (the .y halves stay zero)
-          acc_a[0][c].x += sj[0];
-          acc_b[0][c].x += sj[1];
-          acc_a[1][c].x += sj[2];
-          acc_b[1][c].x += sj[3];
+          acc_a[0][c].x += sj[0].x + sj[0].y;
+          acc_b[0][c].x += sj[1].x + sj[1].y;
+          acc_a[1][c].x += sj[2].x + sj[2].y;
+          acc_b[1][c].x += sj[3].x + sj[3].y;
         }
       }
     } else {
