@@ -234,18 +234,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (a.bias)
     for (int e = threadIdx.x; e < E; e += blockDim.x) cp_async4(&s_bias[e], a.bias + e);
 
-  // ---- R: partial router logits; a CTA item is (hidden chunk, token group, block of kWarps rows)
+  // ---- R: partial router logits; a CTA item is (hidden chunk, token group, block of kWarps rows).  Token
+  // groups are as small as spreads the items over the grid (a warp's work is one row for each token of its
+  // group, so fewer tokens per item is a shorter phase), at most kTokGroup tokens.
   {
     const int nch = (a.H + kRouterChunk - 1) / kRouterChunk;
-    const int ntg = (T + kTokGroup - 1) / kTokGroup;
     const int nrb = (R + kWarps - 1) / kWarps;
+    const int groups_fit = max(1, static_cast<int>(gridDim.x) / (nch * nrb));
+    const int tgs = min(kTokGroup, (T + groups_fit - 1) / groups_fit);
+    const int ntg = (T + tgs - 1) / tgs;
     const int items = nch * ntg * nrb;
     float* xs = reinterpret_cast<float*>(smem);
     int staged = -1;
     for (int i = blockIdx.x; i < items; i += gridDim.x) {
       const int rb = i % nrb, cg = i / nrb;  // consecutive items of a CTA share their x chunk when they can
       const int ch = cg % nch, tg = cg / nch;
-      const int t0 = tg * kTokGroup, nt = min(kTokGroup, T - t0);
+      const int t0 = tg * tgs, nt = min(tgs, T - t0);
       if (a.router_bf16)
         router_item<XT, __nv_bfloat16>(a, xs, rb, cg, ch, t0, nt, R, staged);
       else
