@@ -438,30 +438,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     ok = cta_grid_sync(a, &s_abort, &s_flag);
   }
 
-  // ---- C: combine
+  // ---- C: combine.  A warp takes 32 consecutive float4 of the output (the warps of the grid in turn, CTA
+  // first, so a small batch spreads over many SMs); each lane asks for its first kCombineK slot rows (and the
+  // shared expert's row) at once, then adds them in k order.
   if (ok) {
+    constexpr int kCombineK = 8;
     const int H4 = a.H / 4;
     const long long total = static_cast<long long>(T) * H4;
+    const long long nchunk = (total + 31) / 32;
     const float4* ys = reinterpret_cast<const float4*>(a.y_slots);
     const float4* sh = reinterpret_cast<const float4*>(a.y_s);
-    for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    for (long long u = blockIdx.x + static_cast<long long>(gridDim.x) * warp; u < nchunk;
+         u += static_cast<long long>(gridDim.x) * kWarps) {
+      const long long idx = u * 32 + lane;
+      if (idx >= total) continue;
       const long long t = idx / H4;
       const int c = static_cast<int>(idx - t * H4);
-      float4 acc = __ldcg(ys + (t * K) * H4 + c);
-      for (int k = 1; k < K; ++k) {
-        const float4 v = __ldcg(ys + (t * K + k) * H4 + c);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+      const float4* yt = ys + (t * K) * H4 + c;
+      float4 v[kCombineK];
+#pragma unroll
+      for (int k = 0; k < kCombineK; ++k)
+        if (k < K) v[k] = __ldcg(yt + k * H4);
+      const float4 vs = a.has_shared ? __ldcg(sh + t * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 acc = v[0];
+#pragma unroll
+      for (int k = 1; k < kCombineK; ++k)
+        if (k < K) {
+          acc.x += v[k].x;
+          acc.y += v[k].y;
+          acc.z += v[k].z;
+          acc.w += v[k].w;
+        }
+      for (int k = kCombineK; k < K; ++k) {
+        const float4 w = __ldcg(yt + k * H4);
+        acc.x += w.x;
+        acc.y += w.y;
+        acc.z += w.z;
+        acc.w += w.w;
       }
       if (a.has_shared) {
-        const float4 v = __ldcg(sh + t * H4 + c);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+        acc.x += vs.x;
+        acc.y += vs.y;
+        acc.z += vs.z;
+        acc.w += vs.w;
       }
       if constexpr (sizeof(XT) == 4) {
         reinterpret_cast<float4*>(a.out)[idx] = acc;
