@@ -59,7 +59,7 @@ __device__ __forceinline__ void warp_select(const float (&v)[8], float m, const 
                                             int32_t* __restrict__ ids, float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
   const int E = rc.E, K = rc.K;
-  uint32_t taken = 0;  // bit i: v[i] chosen, or not eligible
+  uint32_t taken = 0;  // bit i: v[i] not eligible (its group is not among the kept ones)
   if (rc.n_groups > 1) {
     const int gs = E / rc.n_groups;
     float my_gs = -INFINITY;  // lane g: score of group g
@@ -96,35 +96,62 @@ __device__ __forceinline__ void warp_select(const float (&v)[8], float m, const 
     }
   }
 
-  // K rounds: each lane's best eligible logit (lower expert on ties), then over the warp the largest value
-  // (as an order-preserving 32-bit key, one redux) and the lowest expert holding it (a second redux).
-  // The same selection as a pairwise (value, lower index) maximum; -0 counts as +0, as in a float compare.
+  // Candidates as order-preserving 32-bit keys (-0 counts as +0, as in a float compare; -inf is 0x007FFFFF)
+  // and an ineligible one (past E, or in an excluded group) as key 0, below every expert.  Each lane sorts
+  // its eight once (key descending, lower expert first: a strict order, the experts differ), so its best
+  // remaining candidate is always its first.  Then K rounds: the largest first key over the warp (one
+  // redux); when one lane holds it that lane wins, else the lowest expert among the holders (a second
+  // redux, only on equal values); the winner drops its first candidate.  The same selection as a pairwise
+  // (value, lower index) maximum.
   auto key = [](float f) {
     const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
   };
+  uint32_t ck[8];
+  int ce[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    ce[i] = lane + 32 * i;
+    ck[i] = (ce[i] < E && !((taken >> i) & 1u)) ? key(v[i]) : 0u;
+  }
+  auto cas = [&](int i, int j) {  // the better of candidates i and j to i
+    const bool sw = ck[j] > ck[i] || (ck[j] == ck[i] && ce[j] < ce[i]);
+    const uint32_t ki = ck[i], kj = ck[j];
+    const int ei = ce[i], ej = ce[j];
+    ck[i] = sw ? kj : ki;
+    ck[j] = sw ? ki : kj;
+    ce[i] = sw ? ej : ei;
+    ce[j] = sw ? ei : ej;
+  };
+  // Batcher's odd-even merge sort of 8: 19 compare-exchanges in 6 layers
+  cas(0, 2); cas(1, 3); cas(4, 6); cas(5, 7);
+  cas(0, 4); cas(1, 5); cas(2, 6); cas(3, 7);
+  cas(0, 1); cas(2, 3); cas(4, 5); cas(6, 7);
+  cas(2, 4); cas(3, 5);
+  cas(1, 4); cas(3, 6);
+  cas(1, 2); cas(3, 4); cas(5, 6);
   int my_e = 0;
   float my_v = 0.f;
   for (int k = 0; k < K; ++k) {
-    float bv = -INFINITY;
-    int be = 0x7FFFFFFF;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
-        bv = v[i];
-        be = e;
-      }
-    }
-    const uint32_t kb = key(bv);
-    const uint32_t km = __reduce_max_sync(0xffffffffu, kb);
-    be = static_cast<int>(__reduce_min_sync(0xffffffffu, kb == km ? static_cast<uint32_t>(be) : 0xFFFFFFFFu));
-    bv = __uint_as_float((km & 0x80000000u) ? (km & 0x7FFFFFFFu) : ~km);
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    const uint32_t km = __reduce_max_sync(0xffffffffu, ck[0]);
+    const unsigned holders = __ballot_sync(0xffffffffu, ck[0] == km);
+    int wl;
+    if (holders & (holders - 1u))  // equal values in several lanes (uniform branch)
+      wl = static_cast<int>(__reduce_min_sync(0xffffffffu, ck[0] == km ? static_cast<uint32_t>(ce[0]) : 0xFFFFFFFFu)) & 31;
+    else
+      wl = __ffs(holders) - 1;
+    const int be = __shfl_sync(0xffffffffu, ce[0], wl);
     if (lane == k) {
       my_e = be;
-      my_v = bv;
+      my_v = __uint_as_float((km & 0x80000000u) ? (km & 0x7FFFFFFFu) : ~km);
     }
+    const bool w = lane == wl;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) {
+      ck[i] = w ? ck[i + 1] : ck[i];
+      ce[i] = w ? ce[i + 1] : ce[i];
+    }
+    ck[7] = w ? 0u : ck[7];
   }
   float ev, denom;
   if (rc.gating == MOE_GATING_SIGMOID) {
