@@ -48,6 +48,47 @@ __device__ __forceinline__ void raw_decode(const Raw8<__nv_bfloat16>& r, float (
   }
 }
 
+// An order-preserving 32-bit key of a non-NaN float (a > b as floats iff key(a) > key(b); -0 and +0 share
+// the key of +0; -inf is 0x007FFFFF, so key 0 stays below every value), and the value of a key.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Routing weights of one token, by one warp: lane k < K holds the k-th selected expert my_e and its biased
+// logit my_v; v[i] are the lane's biased logits of experts lane + 32 i (NaN as -inf; used by the softmax
+// over all E experts), m their maximum.  Softmax or sigmoid gate values, renormalised over the K selected
+// when asked; lane k writes ids[k] and wout[k].
+__device__ __forceinline__ void warp_weights(int my_e, float my_v, const float (&v)[8], float m, const RouteCfg& rc,
+                                             int32_t* __restrict__ ids, float* __restrict__ wout) {
+  const int lane = threadIdx.x & 31;
+  const int E = rc.E, K = rc.K;
+  float ev, denom;
+  if (rc.gating == MOE_GATING_SIGMOID) {
+    ev = (lane < K) ? 1.0f / (1.0f + expf(-my_v)) : 0.f;
+    denom = rc.renorm ? warp_sum(ev) : 1.0f;
+  } else {
+    ev = (lane < K) ? expf(my_v - m) : 0.f;
+    if (rc.renorm) {
+      denom = warp_sum(ev);
+    } else {
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) s += expf(v[i] - m);
+      denom = warp_sum(s);
+    }
+  }
+  const float inv = denom > 1e-20f ? 1.0f / denom : (rc.renorm ? 1.0f / K : 1.0f);
+  if (lane < K) {
+    ids[lane] = my_e;
+    wout[lane] = ev * inv;
+  }
+}
+
 // Top-K (+ renormalisation) of one token, by one warp, from the lane's biased
 // logits v[i] of experts e = lane + 32 i (NaN already mapped to -inf; entries
 // beyond E are -inf) and m, their maximum over the warp.  With n_groups > 1 the
@@ -103,16 +144,12 @@ __device__ __forceinline__ void warp_select(const float (&v)[8], float m, const 
   // redux); when one lane holds it that lane wins, else the lowest expert among the holders (a second
   // redux, only on equal values); the winner drops its first candidate.  The same selection as a pairwise
   // (value, lower index) maximum.
-  auto key = [](float f) {
-    const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  };
   uint32_t ck[8];
   int ce[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     ce[i] = lane + 32 * i;
-    ck[i] = (ce[i] < E && !((taken >> i) & 1u)) ? key(v[i]) : 0u;
+    ck[i] = (ce[i] < E && !((taken >> i) & 1u)) ? order_key(v[i]) : 0u;
   }
   auto cas = [&](int i, int j) {  // the better of candidates i and j to i
     const bool sw = ck[j] > ck[i] || (ck[j] == ck[i] && ce[j] < ce[i]);
@@ -143,7 +180,7 @@ __device__ __forceinline__ void warp_select(const float (&v)[8], float m, const 
     const int be = __shfl_sync(0xffffffffu, ce[0], wl);
     if (lane == k) {
       my_e = be;
-      my_v = __uint_as_float((km & 0x80000000u) ? (km & 0x7FFFFFFFu) : ~km);
+      my_v = order_key_value(km);
     }
     const bool w = lane == wl;
 #pragma unroll
@@ -153,27 +190,7 @@ __device__ __forceinline__ void warp_select(const float (&v)[8], float m, const 
     }
     ck[7] = w ? 0u : ck[7];
   }
-  float ev, denom;
-  if (rc.gating == MOE_GATING_SIGMOID) {
-    ev = (lane < K) ? 1.0f / (1.0f + expf(-my_v)) : 0.f;
-    denom = rc.renorm ? warp_sum(ev) : 1.0f;
-  } else {
-    ev = (lane < K) ? expf(my_v - m) : 0.f;
-    if (rc.renorm) {
-      denom = warp_sum(ev);
-    } else {
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (lane + 32 * i < E) s += expf(v[i] - m);
-      denom = warp_sum(s);
-    }
-  }
-  const float inv = denom > 1e-20f ? 1.0f / denom : (rc.renorm ? 1.0f / K : 1.0f);
-  if (lane < K) {
-    ids[lane] = my_e;
-    wout[lane] = ev * inv;
-  }
+  warp_weights(my_e, my_v, v, m, rc, ids, wout);
 }
 
 // warp_select on the E raw logits of `row` (global or shared memory) plus the

@@ -32,6 +32,9 @@ CASES = {
     "long_rows_split_K": (spec(6, 4096, 8, 64, 2, dt="f32", shared=32), {}),
     "max_pairs_E256_K32": (spec(64, 128, 256, 32, 32, dt="f32"), {}),
     "skew_all_to_two": (spec(48, 256, 8, 64, 2, dt="f32"), dict(skew=True)),
+    # one token: the CTA-wide ranking; logits = bias exactly (zero router), five values over 64 experts
+    "T1_tied_logits": (spec(1, 256, 64, 64, 8, dt="f32"), dict(ties=True)),
+    "T1_tied_logits_no_renorm_E256": (spec(1, 256, 256, 32, 8, dt="f32", renorm=False), dict(ties=True)),
 }
 
 
@@ -41,6 +44,8 @@ def _workload(s, opt, seed):
         bias = np.linspace(2, -2, s.E)
     if opt.get("skew"):
         bias = np.array([50.0, 40.0] + [0.0] * (s.E - 2))
+    if opt.get("ties"):
+        return make(s, seed=seed, bias_values=[float((e * 7) % 5) for e in range(s.E)], router_std=0.0)
     return make(s, seed=seed, bias_values=bias)
 
 
@@ -104,6 +109,10 @@ def test_fused_matches_steps_and_oracle(case):
     assert torch.equal(_bits(rt_f["topk_ids"]), _bits(gids.reshape(-1)))
     assert torch.equal(_bits(rt_f["logits"]), _bits(logits.reshape(-1)))
     assert torch.equal(_bits(rt_f["topk_w"]), _bits(gw.reshape(-1)))
+    if opt.get("ties"):  # logits equal the bias: the K largest, the lower expert first among equal values
+        b = np.array([float((e * 7) % 5) for e in range(s.E)])
+        want = sorted(range(s.E), key=lambda e: (-b[e], e))[: s.K]
+        assert rt_f["topk_ids"].cpu().numpy().tolist() == want
     # the permutation is the stable counting sort of the ids
     ids = rt_f["topk_ids"].cpu().numpy()
     order = np.argsort(ids, kind="stable")
