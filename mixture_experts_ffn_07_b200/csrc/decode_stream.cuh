@@ -462,10 +462,9 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
       };
       int item = static_cast<int>(blockIdx.x) * batch;
       int end = min(total, item + batch);
-      // the batches after this one, claimed two ahead so that the counter's answer is there when needed
-      // (claims of one CTA only grow: a claim past the end ends its stream)
+      // the batch after this one, claimed when this one starts, so that the counter's answer is there when
+      // needed (claims of one CTA only grow: a claim past the end ends its stream)
       int next = item < end ? claim() : total;
-      int next2 = next < total ? claim() : total;
       const uint64_t pol = l2_policy_evict_first(), apol = l2_policy_evict_last();
       const int kshift = (p.K & (p.K - 1)) == 0 ? __ffs(p.K) - 1 : -1;  // pair -> token without a division
       unsigned gdone[(kMaxGroups + 31) / 32];  // groups whose gate/up items are all finished (known here)
@@ -511,9 +510,8 @@ __device__ __forceinline__ bool run_stream(const Maps& maps, const Params& p, co
         if (!have || kc >= m.nkc) {  // the next item, from this batch or the next
           if (have && ++item >= end) {
             item = next;
-            next = next2;
             end = min(total, item + batch);
-            if (next2 < total) next2 = claim();
+            next = item < total ? claim() : total;
           }
           const int hint = have ? m.g : 0;
           have = true;
